@@ -1,0 +1,297 @@
+/*
+ * moesq.h -- C ABI of the paired-4:8 sparse NVFP4 MoE expert library (sm_100a).
+ *
+ * The library runs the routed-expert MLP of a Mixture-of-Experts layer whose
+ * expert weights are NVFP4 (E2M1) with paired-4:8 structured sparsity along K,
+ * an FP8-E4M3 block scale per 32 dense K elements and an FP32 per-tensor global
+ * scale, kept in "pair-bitmask" storage; activations are NVFP4 with dynamic
+ * per-32 group scales and a static FP32 global per expert linear.  Sources:
+ *   [storage]  "Sparse storage layout (paired48_sparse, pair-bitmask v1)",
+ *              Qwen3.5-397B-A17B-P48NVFP4-MoESQ model card;
+ *   [format]   "Compression details" table, same card;
+ *   [kernel]   header list of the same card (paired-4:8 sparse NVFP4 grouped
+ *              GEMM, SM100) and the MoESQ repository README ("Kernels");
+ *   [fold]     gate/up global-scale note of the Qwen3.8-Flash-Next- and
+ *              Qwen3-30B-A3B-P48NVFP4-MoESQ model cards;
+ *   [export]   MoESQ repository README, "Usage" (Output bullet).
+ *
+ * Conventions common to every call
+ *  - Pointers named d_* or documented as "device" are CUDA device pointers; the
+ *    caller owns every buffer.  No call allocates, frees or synchronises, except
+ *    moesq_moe_forward_host (host buffers, documented there).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream);
+ *    work is enqueued asynchronously on it.
+ *  - Row-major, K innermost.  A packed NVFP4 byte holds element 2i in its low
+ *    nibble and element 2i+1 in its high nibble.  bf16 tensors are passed as
+ *    uint16_t bit patterns.
+ *  - Argument errors (null pointers, bad sizes, misalignment, too-small
+ *    workspace) are returned synchronously and nothing is enqueued.
+ *    Data-dependent errors found on the device (bad mask nibble, expert id out
+ *    of range, a bounded wait that gave up) are OR-ed as MOESQ_DFLAG_* bits into
+ *    the caller's int32 word `d_status` (device memory, may be NULL to ignore);
+ *    the caller reads it when it chooses.  A flagged call still writes only
+ *    inside its output buffers.
+ *  - Every device pointer must be 16-byte aligned.
+ *
+ * Arithmetic readings (the pages name the formats, not the arithmetic):
+ *  - NVFP4 quantisation of a group of 32 values x with global g (weights and
+ *    activations alike), every step IEEE binary32 round-to-nearest-even:
+ *        amax = max|x|;  s = amax / (6*g) (s = 0 if 6*g == 0);
+ *        sc = E4M3(s), nearest-even, saturating at 448;
+ *        sdq = value(sc) * g;  if sdq == 0 all codes are 0x0, else
+ *        inv = 1/sdq and code = E2M1(x * inv): nearest of {0,.5,1,1.5,2,3,4,6},
+ *        ties to the even code, |v| > 6 -> 6, sign bit = sign of the input.
+ *  - Weight global g_w = amax|W_pruned| / (6*448), the multiplier convention.
+ *  - Gate/up fold [fold]: the kernel applies the gate global to the fused
+ *    gate_up weight; each up block scale sc becomes E4M3(value(sc) * (g_up /
+ *    g_gate)) (nearest-even, saturating).
+ *  - SwiGLU: h = silu(gate) * up, silu(x) = x / (1 + exp(-x)), gate = rows
+ *    [0, I) of the fused [2I, K] weight, up = rows [I, 2I).
+ *  - Combine: out[t] = sum_j w[t,j] * y[slot(t,j)], float32 in j order (one
+ *    rounding per product and per sum), then bf16 nearest-even.
+ */
+#ifndef MOESQ_H
+#define MOESQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum moesq_status {
+  MOESQ_OK = 0,
+  MOESQ_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad enum, misaligned pointer */
+  MOESQ_ERR_UNSUPPORTED_SHAPE = 2, /* a size outside what the kernels support (see each call) */
+  MOESQ_ERR_BAD_SPARSITY = 3,      /* host-visible sparsity violation (moesq_*_host helpers only) */
+  MOESQ_ERR_CUDA = 4,              /* a CUDA runtime/driver call failed (launch, tensor map) */
+  MOESQ_ERR_TIMEOUT = 5,           /* reserved for callers that translate MOESQ_DFLAG_TIMEOUT */
+  MOESQ_ERR_WORKSPACE = 6,         /* workspace pointer NULL or smaller than required */
+  MOESQ_ERR_DEVICE = 7             /* current device is not sm_100 */
+} moesq_status;
+
+/* bits OR-ed into *d_status by the device */
+#define MOESQ_DFLAG_BAD_SPARSITY 0x1 /* a mask nibble without exactly 2 bits set, or
+                                        a dense chunk with more than 2 nonzero bytes */
+#define MOESQ_DFLAG_BAD_EXPERT 0x2   /* a top-k expert id outside [0, E) */
+#define MOESQ_DFLAG_TIMEOUT 0x4      /* a bounded pipeline wait gave up; outputs are garbage */
+#define MOESQ_DFLAG_CAPACITY 0x8     /* routed rows exceed the capacity passed by the caller */
+
+typedef void* moesq_stream_t; /* a cudaStream_t */
+
+/* Human-readable text of a status code (static storage). */
+const char* moesq_status_string(int status);
+
+/* ABI version of this header (incremented on any incompatible change). */
+int moesq_abi_version(void);
+
+/* ------------------------------------------------------------------------- *
+ * Storage codecs  [storage], [export]
+ * ------------------------------------------------------------------------- */
+
+/* Pair-bitmask -> dense packed NVFP4.
+ *   packed  device u8 [rows, K/4]   weight_sparse_packed (2 kept bytes of every 4, K order)
+ *   mask    device u8 [rows, K/16]  weight_sparse_mask (bit i = byte i kept, low nibble = lower-K chunk)
+ *   dense   device u8 [rows, K/2]   output: kept bytes in place, pruned bytes 0
+ * K % 64 == 0.  A nibble without exactly 2 bits set raises MOESQ_DFLAG_BAD_SPARSITY
+ * and its chunk is written as zeros.  Lossless: encode(decode(p, m), m) == (p, m). */
+moesq_status moesq_decode(const uint8_t* packed, const uint8_t* mask, uint8_t* dense,
+                          int64_t rows, int64_t K, int32_t* d_status, moesq_stream_t stream);
+
+/* Dense packed NVFP4 -> pair-bitmask.
+ *   dense     device u8 [rows, K/2]
+ *   mask_hint device u8 [rows, K/16] or NULL.  With a hint the hinted bytes are kept
+ *             (nonzero bytes outside it raise MOESQ_DFLAG_BAD_SPARSITY); without it
+ *             the nonzero bytes are kept and each chunk is filled up to 2 with its
+ *             lowest-index zero bytes (more than 2 nonzero bytes raises the flag).
+ *   packed    device u8 [rows, K/4] output;  mask device u8 [rows, K/16] output
+ *             (may alias mask_hint).
+ * K % 64 == 0. */
+moesq_status moesq_encode(const uint8_t* dense, const uint8_t* mask_hint, uint8_t* packed,
+                          uint8_t* mask, int64_t rows, int64_t K, int32_t* d_status,
+                          moesq_stream_t stream);
+
+/* Export of bf16 expert weights to pair-bitmask NVFP4 storage (prune + quantise +
+ * encode), E experts at once.
+ *   w       device bf16 [E, out, K]
+ *   n_seg   1 or 2: rows [0,out) split into n_seg equal segments, each with its own
+ *           FP32 global (2 = fused gate_up with separate gate and up globals)
+ *   packed  device u8 [E, out, K/4];  mask device u8 [E, out, K/16];
+ *   scale   device u8 [E, out, K/32] (E4M3 codes);  g_w device f32 [E, n_seg]
+ *   ws      device workspace of moesq_quant_weight_workspace_size() bytes
+ * Pruning: each 8-element chunk keeps the 2 pairs with the largest a*a+b*b (fp32 on
+ * the bf16 values; ties to the lower pair).  Then the NVFP4 rule above with
+ * g_w = amax/(6*448) per segment.  K % 64 == 0, out % n_seg == 0. */
+moesq_status moesq_quant_weight(const uint16_t* w, int64_t E, int64_t out, int64_t K,
+                                int32_t n_seg, uint8_t* packed, uint8_t* mask, uint8_t* scale,
+                                float* g_w, void* ws, size_t ws_bytes, moesq_stream_t stream);
+moesq_status moesq_quant_weight_workspace_size(int64_t E, int32_t n_seg, size_t* bytes);
+
+/* ------------------------------------------------------------------------- *
+ * Load-time repack into the tensor-core operand layouts  [storage] ("at load
+ * time ... compresses it into the kernel's own layout"), [fold]
+ * ------------------------------------------------------------------------- */
+
+typedef enum moesq_linear_kind {
+  MOESQ_LINEAR_DOWN = 0,          /* plain linear [out, K] */
+  MOESQ_LINEAR_GATE_UP = 1,       /* fused [2I, K], gate rows first, one global (g_w[e]) */
+  MOESQ_LINEAR_GATE_UP_SPLIT = 2  /* fused [2I, K], globals g_w[2e] (gate), g_w[2e+1] (up): folded */
+} moesq_linear_kind;
+
+/* Bytes of the repacked metadata and block scales of ONE expert linear. */
+moesq_status moesq_repack_sizes(int64_t out, int64_t K, size_t* meta_bytes, size_t* sf_bytes);
+
+/* Mask + block scales -> tcgen05 sparse metadata and scale-factor blocks.
+ *   mask   device u8 [E, out, K/16];  scale device u8 [E, out, K/32];
+ *   g_w    device f32 [E] (DOWN, GATE_UP) or [E, 2] (GATE_UP_SPLIT)
+ *   meta   device u8 [E * meta_bytes]: per expert, per 128-row tile, per 256 dense
+ *          K: 128 rows x 16 bytes, row r at 16r; each chunk's nibble = i0 | i1<<2
+ *          (ascending kept byte positions), lower-K chunk in the low nibble
+ *   sf     device u8 [E * sf_bytes]: per expert, per tile, per 128 dense K a 512-byte
+ *          block, row r scale j at (r%32)*16 + (r/32)*4 + j
+ *   alpha_w device f32 [E]: the weight global the GEMM applies (gate global for gate_up)
+ * Tile row order: DOWN identity; GATE_UP tile t = gate rows 64t..64t+63 then up rows
+ * I+64t..I+64t+63.  The packed values are used as stored (no repack).
+ * out % 128 == 0, K % 128 == 0.  Bad nibbles raise MOESQ_DFLAG_BAD_SPARSITY. */
+moesq_status moesq_repack_meta(const uint8_t* mask, const uint8_t* scale, const float* g_w,
+                               int64_t E, int64_t out, int64_t K, int32_t kind, uint8_t* meta,
+                               uint8_t* sf, float* alpha_w, int32_t* d_status,
+                               moesq_stream_t stream);
+
+/* ------------------------------------------------------------------------- *
+ * Routing  ([kernel]: the grouped GEMM runs over the tokens routed to each expert)
+ * ------------------------------------------------------------------------- */
+
+/* Top-k routing -> per-expert contiguous slot groups, order (expert, token, j).
+ *   topk_ids      device i32 [T, k]
+ *   expert_offsets device i32 [E+1] output: exclusive scan of per-expert counts
+ *   pad_offsets   device i32 [E+1] output: same with each count rounded up to 128
+ *                 (row of expert e's first slot in the padded activation buffers)
+ *   slot_token    device i32 [T*k] output: token of each slot
+ *   token_slot    device i32 [T, k] output: slot of each (token, j)
+ *   ws            device workspace of moesq_permute_workspace_size() bytes
+ * Ids outside [0, E) raise MOESQ_DFLAG_BAD_EXPERT and are routed to expert 0.
+ * 1 <= E <= 4096, 1 <= k <= 32, T*k < 2^31. */
+moesq_status moesq_permute(const int32_t* topk_ids, int64_t T, int32_t k, int32_t E,
+                           int32_t* expert_offsets, int32_t* pad_offsets, int32_t* slot_token,
+                           int32_t* token_slot, void* ws, size_t ws_bytes, int32_t* d_status,
+                           moesq_stream_t stream);
+moesq_status moesq_permute_workspace_size(int64_t T, int32_t k, int32_t E, size_t* bytes);
+
+/* Upper bound of the padded row count for S slots over E experts. */
+int64_t moesq_padded_rows(int64_t S, int32_t E);
+
+/* Weighted combine: out[t] = bf16( sum_j w[t,j] * y[token_slot[t,j]] ), float32, j order.
+ *   y device bf16 [S, H];  token_slot device i32 [T, k];  topk_w device f32 [T, k];
+ *   out device bf16 [T, H].  H % 8 == 0. */
+moesq_status moesq_unpermute(const uint16_t* y, const int32_t* token_slot, const float* topk_w,
+                             int64_t T, int32_t k, int64_t H, uint16_t* out,
+                             moesq_stream_t stream);
+
+/* ------------------------------------------------------------------------- *
+ * Activation quantisation  [format] ("dynamic per-32 group scales, FP32
+ * per-tensor global scale stored per expert linear")
+ * ------------------------------------------------------------------------- */
+
+typedef enum moesq_sf_layout {
+  MOESQ_SF_LINEAR = 0, /* codes [rows, K/2], scales [rows, K/32], row = output row index */
+  MOESQ_SF_KERNEL = 1  /* padded GEMM operand: codes [P, K/2] at row p = pad_offsets[e] +
+                          (s - expert_offsets[e]); scales in 512-byte blocks
+                          [P/128][K/128][512], row r scale j at (r%32)*16+(r/32)*4+j */
+} moesq_sf_layout;
+
+/* bf16 -> NVFP4 codes + E4M3 per-32 scales, one output row per slot.
+ *   x              device bf16 [T, K]
+ *   gather         device i32 [rows] (row of x for each output row) or NULL (identity)
+ *   expert_offsets device i32 [E+1] or NULL (then every row uses g_in[0])
+ *   pad_offsets    device i32 [E+1], required for MOESQ_SF_KERNEL
+ *   g_in           device f32 [E] (or [1] without expert_offsets): input globals
+ *   codes, sf      device outputs in the chosen layout
+ * K % 128 == 0. */
+moesq_status moesq_quant_act(const uint16_t* x, int64_t K, const int32_t* gather,
+                             const int32_t* expert_offsets, const int32_t* pad_offsets,
+                             int32_t E, const float* g_in, int64_t rows, int32_t layout,
+                             uint8_t* codes, uint8_t* sf, moesq_stream_t stream);
+
+/* ------------------------------------------------------------------------- *
+ * Grouped sparse GEMM  [kernel]
+ * ------------------------------------------------------------------------- */
+
+typedef struct moesq_linear {
+  const uint8_t* packed; /* device u8 [E, out, K/4]  weight_sparse_packed, used as stored */
+  const uint8_t* meta;   /* device, moesq_repack_meta output */
+  const uint8_t* sf;     /* device, moesq_repack_meta output */
+  const float* alpha_w;  /* device f32 [E] */
+  int64_t out;           /* output features (2I for gate_up) */
+  int64_t K;             /* dense K */
+  int32_t E;             /* experts */
+  int32_t kind;          /* moesq_linear_kind (GATE_UP_SPLIT behaves as GATE_UP here) */
+} moesq_linear;
+
+typedef enum moesq_epilogue {
+  MOESQ_EPI_F32 = 0,         /* out f32 [S, W.out], row = slot, column = original weight row */
+  MOESQ_EPI_BF16 = 1,        /* out bf16 [S, W.out] */
+  MOESQ_EPI_SWIGLU_NVFP4 = 2 /* gate_up only: h = silu(gate)*up requantised with g_next[e]:
+                                out u8 codes [P, I/2] (padded rows), out_sf blocks
+                                [P/128][I/128][512] -- the next GEMM's B operand */
+} moesq_epilogue;
+
+/* y[s, m] = g_act[e] * alpha_w[e] * sum_k W_e[m, k] * A[s, k] for every slot s of expert e.
+ *   act_codes  device u8 [P_cap, K/2] padded rows (moesq_quant_act, MOESQ_SF_KERNEL)
+ *   act_sf     device u8 [P_cap/128][K/128][512]
+ *   g_act      device f32 [E]
+ *   expert_offsets, pad_offsets  device i32 [E+1] (moesq_permute)
+ *   S          number of slots (expert_offsets[E]); P_cap = padded row capacity of the
+ *              act/out buffers, >= moesq_padded_rows(S, E) and a multiple of 128
+ *   g_next     device f32 [E] (SWIGLU only, else NULL)
+ *   ws         device workspace of moesq_grouped_gemm_workspace_size() bytes (may be 0)
+ * Weights are the sparse operand A of tcgen05.mma.sp (M = weight rows), tokens are
+ * B (N).  out % 128 == 0, K % 128 == 0, out % 256 == 0 for SWIGLU.
+ * Bounded waits that give up raise MOESQ_DFLAG_TIMEOUT. */
+moesq_status moesq_grouped_gemm(const moesq_linear* W, const uint8_t* act_codes,
+                                const uint8_t* act_sf, const float* g_act,
+                                const int32_t* expert_offsets, const int32_t* pad_offsets,
+                                int64_t S, int64_t P_cap, int32_t epilogue, const float* g_next,
+                                void* out, uint8_t* out_sf, void* ws, size_t ws_bytes,
+                                int32_t* d_status, moesq_stream_t stream);
+moesq_status moesq_grouped_gemm_workspace_size(const moesq_linear* W, int64_t S, size_t* bytes);
+
+/* ------------------------------------------------------------------------- *
+ * The whole routed-expert MLP of one MoE layer
+ * ------------------------------------------------------------------------- */
+
+typedef struct moesq_moe_layer {
+  int32_t E, k;
+  int64_t H, I;
+  moesq_linear gate_up;      /* out = 2I, K = H, kind GATE_UP or GATE_UP_SPLIT (already folded) */
+  moesq_linear down;         /* out = H, K = I */
+  const float* g_in_gate_up; /* device f32 [E] static input globals of gate_up */
+  const float* g_in_down;    /* device f32 [E] static input globals of down */
+} moesq_moe_layer;
+
+/* permute -> quant_act -> gate_up (fused SwiGLU + NVFP4 requant) -> down -> combine.
+ *   x device bf16 [T, H];  topk_ids device i32 [T, k];  topk_w device f32 [T, k]
+ *   out device bf16 [T, H];  ws device workspace of moesq_moe_forward_workspace_size(). */
+moesq_status moesq_moe_forward(const moesq_moe_layer* L, const uint16_t* x,
+                               const int32_t* topk_ids, const float* topk_w, int64_t T,
+                               uint16_t* out, void* ws, size_t ws_bytes, int32_t* d_status,
+                               moesq_stream_t stream);
+moesq_status moesq_moe_forward_workspace_size(const moesq_moe_layer* L, int64_t T,
+                                              size_t* bytes);
+
+/* Same as moesq_moe_forward with HOST inputs and output: copies x/topk_ids/topk_w
+ * host->device into `ws` (which must also hold the forward workspace; see
+ * moesq_moe_forward_host_workspace_size), runs the layer, copies out back to the
+ * host buffer and synchronises `stream`.  Host buffers should be pinned for speed. */
+moesq_status moesq_moe_forward_host(const moesq_moe_layer* L, const uint16_t* h_x,
+                                    const int32_t* h_topk_ids, const float* h_topk_w,
+                                    int64_t T, uint16_t* h_out, void* ws, size_t ws_bytes,
+                                    int32_t* d_status, moesq_stream_t stream);
+moesq_status moesq_moe_forward_host_workspace_size(const moesq_moe_layer* L, int64_t T,
+                                                   size_t* bytes);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOESQ_H */

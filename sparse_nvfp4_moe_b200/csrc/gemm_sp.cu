@@ -1,0 +1,518 @@
+// Grouped paired-4:8 sparse NVFP4 GEMM on the sm_100a tensor cores.
+//
+// The pages' kernel is a "paired-4:8 sparse NVFP4 grouped GEMM" for SM100
+// (header list of the Qwen3.5-397B-A17B-P48NVFP4-MoESQ model card; "Kernels" of
+// the MoESQ repository README).  The scale group is 32 dense K because the
+// Blackwell sparse NVFP4 MMA takes one scale per 32 dense K = 16 kept values
+// ("Compression details", same card).  This kernel:
+//
+//   * puts the weights on the sparse operand A of tcgen05.mma.sp (M = 128
+//     weight rows per tile) and the routed tokens of one expert on B (N <= 128),
+//     so the compressed weight bytes are the streamed operand and the weight
+//     values are read exactly as stored (weight_sparse_packed is the compressed
+//     A operand: kept elements in K order);
+//   * is persistent: one CTA per SM walks a static list of (expert, token tile,
+//     weight tile) work items built on the device from the routing offsets, so
+//     empty experts cost nothing;
+//   * is warp-specialised: warp 0 issues TMA (values and tokens) and bulk copies
+//     (metadata, block scales) into a 6-stage shared-memory ring; warp 1 owns
+//     TMEM, copies metadata and scales smem->TMEM (tcgen05.cp) and issues the
+//     MMAs (dense K = 128 each, two per stage); warps 2..5 drain the
+//     double-buffered FP32 accumulators (tcgen05.ld) while the next tile runs;
+//   * fuses the epilogue: FP32 or bf16 output per slot, or SwiGLU followed by
+//     NVFP4 requantisation written straight into the next GEMM's B operand
+//     layout (codes + 512-byte scale blocks).
+//
+// Every mbarrier wait is bounded (2 s); on expiry the kernel flags
+// MOESQ_DFLAG_TIMEOUT, drains its own copies in flight, frees TMEM and exits.
+#include "common.cuh"
+
+#include <mutex>
+
+namespace moesq {
+namespace sp {
+
+constexpr int BM = 128;           // weight rows per tile
+constexpr int BN = 128;           // max tokens per tile
+constexpr int BK = 256;           // dense K per pipeline stage (two MMAs)
+constexpr int STAGES = 6;
+constexpr int A_BYTES = BM * BK / 4;       // compressed values: 64 B per row (SW64)
+constexpr int B_BYTES = BN * BK / 2;       // token codes: 128 B per row (SW128)
+constexpr int E_BYTES = BM * 16;           // metadata: 16 B per row
+constexpr int SF_BYTES = 2 * 512;          // two 512-byte scale blocks
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + E_BYTES + 2 * SF_BYTES;  // 28672
+constexpr int EPI_LD = 65;                 // floats per staged accumulator row (64 + pad)
+constexpr int EPI_BYTES = BM * EPI_LD * 4;
+constexpr int MAX_E = 1024;
+constexpr int THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TM_ACC = 0, TM_E = 256, TM_SFA = 264, TM_SFB = 272;
+
+struct Params {
+  const uint8_t* meta;
+  const uint8_t* sfw;
+  const float* alpha_w;
+  const uint8_t* act_sf;
+  const float* g_act;
+  const int32_t* expert_offsets;
+  const int32_t* pad_offsets;
+  const float* g_next;
+  void* out;
+  uint8_t* out_sf;
+  int32_t* d_status;
+  int E, M, K, epi, gate_up;
+  int64_t S, P_cap;
+};
+
+struct Smem {
+  uint64_t full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], done;
+  uint32_t tmem_base;
+  int abort;
+  int tile_start[MAX_E + 1];
+};
+
+constexpr size_t SMEM_BYTES = 1024 /*align*/ + (size_t)STAGES * STAGE_BYTES + EPI_BYTES + sizeof(Smem);
+
+__device__ __forceinline__ uint32_t make_idesc(uint32_t n) {
+  return (1u << 2)            // sparse
+         | (1u << 7)          // A: E2M1
+         | (1u << 10)         // B: E2M1
+         | ((n >> 3) << 17)   // N
+         | (0u << 23)         // scale factors UE4M3
+         | ((uint32_t)(BM >> 4) << 24);
+}
+
+struct Tile {
+  int e, nt, mt, n_rows;
+};
+
+__device__ __forceinline__ Tile decode_tile(const Smem& s, int id, int MT, int E,
+                                            const int32_t* __restrict__ off) {
+  Tile t;
+  const int q = id / MT;
+  t.mt = id % MT;
+  int lo = 0, hi = E - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s.tile_start[mid] <= q) lo = mid;
+    else hi = mid - 1;
+  }
+  t.e = lo;
+  t.nt = q - s.tile_start[lo];
+  const int te = off[lo + 1] - off[lo];
+  const int r = te - t.nt * BN;
+  t.n_rows = r < BN ? r : BN;
+  return t;
+}
+
+// bounded wait used only while draining at exit: ignores the abort flag
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > 200000000ull) return;
+  }
+}
+
+__device__ __forceinline__ float silu(float x) { return x / (1.0f + expf(-x)); }
+
+__global__ void __launch_bounds__(THREADS, 1)
+    k_grouped_gemm_sp(const __grid_constant__ CUtensorMap tmap_a,
+                      const __grid_constant__ CUtensorMap tmap_b, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  float* epi = (float*)(smem + STAGES * STAGE_BYTES);
+  Smem& S = *(Smem*)(smem + STAGES * STAGE_BYTES + EPI_BYTES);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int E = p.E, MT = p.M / BM;
+  const int nkb = (p.K + BK - 1) / BK, kb128 = p.K / 128;
+  const int32_t* off = p.expert_offsets;
+
+  // ---- set-up: barriers, tile prefix, TMEM
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&S.full[i], 1);
+      mbar_init(&S.empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&S.acc_full[i], 1);
+      mbar_init(&S.acc_empty[i], 4);
+    }
+    mbar_init(&S.done, 1);
+    S.abort = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmap_a);
+    tma_prefetch_desc(&tmap_b);
+  }
+  if (warp == 0) {  // tile_start[e] = sum over e' < e of ceil(T_e' / BN)
+    int run = 0;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+      const int e = e0 + lane;
+      int v = 0;
+      if (e < E) v = (off[e + 1] - off[e] + BN - 1) / BN;
+      int x = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (e < E) S.tile_start[e] = run + x - v;
+      run += __shfl_sync(0xffffffffu, x, 31);
+    }
+    if (lane == 0) S.tile_start[E] = run;
+  }
+  if (warp == 1) {
+    tmem_alloc(&S.tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+  const int total = S.tile_start[E] * MT;
+  volatile int* abort = &S.abort;
+
+  if (warp == 0) {
+    // ================================================================ producer
+    if (elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      long fills = 0;
+      for (int id = blockIdx.x; id < total; id += gridDim.x) {
+        const Tile t = decode_tile(S, id, MT, E, off);
+        int r0, r1;
+        if (p.gate_up) {
+          r0 = t.e * p.M + 64 * t.mt;
+          r1 = t.e * p.M + p.M / 2 + 64 * t.mt;
+        } else {
+          r0 = t.e * p.M + BM * t.mt;
+          r1 = r0 + 64;
+        }
+        int prow = p.pad_offsets[t.e] + t.nt * BN;
+        if (prow < 0 || (int64_t)prow + BN > p.P_cap) {  // inconsistent offsets: stay in bounds
+          flag(p.d_status, MOESQ_DFLAG_CAPACITY);
+          prow = 0;
+        }
+        const uint8_t* meta = p.meta + (size_t)(t.e * MT + t.mt) * nkb * 2048;
+        const uint8_t* sfa = p.sfw + (size_t)(t.e * MT + t.mt) * kb128 * 512;
+        const uint8_t* sfb = p.act_sf + (size_t)(prow / 128) * kb128 * 512;
+        for (int kb = 0; kb < nkb; ++kb) {
+          mbar_wait(&S.empty[stage], phase ^ 1, abort, p.d_status);
+          const int nk = (kb128 - 2 * kb) >= 2 ? 2 : 1;
+          uint8_t* st = smem + stage * STAGE_BYTES;
+          mbar_arrive_expect_tx(&S.full[stage],
+                                A_BYTES + B_BYTES + E_BYTES + 2 * nk * 512);
+          tma_load_2d(st, &tmap_a, kb * 64, r0, &S.full[stage]);
+          tma_load_2d(st + A_BYTES / 2, &tmap_a, kb * 64, r1, &S.full[stage]);
+          tma_load_2d(st + A_BYTES, &tmap_b, kb * 128, prow, &S.full[stage]);
+          bulk_load(st + A_BYTES + B_BYTES, meta + (size_t)kb * 2048, E_BYTES, &S.full[stage]);
+          bulk_load(st + A_BYTES + B_BYTES + E_BYTES, sfa + (size_t)kb * 1024, nk * 512,
+                    &S.full[stage]);
+          bulk_load(st + A_BYTES + B_BYTES + E_BYTES + SF_BYTES, sfb + (size_t)kb * 1024,
+                    nk * 512, &S.full[stage]);
+          ++fills;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      // drain: every slot's last fill must have landed before the CTA exits
+      for (int s = 0; s < STAGES; ++s) {
+        if (fills > s) {
+          const long u = s + (long)STAGES * ((fills - 1 - s) / STAGES);
+          drain_wait(&S.full[s], (uint32_t)((u / STAGES) & 1));
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ================================================================ MMA issuer
+    if (elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t acc_phase[2] = {0u, 0u};
+      int buf = 0;
+      for (int id = blockIdx.x; id < total; id += gridDim.x) {
+        const Tile t = decode_tile(S, id, MT, E, off);
+        int n_mma = (t.n_rows + 15) / 16 * 16;
+        if (n_mma < 16) n_mma = 16;
+        const uint32_t idesc = make_idesc((uint32_t)n_mma);
+        const uint32_t d_tmem = tmem + TM_ACC + buf * BN;
+        mbar_wait(&S.acc_empty[buf], acc_phase[buf] ^ 1, abort, p.d_status);
+        tc_fence_after();
+        for (int kb = 0; kb < nkb; ++kb) {
+          mbar_wait(&S.full[stage], phase, abort, p.d_status);
+          tc_fence_after();
+          const int nk = (kb128 - 2 * kb) >= 2 ? 2 : 1;
+          const uint32_t st = smem_u32(smem + stage * STAGE_BYTES);
+          const uint32_t sA = st, sB = st + A_BYTES, sE = sB + B_BYTES, sSFA = sE + E_BYTES,
+                         sSFB = sSFA + SF_BYTES;
+          tc_cp_128x128b(tmem + TM_E, smem_desc(sE, 16, 128, SWZ_NONE));
+          for (int kk = 0; kk < nk; ++kk) {
+            tc_cp_32x128b_warpx4(tmem + TM_SFA + 4 * kk, smem_desc(sSFA + 512 * kk, 16, 128, SWZ_NONE));
+            tc_cp_32x128b_warpx4(tmem + TM_SFB + 4 * kk, smem_desc(sSFB + 512 * kk, 16, 128, SWZ_NONE));
+          }
+          for (int kk = 0; kk < nk; ++kk) {
+            const uint64_t adesc = smem_desc(sA + 32 * kk, 16, 512, SWZ_64B);
+            const uint64_t bdesc = smem_desc(sB + 64 * kk, 16, 1024, SWZ_128B);
+            tc_mma_sp_nvf4(d_tmem, adesc, bdesc, tmem + TM_E + 2 * kk, idesc,
+                           tmem + TM_SFA + 4 * kk, tmem + TM_SFB + 4 * kk,
+                           (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(&S.empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        tc_commit(&S.acc_full[buf]);
+        acc_phase[buf] ^= 1;
+        buf ^= 1;
+      }
+      // drain: all tensor-core work of this CTA complete before TMEM is freed
+      tc_commit(&S.done);
+      drain_wait(&S.done, 0);
+    }
+    __syncwarp();
+  } else {
+    // ================================================================ epilogue
+    const int q = warp & 3;            // TMEM lane quarter this warp may access
+    const int et = threadIdx.x - 64;   // 0..127
+    uint32_t acc_phase[2] = {0u, 0u};
+    int buf = 0;
+    const int I = p.M / 2;
+    for (int id = blockIdx.x; id < total; id += gridDim.x) {
+      const Tile t = decode_tile(S, id, MT, E, off);
+      const float alpha = __fmul_rn(p.g_act[t.e], p.alpha_w[t.e]);
+      mbar_wait(&S.acc_full[buf], acc_phase[buf], abort, p.d_status);
+      tc_fence_after();
+      for (int c0 = 0; c0 < t.n_rows; c0 += 64) {
+        // phase 1: this warp's 32 accumulator rows, 64 token columns -> smem (x alpha)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tmem + TM_ACC + buf * BN + c0 + 32 * h + ((uint32_t)(32 * q) << 16), r);
+          tmem_ld_wait();
+          float* row = epi + (32 * q + lane) * EPI_LD + 32 * h;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) row[j] = __fmul_rn(__uint_as_float(r[j]), alpha);
+        }
+        if (c0 + 64 >= t.n_rows) {  // accumulator fully read: hand it back to the MMA warp
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S.acc_empty[buf]);
+        }
+        named_bar_sync(1, 128);
+        // phase 2: one token column per thread
+        const int j = et & 63, half = et >> 6;
+        const int n = t.nt * BN + c0 + j;
+        if (c0 + j < t.n_rows) {
+          if (p.epi == MOESQ_EPI_SWIGLU_NVFP4) {
+            float h[32];
+            float amax = 0.0f;
+#pragma unroll
+            for (int f = 0; f < 32; ++f) {
+              const float gv = epi[(32 * half + f) * EPI_LD + j];
+              const float uv = epi[(64 + 32 * half + f) * EPI_LD + j];
+              h[f] = __fmul_rn(silu(gv), uv);
+              amax = fmaxf(amax, fabsf(h[f]));
+            }
+            const GroupScale gs = nvfp4_group_scale(amax, p.g_next[t.e]);
+            uint32_t o[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              uint32_t word = 0;
+#pragma unroll
+              for (int u = 0; u < 8; ++u) word |= nvfp4_code(h[8 * c + u], gs.inv) << (4 * u);
+              o[c] = word;
+            }
+            const int64_t prow = (int64_t)p.pad_offsets[t.e] + n;
+            const int fb = 64 * t.mt + 32 * half;  // first feature of this group
+            if (prow >= 0 && prow < p.P_cap) {
+              uint8_t* codes = (uint8_t*)p.out;
+              *reinterpret_cast<uint4*>(codes + prow * (I / 2) + fb / 2) = make_uint4(o[0], o[1], o[2], o[3]);
+              const int64_t blk = (prow / 128) * (I / 128) + fb / 128;
+              p.out_sf[blk * 512 + sf_block_offset((uint32_t)(prow % 128), (uint32_t)((fb / 32) % 4))] =
+                  (uint8_t)gs.sc;
+            }
+          } else {
+            const int64_t s = (int64_t)off[t.e] + n;
+            int col0;  // first output column of this thread's 64 rows
+            if (p.gate_up) col0 = half == 0 ? 64 * t.mt : I + 64 * t.mt;
+            else col0 = BM * t.mt + 64 * half;
+            const float* src = epi + (64 * half) * EPI_LD + j;
+            if (s < 0 || s >= p.S) {
+              // inconsistent offsets: write nothing outside the output
+            } else if (p.epi == MOESQ_EPI_F32) {
+              float* y = (float*)p.out + s * p.M + col0;
+#pragma unroll
+              for (int c = 0; c < 16; ++c)
+                *reinterpret_cast<float4*>(y + 4 * c) =
+                    make_float4(src[(4 * c) * EPI_LD], src[(4 * c + 1) * EPI_LD],
+                                src[(4 * c + 2) * EPI_LD], src[(4 * c + 3) * EPI_LD]);
+            } else {
+              uint16_t* y = (uint16_t*)p.out + s * p.M + col0;
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                uint32_t w[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                  w[u] = float_to_bf16_bits(src[(8 * c + 2 * u) * EPI_LD]) |
+                         (float_to_bf16_bits(src[(8 * c + 2 * u + 1) * EPI_LD]) << 16);
+                *reinterpret_cast<uint4*>(y + 8 * c) = make_uint4(w[0], w[1], w[2], w[3]);
+              }
+            }
+          }
+        }
+        named_bar_sync(1, 128);
+      }
+      if (t.n_rows <= 0) {  // cannot happen for listed tiles; keep the handshake balanced
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.acc_empty[buf]);
+      }
+      acc_phase[buf] ^= 1;
+      buf ^= 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace sp
+
+// ------------------------------------------------------------------- host ---
+typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                     const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                     const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                     CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static PFN_encodeTiled get_encode_fn() {
+  static PFN_encodeTiled fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (PFN_encodeTiled)ptr;
+  });
+  return fn;
+}
+
+static bool make_tmap_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                         uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swz) {
+  PFN_encodeTiled enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static int device_sms(int* dev_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  int sms = 0, major = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return -1;
+  if (dev_out) *dev_out = dev;
+  return major == 10 ? sms : 0;
+}
+
+}  // namespace moesq
+
+using namespace moesq;
+
+extern "C" moesq_status moesq_grouped_gemm_workspace_size(const moesq_linear* W, int64_t S,
+                                                          size_t* bytes) {
+  MOESQ_REQUIRE(W && bytes && S >= 0, MOESQ_ERR_INVALID_ARG);
+  *bytes = 0;
+  return MOESQ_OK;
+}
+
+extern "C" moesq_status moesq_grouped_gemm(const moesq_linear* W, const uint8_t* act_codes,
+                                           const uint8_t* act_sf, const float* g_act,
+                                           const int32_t* expert_offsets,
+                                           const int32_t* pad_offsets, int64_t S, int64_t P_cap,
+                                           int32_t epilogue, const float* g_next, void* out,
+                                           uint8_t* out_sf, void* ws, size_t ws_bytes,
+                                           int32_t* d_status, moesq_stream_t stream) {
+  (void)ws;
+  (void)ws_bytes;
+  MOESQ_REQUIRE(W, MOESQ_ERR_INVALID_ARG);
+  MOESQ_REQUIRE(W->packed && W->meta && W->sf && W->alpha_w, MOESQ_ERR_INVALID_ARG);
+  MOESQ_REQUIRE(act_codes && act_sf && g_act && expert_offsets && pad_offsets && out,
+                MOESQ_ERR_INVALID_ARG);
+  MOESQ_REQUIRE(epilogue >= MOESQ_EPI_F32 && epilogue <= MOESQ_EPI_SWIGLU_NVFP4,
+                MOESQ_ERR_INVALID_ARG);
+  MOESQ_REQUIRE(W->E >= 1 && W->E <= sp::MAX_E && W->out > 0 && W->K > 0 && S >= 0 && P_cap >= 0,
+                MOESQ_ERR_INVALID_ARG);
+  MOESQ_REQUIRE(W->out % 128 == 0 && W->K % 128 == 0 && P_cap % 128 == 0,
+                MOESQ_ERR_UNSUPPORTED_SHAPE);
+  MOESQ_REQUIRE(W->out * (int64_t)W->E < (1ll << 31) && W->K < (1 << 20), MOESQ_ERR_UNSUPPORTED_SHAPE);
+  MOESQ_REQUIRE(P_cap >= moesq_padded_rows(S, W->E) && P_cap < (1ll << 31),
+                MOESQ_ERR_UNSUPPORTED_SHAPE);
+  const bool gate_up = W->kind != MOESQ_LINEAR_DOWN;
+  if (epilogue == MOESQ_EPI_SWIGLU_NVFP4) {
+    MOESQ_REQUIRE(gate_up && g_next && out_sf, MOESQ_ERR_INVALID_ARG);
+    MOESQ_REQUIRE(W->out % 256 == 0, MOESQ_ERR_UNSUPPORTED_SHAPE);
+  }
+  if (gate_up) MOESQ_REQUIRE(W->out % 256 == 0, MOESQ_ERR_UNSUPPORTED_SHAPE);
+  MOESQ_REQUIRE(moesq_aligned16(W->packed) && moesq_aligned16(W->meta) && moesq_aligned16(W->sf) &&
+                    moesq_aligned16(act_codes) && moesq_aligned16(act_sf) && moesq_aligned16(out) &&
+                    moesq_aligned16(out_sf),
+                MOESQ_ERR_INVALID_ARG);
+  if (S == 0) return MOESQ_OK;
+  int dev = 0;
+  const int sms = device_sms(&dev);
+  if (sms < 0) return MOESQ_ERR_CUDA;
+  if (sms == 0) return MOESQ_ERR_DEVICE;
+
+  CUtensorMap ta, tb;
+  if (!make_tmap_u8(&ta, W->packed, (uint64_t)(W->K / 4), (uint64_t)(W->E * W->out), 64, 64,
+                    CU_TENSOR_MAP_SWIZZLE_64B))
+    return MOESQ_ERR_CUDA;
+  if (!make_tmap_u8(&tb, act_codes, (uint64_t)(W->K / 2), (uint64_t)P_cap, 128, 128,
+                    CU_TENSOR_MAP_SWIZZLE_128B))
+    return MOESQ_ERR_CUDA;
+
+  static int attr_done[64] = {0};
+  if (dev < 64 && !attr_done[dev]) {
+    if (cudaFuncSetAttribute(sp::k_grouped_gemm_sp, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sp::SMEM_BYTES) != cudaSuccess)
+      return MOESQ_ERR_CUDA;
+    attr_done[dev] = 1;
+  }
+  sp::Params prm;
+  prm.meta = W->meta;
+  prm.sfw = W->sf;
+  prm.alpha_w = W->alpha_w;
+  prm.act_sf = act_sf;
+  prm.g_act = g_act;
+  prm.expert_offsets = expert_offsets;
+  prm.pad_offsets = pad_offsets;
+  prm.g_next = g_next;
+  prm.out = out;
+  prm.out_sf = out_sf;
+  prm.d_status = d_status;
+  prm.E = W->E;
+  prm.M = (int)W->out;
+  prm.K = (int)W->K;
+  prm.epi = epilogue;
+  prm.gate_up = gate_up ? 1 : 0;
+  prm.S = S;
+  prm.P_cap = P_cap;
+  sp::k_grouped_gemm_sp<<<sms, sp::THREADS, sp::SMEM_BYTES, (cudaStream_t)stream>>>(ta, tb, prm);
+  MOESQ_CHECK_LAUNCH();
+  return MOESQ_OK;
+}

@@ -1,0 +1,99 @@
+// Dynamic NVFP4 activation quantisation (bf16 -> E2M1 codes + E4M3 per-32 scales).
+//
+// "Activations: NVFP4, dynamic per-32 group scales, FP32 per-tensor global scale
+// stored per expert linear" ("Compression details" table, Qwen3.5-397B-A17B-
+// P48NVFP4-MoESQ model card).  One output row per routed slot: the row of x of
+// its token is gathered and quantised with the input global of its expert.  One
+// thread per 32-element group: 64 bytes of bf16 in (4 x 16-byte loads, a warp
+// reads 2 KB contiguous), 16 bytes of codes and one scale byte out.  In the
+// KERNEL layout rows land in the padded, 128-row aligned GEMM operand buffer
+// and scales in the 512-byte tensor-core scale-factor blocks.
+#include "common.cuh"
+
+namespace moesq {
+
+__device__ __forceinline__ int find_expert(const int32_t* __restrict__ off, int E, int64_t s) {
+  int lo = 0, hi = E - 1;  // largest e with off[e] <= s
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (off[mid] <= s) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+__global__ void k_quant_act(const uint16_t* __restrict__ x, int64_t K, const int32_t* __restrict__ gather,
+                            const int32_t* __restrict__ expert_offsets,
+                            const int32_t* __restrict__ pad_offsets, int E,
+                            const float* __restrict__ g_in, int64_t rows, int layout,
+                            uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+  const int64_t G = K / 32;
+  const int64_t n = rows * G;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t s = i / G, grp = i % G;
+    const int64_t src = gather ? (int64_t)gather[s] : s;
+    int e = 0;
+    if (expert_offsets) e = find_expert(expert_offsets, E, s);
+    const float g = g_in[e];
+    float v[32];
+    const uint4* q = reinterpret_cast<const uint4*>(x + src * K + 32 * grp);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint4 u = q[c];
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        v[8 * c + 2 * j] = bf16_bits_to_float(w[j] & 0xFFFF);
+        v[8 * c + 2 * j + 1] = bf16_bits_to_float(w[j] >> 16);
+      }
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(v[j]));
+    const GroupScale gs = nvfp4_group_scale(amax, g);
+    uint32_t o[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) word |= nvfp4_code(v[8 * c + j], gs.inv) << (4 * j);
+      o[c] = word;
+    }
+    int64_t row = s;
+    if (layout == MOESQ_SF_KERNEL) row = (int64_t)pad_offsets[e] + (s - expert_offsets[e]);
+    *reinterpret_cast<uint4*>(codes + row * (K / 2) + 16 * grp) = make_uint4(o[0], o[1], o[2], o[3]);
+    if (layout == MOESQ_SF_KERNEL) {
+      const int64_t blk = (row / 128) * (K / 128) + grp / 4;
+      sf[blk * 512 + sf_block_offset((uint32_t)(row % 128), (uint32_t)(grp % 4))] = (uint8_t)gs.sc;
+    } else {
+      sf[s * G + grp] = (uint8_t)gs.sc;
+    }
+  }
+}
+
+}  // namespace moesq
+
+using namespace moesq;
+
+extern "C" moesq_status moesq_quant_act(const uint16_t* x, int64_t K, const int32_t* gather,
+                                        const int32_t* expert_offsets, const int32_t* pad_offsets,
+                                        int32_t E, const float* g_in, int64_t rows, int32_t layout,
+                                        uint8_t* codes, uint8_t* sf, moesq_stream_t stream) {
+  MOESQ_REQUIRE(K >= 0 && rows >= 0, MOESQ_ERR_INVALID_ARG);
+  MOESQ_REQUIRE(layout == MOESQ_SF_LINEAR || layout == MOESQ_SF_KERNEL, MOESQ_ERR_INVALID_ARG);
+  MOESQ_REQUIRE(K % 128 == 0, MOESQ_ERR_UNSUPPORTED_SHAPE);
+  if (rows == 0 || K == 0) return MOESQ_OK;
+  MOESQ_REQUIRE(x && g_in && codes && sf, MOESQ_ERR_INVALID_ARG);
+  MOESQ_REQUIRE(moesq_aligned16(x) && moesq_aligned16(codes) && moesq_aligned16(sf),
+                MOESQ_ERR_INVALID_ARG);
+  if (expert_offsets) MOESQ_REQUIRE(E >= 1, MOESQ_ERR_INVALID_ARG);
+  if (layout == MOESQ_SF_KERNEL) MOESQ_REQUIRE(expert_offsets && pad_offsets, MOESQ_ERR_INVALID_ARG);
+  const int64_t n = rows * (K / 32);
+  int64_t g = (n + 127) / 128;
+  if (g > 148 * 32) g = 148 * 32;
+  k_quant_act<<<(int)g, 128, 0, (cudaStream_t)stream>>>(x, K, gather, expert_offsets, pad_offsets,
+                                                       E, g_in, rows, layout, codes, sf);
+  MOESQ_CHECK_LAUNCH();
+  return MOESQ_OK;
+}

@@ -1,0 +1,252 @@
+// Routing permutation (top-k -> per-expert slot groups) and weighted combine.
+//
+// The grouped GEMM of the pages runs over the tokens the router sends to each
+// expert (kernel line of the Qwen3.5-397B-A17B-P48NVFP4-MoESQ model card).  The
+// slot order is (expert, token, j): a stable counting sort of the flattened
+// top-k ids in three passes -- per-chunk histograms, one block scanning them,
+// and a stable scatter in which warps of a chunk take turns (match_any gives
+// the rank inside a warp).  Each expert's group also gets a 128-row aligned
+// place in the padded GEMM operand buffers (pad_offsets).
+#include "common.cuh"
+
+namespace moesq {
+
+constexpr int PERM_CHUNK = 1024;   // flattened (token, j) entries per block
+constexpr int PERM_THREADS = 1024;
+
+__device__ __forceinline__ int clamp_expert(int e, int E, int32_t* d_status) {
+  if (e < 0 || e >= E) {
+    flag(d_status, MOESQ_DFLAG_BAD_EXPERT);
+    return 0;
+  }
+  return e;
+}
+
+// pass 1: counts[e][c] of chunk c (expert-major, so pass 2 reads rows)
+__global__ void __launch_bounds__(PERM_THREADS) k_perm_count(const int32_t* __restrict__ ids,
+                                                             int64_t S, int E, int nchunks,
+                                                             int32_t* __restrict__ counts,
+                                                             int32_t* d_status) {
+  extern __shared__ int32_t hist[];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int64_t i = (int64_t)blockIdx.x * PERM_CHUNK + threadIdx.x;
+  if (i < S) atomicAdd(&hist[clamp_expert(ids[i], E, d_status)], 1);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    counts[(int64_t)e * nchunks + blockIdx.x] = hist[e];
+}
+
+// block-wide exclusive scan of one int per thread (PERM_THREADS threads)
+__device__ __forceinline__ int32_t block_excl_scan(int32_t v, int32_t* warp_sums, int32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int32_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sums[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int32_t w = warp_sums[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    warp_sums[lane] = w;  // inclusive
+    if (lane == 31) *total = w;
+  }
+  __syncthreads();
+  const int32_t r = x - v + (warp > 0 ? warp_sums[warp - 1] : 0);
+  __syncthreads();
+  return r;
+}
+
+// pass 2 (one block): per-expert exclusive scan over chunks (in place, a warp per
+// expert), then the expert offsets and their 128-row padded versions
+__global__ void __launch_bounds__(PERM_THREADS) k_perm_scan(int32_t* __restrict__ counts,
+                                                            int nchunks, int E,
+                                                            int32_t* __restrict__ expert_offsets,
+                                                            int32_t* __restrict__ pad_offsets) {
+  extern __shared__ int32_t sm[];
+  int32_t* tot = sm;  // [E]
+  __shared__ int32_t warp_sums[32];
+  __shared__ int32_t total;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int e = warp; e < E; e += PERM_THREADS / 32) {
+    int32_t* row = counts + (int64_t)e * nchunks;
+    int32_t run = 0;
+    for (int c0 = 0; c0 < nchunks; c0 += 32) {
+      const int c = c0 + lane;
+      const int32_t v = c < nchunks ? row[c] : 0;
+      int32_t x = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (c < nchunks) row[c] = run + x - v;
+      run += __shfl_sync(0xffffffffu, x, 31);
+    }
+    if (lane == 0) tot[e] = run;
+  }
+  __syncthreads();
+  // block scan over experts: each thread owns a run of consecutive experts
+  const int ept = (E + PERM_THREADS - 1) / PERM_THREADS;
+  const int e0 = threadIdx.x * ept;
+  int32_t la = 0, lb = 0;
+  for (int j = 0; j < ept; ++j)
+    if (e0 + j < E) {
+      la += tot[e0 + j];
+      lb += (tot[e0 + j] + 127) / 128 * 128;
+    }
+  int32_t ta, tb;
+  int32_t ea = block_excl_scan(la, warp_sums, &total);
+  ta = total;
+  int32_t eb = block_excl_scan(lb, warp_sums, &total);
+  tb = total;
+  for (int j = 0; j < ept; ++j)
+    if (e0 + j < E) {
+      expert_offsets[e0 + j] = ea;
+      pad_offsets[e0 + j] = eb;
+      ea += tot[e0 + j];
+      eb += (tot[e0 + j] + 127) / 128 * 128;
+    }
+  if (threadIdx.x == 0) {
+    expert_offsets[E] = ta;
+    pad_offsets[E] = tb;
+  }
+}
+
+// pass 3: stable scatter; warps of the chunk take turns in order
+__global__ void __launch_bounds__(PERM_THREADS) k_perm_scatter(
+    const int32_t* __restrict__ ids, int64_t S, int k, int E, const int32_t* __restrict__ chunk_base,
+    const int32_t* __restrict__ expert_offsets, int32_t* __restrict__ slot_token,
+    int32_t* __restrict__ token_slot) {
+  extern __shared__ int32_t run[];  // [E] next free slot of each expert for this chunk
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    run[e] = expert_offsets[e] + chunk_base[(int64_t)e * gridDim.x + blockIdx.x];
+  __syncthreads();
+  const int64_t i = (int64_t)blockIdx.x * PERM_CHUNK + threadIdx.x;
+  const bool valid = i < S;
+  int e = 0;
+  if (valid) {
+    e = ids[i];
+    if (e < 0 || e >= E) e = 0;
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const unsigned vmask = __ballot_sync(0xffffffffu, valid);
+  const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : -1);
+  const int rank = __popc(peers & ((1u << lane) - 1u));
+  const int cnt = __popc(peers);
+  const bool leader = valid && (rank == cnt - 1);
+  for (int w = 0; w < PERM_THREADS / 32; ++w) {
+    if (warp == w && valid) {
+      const int pos = run[e] + rank;
+      __syncwarp(vmask);
+      if (leader) run[e] = pos + 1;
+      slot_token[pos] = (int32_t)(i / k);
+      token_slot[i] = pos;
+    }
+    __syncthreads();
+  }
+}
+
+// combine: thread per (token, 8 features); float32 in j order, no fused multiply-add
+__global__ void k_unpermute(const uint16_t* __restrict__ y, const int32_t* __restrict__ token_slot,
+                            const float* __restrict__ topk_w, int64_t T, int k, int64_t H,
+                            uint16_t* __restrict__ out) {
+  const int64_t vec = H / 8;
+  const int64_t n = T * vec;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = i / vec, c = i % vec;
+    float acc[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
+    for (int j = 0; j < k; ++j) {
+      const int64_t s = token_slot[t * k + j];
+      const float w = topk_w[t * k + j];
+      const uint4 u = *reinterpret_cast<const uint4*>(y + s * H + 8 * c);
+      const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        acc[2 * q] = __fadd_rn(acc[2 * q], __fmul_rn(w, bf16_bits_to_float(wd[q] & 0xFFFF)));
+        acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], __fmul_rn(w, bf16_bits_to_float(wd[q] >> 16)));
+      }
+    }
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      o[q] = float_to_bf16_bits(acc[2 * q]) | (float_to_bf16_bits(acc[2 * q + 1]) << 16);
+    *reinterpret_cast<uint4*>(out + t * H + 8 * c) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+}  // namespace moesq
+
+using namespace moesq;
+
+extern "C" int64_t moesq_padded_rows(int64_t S, int32_t E) {
+  if (S < 0 || E <= 0) return 0;
+  const int64_t extra = 127 * (int64_t)(S < E ? S : E);  // only nonempty groups pad
+  return (S + extra + 127) / 128 * 128;
+}
+
+extern "C" moesq_status moesq_permute_workspace_size(int64_t T, int32_t k, int32_t E,
+                                                     size_t* bytes) {
+  MOESQ_REQUIRE(bytes && T >= 0 && k >= 1 && k <= 32 && E >= 1 && E <= 4096,
+                MOESQ_ERR_INVALID_ARG);
+  const int64_t S = T * k;
+  const int64_t nchunks = (S + PERM_CHUNK - 1) / PERM_CHUNK;
+  *bytes = (size_t)((nchunks > 0 ? nchunks : 1) * E) * sizeof(int32_t);
+  return MOESQ_OK;
+}
+
+extern "C" moesq_status moesq_permute(const int32_t* topk_ids, int64_t T, int32_t k, int32_t E,
+                                      int32_t* expert_offsets, int32_t* pad_offsets,
+                                      int32_t* slot_token, int32_t* token_slot, void* ws,
+                                      size_t ws_bytes, int32_t* d_status, moesq_stream_t stream) {
+  MOESQ_REQUIRE(expert_offsets && pad_offsets, MOESQ_ERR_INVALID_ARG);
+  MOESQ_REQUIRE(T >= 0 && k >= 1 && k <= 32 && E >= 1 && E <= 4096, MOESQ_ERR_INVALID_ARG);
+  const int64_t S = T * k;
+  MOESQ_REQUIRE(S < (1ll << 31), MOESQ_ERR_UNSUPPORTED_SHAPE);
+  MOESQ_REQUIRE(S == 0 || (topk_ids && slot_token && token_slot), MOESQ_ERR_INVALID_ARG);
+  size_t need = 0;
+  moesq_permute_workspace_size(T, k, E, &need);
+  MOESQ_REQUIRE(ws && ws_bytes >= need, MOESQ_ERR_WORKSPACE);
+  cudaStream_t s = (cudaStream_t)stream;
+  const int nchunks = (int)((S + PERM_CHUNK - 1) / PERM_CHUNK);
+  int32_t* counts = (int32_t*)ws;
+  const size_t shm = (size_t)E * sizeof(int32_t);
+  if (nchunks > 0) {
+    k_perm_count<<<nchunks, PERM_THREADS, shm, s>>>(topk_ids, S, E, nchunks, counts, d_status);
+    MOESQ_CHECK_LAUNCH();
+  }
+  k_perm_scan<<<1, PERM_THREADS, shm, s>>>(counts, nchunks, E, expert_offsets, pad_offsets);
+  MOESQ_CHECK_LAUNCH();
+  if (nchunks > 0) {
+    k_perm_scatter<<<nchunks, PERM_THREADS, shm, s>>>(topk_ids, S, k, E, counts, expert_offsets,
+                                                       slot_token, token_slot);
+    MOESQ_CHECK_LAUNCH();
+  }
+  return MOESQ_OK;
+}
+
+extern "C" moesq_status moesq_unpermute(const uint16_t* y, const int32_t* token_slot,
+                                        const float* topk_w, int64_t T, int32_t k, int64_t H,
+                                        uint16_t* out, moesq_stream_t stream) {
+  MOESQ_REQUIRE(T >= 0 && k >= 1 && H >= 0, MOESQ_ERR_INVALID_ARG);
+  MOESQ_REQUIRE(H % 8 == 0, MOESQ_ERR_UNSUPPORTED_SHAPE);
+  if (T == 0 || H == 0) return MOESQ_OK;
+  MOESQ_REQUIRE(y && token_slot && topk_w && out, MOESQ_ERR_INVALID_ARG);
+  MOESQ_REQUIRE(moesq_aligned16(y) && moesq_aligned16(out), MOESQ_ERR_INVALID_ARG);
+  const int64_t n = T * (H / 8);
+  int64_t g = (n + 255) / 256;
+  if (g > 148 * 16) g = 148 * 16;
+  k_unpermute<<<(int)g, 256, 0, (cudaStream_t)stream>>>(y, token_slot, topk_w, T, k, H, out);
+  MOESQ_CHECK_LAUNCH();
+  return MOESQ_OK;
+}
