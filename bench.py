@@ -38,7 +38,7 @@ METRIC = "dense-equiv TFLOP/s & % roofline, sparse NVFP4 MoE grouped GEMM (1 B20
 UNIT = "TFLOP/s"
 B_W, B_A = 0.34375, 0.53125     # bytes per dense element: sparse weight storage, NVFP4-32 activation
 FP4_SPARSE_OVER_BF16 = 8.0      # nominal dense-equivalent sparse FP4 (18 PF) / dense bf16 (2.25 PF)
-KERNELS_PER_STEP = 7            # permute x3, quant_act, gate_up GEMM, down GEMM, combine
+KERNELS_PER_STEP = 7            # permute x3, routed quant, gate_up GEMM, down GEMM, combine
 
 
 def parse_args():
@@ -215,8 +215,9 @@ class Bench:
                              self.token_slot, self.perm_ws, self.perm_ws_n, self.status)
 
     def quant_act(self):
-        self.M.moesq_quant_act(self.x.view(self.torch.uint16), self.cfg.H, self.slot_token, self.eo, self.po,
-                               self.cfg.E, self.g_in_gu, self.S, self.M.SF_KERNEL, self.a_codes, self.a_sf)
+        self.M.moesq_quant_act_routed(self.x.view(self.torch.uint16), self.T, self.cfg.H, self.ids,
+                                      self.token_slot, self.cfg.k, self.eo, self.po, self.cfg.E, self.g_in_gu,
+                                      self.a_codes, self.a_sf)
 
     def gemm_gate_up(self):
         self.M.moesq_grouped_gemm(self.lin["gate_up"].struct, self.a_codes, self.a_sf, self.g_in_gu, self.eo,
@@ -234,22 +235,42 @@ class Bench:
 
     STAGES = ("permute", "quant_act", "gemm_gate_up", "gemm_down", "combine")
 
+    def graphs(self):
+        """Each stage captured once as a CUDA graph, so timed replays carry no host
+        launch gaps (the L2 flush before each step keeps the host ahead)."""
+        torch = self.torch
+        if getattr(self, "_graphs", None) is None:
+            for s in self.STAGES:       # first calls outside capture (one-time attribute set-up)
+                getattr(self, s)()
+            torch.cuda.synchronize()
+            self._graphs = {}
+            for s in self.STAGES:
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    getattr(self, s)()
+                self._graphs[s] = g
+            torch.cuda.synchronize()
+        return self._graphs
+
     def run(self, steps, warmup, flush):
         torch = self.torch
         stream = torch.cuda.current_stream()
+        graphs = self.graphs()
         for _ in range(warmup):
             for s in self.STAGES:
-                getattr(self, s)()
+                graphs[s].replay()
         torch.cuda.synchronize()
         ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in self.STAGES] for _ in range(steps)]
+        torch.cuda.nvtx.range_push("timed")
         for i in range(steps):
             if flush is not None:
                 flush.zero_()
             for j, s in enumerate(self.STAGES):
                 ev[i][j][0].record(stream)
-                getattr(self, s)()
+                graphs[s].replay()
                 ev[i][j][1].record(stream)
+        torch.cuda.nvtx.range_pop()
         torch.cuda.synchronize()
         per = {s: [ev[i][j][0].elapsed_time(ev[i][j][1]) for i in range(steps)] for j, s in enumerate(self.STAGES)}
         return per
@@ -455,7 +476,8 @@ def run_ours(args, rank, world, local_rank):
                 d = a[s] * 1e-3
                 row[k] = {"ms": a[s], "TFLOPs": f2[k] / d / 1e12, "GBps": y2[k] / d / 1e9,
                           "roofline_frac": max(f2[k] / (p_fp4 * 1e12), y2[k] / (peaks["hbm_gbs"] * 1e9)) / d,
-                          "bound": "tensor" if f2[k] / p_fp4 > y2[k] / (peaks["hbm_gbs"] * 1e3) else "hbm"}
+                          "bound": ("tensor" if f2[k] / (p_fp4 * 1e12) > y2[k] / (peaks["hbm_gbs"] * 1e9)
+                                    else "hbm")}
             sweep.append(row)
             del bb
             torch.cuda.empty_cache()

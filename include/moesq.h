@@ -214,6 +214,18 @@ moesq_status moesq_quant_act(const uint16_t* x, int64_t K, const int32_t* gather
                              int32_t E, const float* g_in, int64_t rows, int32_t layout,
                              uint8_t* codes, uint8_t* sf, moesq_stream_t stream);
 
+/* Token-major variant used by moesq_moe_forward: reads each token row of x once and
+ * writes one padded operand row per routed slot (MOESQ_SF_KERNEL layout only).
+ *   x          device bf16 [T, K];  topk_ids, token_slot  device i32 [T, k]
+ *   expert_offsets, pad_offsets  device i32 [E+1] (moesq_permute);  g_in device f32 [E]
+ *   codes, sf  padded operand outputs as for MOESQ_SF_KERNEL.
+ * Same arithmetic as moesq_quant_act; ids outside [0, E) are treated as expert 0. */
+moesq_status moesq_quant_act_routed(const uint16_t* x, int64_t T, int64_t K,
+                                    const int32_t* topk_ids, const int32_t* token_slot, int32_t k,
+                                    const int32_t* expert_offsets, const int32_t* pad_offsets,
+                                    int32_t E, const float* g_in, uint8_t* codes, uint8_t* sf,
+                                    moesq_stream_t stream);
+
 /* ------------------------------------------------------------------------- *
  * Grouped sparse GEMM  [kernel]
  * ------------------------------------------------------------------------- */

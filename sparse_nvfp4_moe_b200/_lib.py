@@ -54,6 +54,8 @@ _SIGS = {
     "moesq_unpermute": (ctypes.c_int, [c_vp, c_vp, c_vp, c_i64, c_i32, c_i64, c_vp, c_vp]),
     "moesq_quant_act": (ctypes.c_int, [c_vp, c_i64, c_vp, c_vp, c_vp, c_i32, c_vp, c_i64, c_i32, c_vp,
                                        c_vp, c_vp]),
+    "moesq_quant_act_routed": (ctypes.c_int, [c_vp, c_i64, c_i64, c_vp, c_vp, c_i32, c_vp, c_vp, c_i32,
+                                              c_vp, c_vp, c_vp, c_vp]),
     "moesq_grouped_gemm": (ctypes.c_int, [ctypes.POINTER(Linear), c_vp, c_vp, c_vp, c_vp, c_vp, c_i64,
                                           c_i64, c_i32, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp, c_vp]),
     "moesq_grouped_gemm_workspace_size": (ctypes.c_int, [ctypes.POINTER(Linear), c_i64,
@@ -191,6 +193,13 @@ def moesq_quant_act(x, K, gather, expert_offsets, pad_offsets, E, g_in, rows, la
     _check("moesq_quant_act", lib().moesq_quant_act(_p(x), K, _p(gather), _p(expert_offsets),
                                                     _p(pad_offsets), E, _p(g_in), rows, layout,
                                                     _p(codes), _p(sf), _stream(stream)))
+
+
+def moesq_quant_act_routed(x, T, K, topk_ids, token_slot, k, expert_offsets, pad_offsets, E, g_in, codes,
+                           sf, stream=None):
+    _check("moesq_quant_act_routed", lib().moesq_quant_act_routed(
+        _p(x), T, K, _p(topk_ids), _p(token_slot), k, _p(expert_offsets), _p(pad_offsets), E, _p(g_in),
+        _p(codes), _p(sf), _stream(stream)))
 
 
 def moesq_grouped_gemm(W: Linear, act_codes, act_sf, g_act, expert_offsets, pad_offsets, S, P_cap,

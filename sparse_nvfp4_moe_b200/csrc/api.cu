@@ -112,8 +112,8 @@ extern "C" moesq_status moesq_moe_forward(const moesq_moe_layer* L, const uint16
   st = moesq_permute(topk_ids, T, L->k, L->E, eo, po, slot_token, token_slot, w + f.off_perm,
                      perm_bytes, d_status, stream);
   if (st != MOESQ_OK) return st;
-  st = moesq_quant_act(x, L->H, slot_token, eo, po, L->E, L->g_in_gate_up, f.S, MOESQ_SF_KERNEL,
-                       a_codes, a_sf, stream);
+  st = moesq_quant_act_routed(x, T, L->H, topk_ids, token_slot, L->k, eo, po, L->E, L->g_in_gate_up,
+                              a_codes, a_sf, stream);
   if (st != MOESQ_OK) return st;
   st = moesq_grouped_gemm(&L->gate_up, a_codes, a_sf, L->g_in_gate_up, eo, po, f.S, f.P,
                           MOESQ_EPI_SWIGLU_NVFP4, L->g_in_down, h_codes, h_sf, nullptr, 0, d_status,

@@ -36,6 +36,37 @@ __device__ __forceinline__ uint32_t e2m1_code(float v) {
   return c | ((__float_as_uint(v) >> 28) & 8u);
 }
 
+// Eight float32 values -> eight E2M1 codes in one word (value i in nibble i),
+// with the hardware conversion cvt.rn.satfinite.e2m1x2.f32: round to nearest,
+// ties to even, saturating at 6, sign kept (the same rule as e2m1_code).  The
+// first source operand of each cvt lands in the high nibble of its byte.
+__device__ __forceinline__ uint32_t e2m1x8(float a0, float a1, float a2, float a3, float a4,
+                                           float a5, float a6, float a7) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(out)
+      : "f"(a0), "f"(a1), "f"(a2), "f"(a3), "f"(a4), "f"(a5), "f"(a6), "f"(a7));
+  return out;
+}
+
+// codes of v[0..7] under a group multiplier (inv == 0: the group is all zeros)
+__device__ __forceinline__ uint32_t nvfp4_word(const float* v, float inv) {
+  if (inv == 0.0f) return 0u;
+  return e2m1x8(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv), __fmul_rn(v[2], inv),
+                __fmul_rn(v[3], inv), __fmul_rn(v[4], inv), __fmul_rn(v[5], inv),
+                __fmul_rn(v[6], inv), __fmul_rn(v[7], inv));
+}
+
+// silu(x) = x / (1 + exp(-x)) with the fast exponential and reciprocal
+__device__ __forceinline__ float silu_fast(float x) {
+  return x * __frcp_rn(1.0f + __expf(-x));
+}
+
 // E4M3 (finite, saturating) code of a nonnegative float32, nearest-even.
 __device__ __forceinline__ uint32_t e4m3_code(float s) {
   return (uint32_t)__nv_cvt_float_to_fp8(s, __NV_SATFINITE, __NV_E4M3);

@@ -17,7 +17,7 @@
 //   * is warp-specialised: warp 0 issues TMA (values and tokens) and bulk copies
 //     (metadata, block scales) into a 6-stage shared-memory ring; warp 1 owns
 //     TMEM, copies metadata and scales smem->TMEM (tcgen05.cp) and issues the
-//     MMAs (dense K = 128 each, two per stage); warps 2..5 drain the
+//     MMAs (dense K = 128 each, two per stage); warps 2..9 drain the
 //     double-buffered FP32 accumulators (tcgen05.ld) while the next tile runs;
 //   * fuses the epilogue: FP32 or bf16 output per slot, or SwiGLU followed by
 //     NVFP4 requantisation written straight into the next GEMM's B operand
@@ -44,7 +44,9 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES + E_BYTES + 2 * SF_BYTES;  // 2867
 constexpr int EPI_LD = 65;                 // floats per staged accumulator row (64 + pad)
 constexpr int EPI_BYTES = BM * EPI_LD * 4;
 constexpr int MAX_E = 1024;
-constexpr int THREADS = 192;
+constexpr int EPI_WARPS = 8;
+constexpr int EPI_THREADS = 32 * EPI_WARPS;
+constexpr int THREADS = 64 + EPI_THREADS;   // producer warp, MMA warp, epilogue warps
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_ACC = 0, TM_E = 256, TM_SFA = 264, TM_SFB = 272;
 
@@ -113,11 +115,10 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-__device__ __forceinline__ float silu(float x) { return x / (1.0f + expf(-x)); }
-
 __global__ void __launch_bounds__(THREADS, 1)
     k_grouped_gemm_sp(const __grid_constant__ CUtensorMap tmap_a,
-                      const __grid_constant__ CUtensorMap tmap_b, const Params p) {
+                      const __grid_constant__ CUtensorMap tmap_b,
+                      const __grid_constant__ CUtensorMap tmap_b32, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   float* epi = (float*)(smem + STAGES * STAGE_BYTES);
@@ -136,13 +137,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.acc_full[i], 1);
-      mbar_init(&S.acc_empty[i], 4);
+      mbar_init(&S.acc_empty[i], EPI_WARPS);
     }
     mbar_init(&S.done, 1);
     S.abort = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmap_a);
     tma_prefetch_desc(&tmap_b);
+    tma_prefetch_desc(&tmap_b32);
   }
   if (warp == 0) {  // tile_start[e] = sum over e' < e of ceil(T_e' / BN)
     int run = 0;
@@ -196,15 +198,18 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint8_t* meta = p.meta + (size_t)(t.e * MT + t.mt) * nkb * 2048;
         const uint8_t* sfa = p.sfw + (size_t)(t.e * MT + t.mt) * kb128 * 512;
         const uint8_t* sfb = p.act_sf + (size_t)(prow / 128) * kb128 * 512;
+        // a tile of <= 32 tokens loads a 32-row B box (decode-sized groups)
+        const bool b32 = t.n_rows <= 32;
+        const uint32_t b_bytes = b32 ? 32 * 128 : B_BYTES;
         for (int kb = 0; kb < nkb; ++kb) {
           mbar_wait(&S.empty[stage], phase ^ 1, abort, p.d_status);
           const int nk = (kb128 - 2 * kb) >= 2 ? 2 : 1;
           uint8_t* st = smem + stage * STAGE_BYTES;
-          mbar_arrive_expect_tx(&S.full[stage],
-                                A_BYTES + B_BYTES + E_BYTES + 2 * nk * 512);
+          mbar_arrive_expect_tx(&S.full[stage], A_BYTES + b_bytes + E_BYTES + 2 * nk * 512);
           tma_load_2d(st, &tmap_a, kb * 64, r0, &S.full[stage]);
           tma_load_2d(st + A_BYTES / 2, &tmap_a, kb * 64, r1, &S.full[stage]);
-          tma_load_2d(st + A_BYTES, &tmap_b, kb * 128, prow, &S.full[stage]);
+          tma_load_2d(st + A_BYTES, b32 ? (const void*)&tmap_b32 : (const void*)&tmap_b, kb * 128, prow,
+                      &S.full[stage]);
           bulk_load(st + A_BYTES + B_BYTES, meta + (size_t)kb * 2048, E_BYTES, &S.full[stage]);
           bulk_load(st + A_BYTES + B_BYTES + E_BYTES, sfa + (size_t)kb * 1024, nk * 512,
                     &S.full[stage]);
@@ -276,8 +281,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncwarp();
   } else {
     // ================================================================ epilogue
-    const int q = warp & 3;            // TMEM lane quarter this warp may access
-    const int et = threadIdx.x - 64;   // 0..127
+    // 8 warps, two per TMEM lane quarter; per 64-column chunk each warp moves its
+    // 32 rows x 32 columns to shared memory (x alpha), then all 256 threads
+    // finish one (column, row-range) item each.
+    const int ew = warp - 2;            // 0..7
+    const int q = warp & 3;             // TMEM lane quarter this warp may access
+    const int hh = ew >> 2;             // which 32-column half of the chunk
+    const int et = threadIdx.x - 64;    // 0..255
     uint32_t acc_phase[2] = {0u, 0u};
     int buf = 0;
     const int I = p.M / 2;
@@ -287,13 +297,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_wait(&S.acc_full[buf], acc_phase[buf], abort, p.d_status);
       tc_fence_after();
       for (int c0 = 0; c0 < t.n_rows; c0 += 64) {
-        // phase 1: this warp's 32 accumulator rows, 64 token columns -> smem (x alpha)
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        {  // phase 1
           uint32_t r[32];
-          tmem_ld_32x32b_x32(tmem + TM_ACC + buf * BN + c0 + 32 * h + ((uint32_t)(32 * q) << 16), r);
+          tmem_ld_32x32b_x32(tmem + TM_ACC + buf * BN + c0 + 32 * hh + ((uint32_t)(32 * q) << 16), r);
           tmem_ld_wait();
-          float* row = epi + (32 * q + lane) * EPI_LD + 32 * h;
+          float* row = epi + (32 * q + lane) * EPI_LD + 32 * hh;
 #pragma unroll
           for (int j = 0; j < 32; ++j) row[j] = __fmul_rn(__uint_as_float(r[j]), alpha);
         }
@@ -302,58 +310,56 @@ __global__ void __launch_bounds__(THREADS, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&S.acc_empty[buf]);
         }
-        named_bar_sync(1, 128);
-        // phase 2: one token column per thread
-        const int j = et & 63, half = et >> 6;
-        const int n = t.nt * BN + c0 + j;
-        if (c0 + j < t.n_rows) {
-          if (p.epi == MOESQ_EPI_SWIGLU_NVFP4) {
-            float h[32];
-            float amax = 0.0f;
+        named_bar_sync(1, EPI_THREADS);
+        if (p.epi == MOESQ_EPI_SWIGLU_NVFP4) {
+          // item: column j, 32-feature group g, half pp of the group (partner = lane ^ 1)
+          const int pp = et & 1, j = (et >> 1) & 63, g = et >> 7;
+          const int n = t.nt * BN + c0 + j;
+          float h[16];
+          float amax = 0.0f;
 #pragma unroll
-            for (int f = 0; f < 32; ++f) {
-              const float gv = epi[(32 * half + f) * EPI_LD + j];
-              const float uv = epi[(64 + 32 * half + f) * EPI_LD + j];
-              h[f] = __fmul_rn(silu(gv), uv);
-              amax = fmaxf(amax, fabsf(h[f]));
-            }
+          for (int f = 0; f < 16; ++f) {
+            const int r = 32 * g + 16 * pp + f;
+            h[f] = __fmul_rn(silu_fast(epi[r * EPI_LD + j]), epi[(64 + r) * EPI_LD + j]);
+            amax = fmaxf(amax, fabsf(h[f]));
+          }
+          amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+          if (c0 + j < t.n_rows) {
             const GroupScale gs = nvfp4_group_scale(amax, p.g_next[t.e]);
-            uint32_t o[4];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              uint32_t word = 0;
-#pragma unroll
-              for (int u = 0; u < 8; ++u) word |= nvfp4_code(h[8 * c + u], gs.inv) << (4 * u);
-              o[c] = word;
-            }
+            const uint2 o = make_uint2(nvfp4_word(h, gs.inv), nvfp4_word(h + 8, gs.inv));
             const int64_t prow = (int64_t)p.pad_offsets[t.e] + n;
-            const int fb = 64 * t.mt + 32 * half;  // first feature of this group
+            const int fb = 64 * t.mt + 32 * g;  // first feature of this group
             if (prow >= 0 && prow < p.P_cap) {
               uint8_t* codes = (uint8_t*)p.out;
-              *reinterpret_cast<uint4*>(codes + prow * (I / 2) + fb / 2) = make_uint4(o[0], o[1], o[2], o[3]);
-              const int64_t blk = (prow / 128) * (I / 128) + fb / 128;
-              p.out_sf[blk * 512 + sf_block_offset((uint32_t)(prow % 128), (uint32_t)((fb / 32) % 4))] =
-                  (uint8_t)gs.sc;
+              *reinterpret_cast<uint2*>(codes + prow * (I / 2) + fb / 2 + 8 * pp) = o;
+              if (pp == 0) {
+                const int64_t blk = (prow / 128) * (I / 128) + fb / 128;
+                p.out_sf[blk * 512 + sf_block_offset((uint32_t)(prow % 128), (uint32_t)((fb / 32) % 4))] =
+                    (uint8_t)gs.sc;
+              }
             }
-          } else {
-            const int64_t s = (int64_t)off[t.e] + n;
-            int col0;  // first output column of this thread's 64 rows
-            if (p.gate_up) col0 = half == 0 ? 64 * t.mt : I + 64 * t.mt;
-            else col0 = BM * t.mt + 64 * half;
-            const float* src = epi + (64 * half) * EPI_LD + j;
-            if (s < 0 || s >= p.S) {
-              // inconsistent offsets: write nothing outside the output
-            } else if (p.epi == MOESQ_EPI_F32) {
+          }
+        } else {
+          // item: column j, 32 consecutive accumulator rows seg*32 ..
+          const int j = et & 63, seg = et >> 6;
+          const int n = t.nt * BN + c0 + j;
+          const int64_t s = (int64_t)off[t.e] + n;
+          if (c0 + j < t.n_rows && s >= 0 && s < p.S) {
+            int col0;  // first output column of these 32 rows
+            if (p.gate_up) col0 = seg < 2 ? 64 * t.mt + 32 * seg : I + 64 * t.mt + 32 * (seg - 2);
+            else col0 = BM * t.mt + 32 * seg;
+            const float* src = epi + (32 * seg) * EPI_LD + j;
+            if (p.epi == MOESQ_EPI_F32) {
               float* y = (float*)p.out + s * p.M + col0;
 #pragma unroll
-              for (int c = 0; c < 16; ++c)
+              for (int c = 0; c < 8; ++c)
                 *reinterpret_cast<float4*>(y + 4 * c) =
                     make_float4(src[(4 * c) * EPI_LD], src[(4 * c + 1) * EPI_LD],
                                 src[(4 * c + 2) * EPI_LD], src[(4 * c + 3) * EPI_LD]);
             } else {
               uint16_t* y = (uint16_t*)p.out + s * p.M + col0;
 #pragma unroll
-              for (int c = 0; c < 8; ++c) {
+              for (int c = 0; c < 4; ++c) {
                 uint32_t w[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u)
@@ -364,12 +370,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
           }
         }
-        named_bar_sync(1, 128);
-      }
-      if (t.n_rows <= 0) {  // cannot happen for listed tiles; keep the handshake balanced
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S.acc_empty[buf]);
+        named_bar_sync(1, EPI_THREADS);
       }
       acc_phase[buf] ^= 1;
       buf ^= 1;
@@ -478,11 +479,14 @@ extern "C" moesq_status moesq_grouped_gemm(const moesq_linear* W, const uint8_t*
   if (sms < 0) return MOESQ_ERR_CUDA;
   if (sms == 0) return MOESQ_ERR_DEVICE;
 
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, tb32;
   if (!make_tmap_u8(&ta, W->packed, (uint64_t)(W->K / 4), (uint64_t)(W->E * W->out), 64, 64,
                     CU_TENSOR_MAP_SWIZZLE_64B))
     return MOESQ_ERR_CUDA;
   if (!make_tmap_u8(&tb, act_codes, (uint64_t)(W->K / 2), (uint64_t)P_cap, 128, 128,
+                    CU_TENSOR_MAP_SWIZZLE_128B))
+    return MOESQ_ERR_CUDA;
+  if (!make_tmap_u8(&tb32, act_codes, (uint64_t)(W->K / 2), (uint64_t)P_cap, 128, 32,
                     CU_TENSOR_MAP_SWIZZLE_128B))
     return MOESQ_ERR_CUDA;
 
@@ -512,7 +516,7 @@ extern "C" moesq_status moesq_grouped_gemm(const moesq_linear* W, const uint8_t*
   prm.gate_up = gate_up ? 1 : 0;
   prm.S = S;
   prm.P_cap = P_cap;
-  sp::k_grouped_gemm_sp<<<sms, sp::THREADS, sp::SMEM_BYTES, (cudaStream_t)stream>>>(ta, tb, prm);
+  sp::k_grouped_gemm_sp<<<sms, sp::THREADS, sp::SMEM_BYTES, (cudaStream_t)stream>>>(ta, tb, tb32, prm);
   MOESQ_CHECK_LAUNCH();
   return MOESQ_OK;
 }

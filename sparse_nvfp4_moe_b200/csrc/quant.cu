@@ -54,12 +54,7 @@ __global__ void k_quant_act(const uint16_t* __restrict__ x, int64_t K, const int
     const GroupScale gs = nvfp4_group_scale(amax, g);
     uint32_t o[4];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t word = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) word |= nvfp4_code(v[8 * c + j], gs.inv) << (4 * j);
-      o[c] = word;
-    }
+    for (int c = 0; c < 4; ++c) o[c] = nvfp4_word(v + 8 * c, gs.inv);
     int64_t row = s;
     if (layout == MOESQ_SF_KERNEL) row = (int64_t)pad_offsets[e] + (s - expert_offsets[e]);
     *reinterpret_cast<uint4*>(codes + row * (K / 2) + 16 * grp) = make_uint4(o[0], o[1], o[2], o[3]);
@@ -72,9 +67,78 @@ __global__ void k_quant_act(const uint16_t* __restrict__ x, int64_t K, const int
   }
 }
 
+// Token-major variant for the MoE forward: thread per (token, 32-group); x is
+// read once per token and written once per routed slot (k times), each with the
+// global of the slot's expert, into the padded operand layout.
+__global__ void k_quant_act_routed(const uint16_t* __restrict__ x, int64_t T, int64_t K,
+                                   const int32_t* __restrict__ topk_ids,
+                                   const int32_t* __restrict__ token_slot, int k,
+                                   const int32_t* __restrict__ expert_offsets,
+                                   const int32_t* __restrict__ pad_offsets, int E,
+                                   const float* __restrict__ g_in, uint8_t* __restrict__ codes,
+                                   uint8_t* __restrict__ sf) {
+  const int64_t G = K / 32;
+  const int64_t n = T * G;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = i / G, grp = i % G;
+    float v[32];
+    const uint4* q = reinterpret_cast<const uint4*>(x + t * K + 32 * grp);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint4 u = q[c];
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        v[8 * c + 2 * j] = bf16_bits_to_float(w[j] & 0xFFFF);
+        v[8 * c + 2 * j + 1] = bf16_bits_to_float(w[j] >> 16);
+      }
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(v[j]));
+    for (int j = 0; j < k; ++j) {
+      int e = topk_ids[t * k + j];
+      if (e < 0 || e >= E) e = 0;
+      const int64_t s = token_slot[t * k + j];
+      const GroupScale gs = nvfp4_group_scale(amax, g_in[e]);
+      uint32_t o[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) o[c] = nvfp4_word(v + 8 * c, gs.inv);
+      const int64_t row = (int64_t)pad_offsets[e] + (s - expert_offsets[e]);
+      *reinterpret_cast<uint4*>(codes + row * (K / 2) + 16 * grp) = make_uint4(o[0], o[1], o[2], o[3]);
+      const int64_t blk = (row / 128) * (K / 128) + grp / 4;
+      sf[blk * 512 + sf_block_offset((uint32_t)(row % 128), (uint32_t)(grp % 4))] = (uint8_t)gs.sc;
+    }
+  }
+}
+
 }  // namespace moesq
 
 using namespace moesq;
+
+extern "C" moesq_status moesq_quant_act_routed(const uint16_t* x, int64_t T, int64_t K,
+                                               const int32_t* topk_ids, const int32_t* token_slot,
+                                               int32_t k, const int32_t* expert_offsets,
+                                               const int32_t* pad_offsets, int32_t E,
+                                               const float* g_in, uint8_t* codes, uint8_t* sf,
+                                               moesq_stream_t stream) {
+  MOESQ_REQUIRE(T >= 0 && K >= 0 && k >= 1 && E >= 1, MOESQ_ERR_INVALID_ARG);
+  MOESQ_REQUIRE(K % 128 == 0, MOESQ_ERR_UNSUPPORTED_SHAPE);
+  if (T == 0 || K == 0) return MOESQ_OK;
+  MOESQ_REQUIRE(x && topk_ids && token_slot && expert_offsets && pad_offsets && g_in && codes && sf,
+                MOESQ_ERR_INVALID_ARG);
+  MOESQ_REQUIRE(moesq_aligned16(x) && moesq_aligned16(codes) && moesq_aligned16(sf),
+                MOESQ_ERR_INVALID_ARG);
+  const int64_t n = T * (K / 32);
+  int64_t g = (n + 127) / 128;
+  if (g > 148 * 32) g = 148 * 32;
+  k_quant_act_routed<<<(int)g, 128, 0, (cudaStream_t)stream>>>(x, T, K, topk_ids, token_slot, k,
+                                                              expert_offsets, pad_offsets, E, g_in,
+                                                              codes, sf);
+  MOESQ_CHECK_LAUNCH();
+  return MOESQ_OK;
+}
 
 extern "C" moesq_status moesq_quant_act(const uint16_t* x, int64_t K, const int32_t* gather,
                                         const int32_t* expert_offsets, const int32_t* pad_offsets,

@@ -147,10 +147,19 @@ __global__ void k_prune_amax(const uint16_t* __restrict__ w, int64_t E, int64_t 
         if ((nib >> p) & 1) amax = fmaxf(amax, fmaxf(fabsf(v[8 * c + 2 * p]), fabsf(v[8 * c + 2 * p + 1])));
     }
     *reinterpret_cast<uint16_t*>(mask + 2 * i) = (uint16_t)m16;
-    // warp-reduce before the atomic when the whole warp is in one segment
+    // one atomic per warp when the whole warp is in one segment
+    // (nonnegative floats order as their bit patterns)
     const int64_t e = row / out, seg = (row % out) / seg_rows;
     const uint32_t key = (uint32_t)(e * n_seg + seg);
-    atomicMax(seg_amax + key, __float_as_uint(amax));  // nonnegative floats order as uints
+    const unsigned act = __activemask();
+    const int leader = __ffs(act) - 1;
+    const uint32_t key0 = __shfl_sync(act, key, leader);
+    if (__all_sync(act, key == key0)) {
+      const uint32_t mx = __reduce_max_sync(act, __float_as_uint(amax));
+      if ((int)(threadIdx.x & 31) == leader) atomicMax(seg_amax + key, mx);
+    } else {
+      atomicMax(seg_amax + key, __float_as_uint(amax));
+    }
   }
 }
 
@@ -179,22 +188,24 @@ __global__ void k_quant_encode(const uint16_t* __restrict__ w, int64_t E, int64_
         if ((m16 >> (4 * c + p)) & 1)
           amax = fmaxf(amax, fmaxf(fabsf(v[8 * c + 2 * p]), fabsf(v[8 * c + 2 * p + 1])));
     const GroupScale gs = nvfp4_group_scale(amax, g);
-    uint32_t outw[2] = {0u, 0u};  // 8 kept bytes of the 4 chunks
+    // the 16 kept values in K order (2 pairs per chunk) -> 8 kept bytes
+    float kept[16];
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       const uint32_t nib = (m16 >> (4 * c)) & 0xF;
-      uint32_t k = 0, bytes = 0;
+      int k = 0;
 #pragma unroll
       for (int p = 0; p < 4; ++p) {
         if ((nib >> p) & 1) {
-          const uint32_t lo = nvfp4_code(v[8 * c + 2 * p], gs.inv);
-          const uint32_t hi = nvfp4_code(v[8 * c + 2 * p + 1], gs.inv);
-          bytes |= (lo | (hi << 4)) << (8 * k);
+          if (k < 2) {
+            kept[4 * c + 2 * k] = v[8 * c + 2 * p];
+            kept[4 * c + 2 * k + 1] = v[8 * c + 2 * p + 1];
+          }
           ++k;
         }
       }
-      outw[c >> 1] |= bytes << (16 * (c & 1));
     }
+    uint32_t outw[2] = {nvfp4_word(kept, gs.inv), nvfp4_word(kept + 8, gs.inv)};
     *reinterpret_cast<uint2*>(packed + 8 * i) = make_uint2(outw[0], outw[1]);
     scale[i] = (uint8_t)gs.sc;
   }

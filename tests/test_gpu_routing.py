@@ -125,3 +125,28 @@ def test_combine_golden_on_gpu(golden):
     M.moesq_unpermute(cuda(y, torch.bfloat16).view(torch.uint16), cuda(np.array(g["token_slot"], np.int32)),
                       cuda(np.array(g["topk_w"], np.float32)), 2, 3, 8, out.view(torch.uint16))
     assert out.float().cpu().numpy()[:, :2].tolist() == g["out"]
+
+
+@pytest.mark.parametrize("cfg_name,T", [("tiny", 64), ("qwen3_30b_a3b", 512), ("qwen3_5_397b_a17b", 16),
+                                        ("kimi_k2", 32)])
+def test_quant_act_routed_bit_exact(cfg_name, T):
+    """Token-major quantisation (x read once per token) equals the per-slot oracle rule."""
+    cfg = W.CONFIGS[cfg_name]
+    x = W.layer_input_bf16(cfg, T)
+    ids, _ = W.routing(cfg, T)
+    ref = R.permute(ids.numpy(), cfg.E)
+    rng = np.random.default_rng(T + 1)
+    g_in = (np.float32(W.activation_global_scale_input(x)) * rng.uniform(0.5, 2.0, cfg.E)).astype(np.float32)
+    want_c, want_s = G.quant_act(x.float().numpy(), ref["slot_token"], ref["expert_offsets"], g_in)
+    want_packed = (want_c[:, 0::2] | (want_c[:, 1::2] << 4)).astype(np.uint8)
+    eo, po, st, ts, _ = gpu_permute(ids.numpy(), cfg.E)
+    Sn, K = T * cfg.k, cfg.H
+    P = M.padded_rows(Sn, cfg.E)
+    codes = torch.empty((P, K // 2), dtype=torch.uint8, device="cuda")
+    sf = torch.empty((P // 128) * (K // 128) * 512, dtype=torch.uint8, device="cuda")
+    M.moesq_quant_act_routed(x.cuda().view(torch.uint16), T, K, ids.cuda(), ts, cfg.k, eo, po, cfg.E,
+                             cuda(g_in), codes, sf)
+    got_c, got_s = kernel_rows_to_slots(codes.cpu().numpy(), sf.cpu().numpy(), ref["expert_offsets"],
+                                        ref["pad_offsets"], K)
+    assert np.array_equal(got_s, want_s)
+    assert np.array_equal(got_c, want_packed)
