@@ -236,8 +236,8 @@ class Bench:
     STAGES = ("permute", "quant_act", "gemm_gate_up", "gemm_down", "combine")
 
     def graphs(self):
-        """Each stage captured once as a CUDA graph, so timed replays carry no host
-        launch gaps (the L2 flush before each step keeps the host ahead)."""
+        """The step as one CUDA graph, and each stage as its own graph (for the
+        per-kernel breakdown).  Replays carry no host launch gaps inside a graph."""
         torch = self.torch
         if getattr(self, "_graphs", None) is None:
             for s in self.STAGES:       # first calls outside capture (one-time attribute set-up)
@@ -249,31 +249,48 @@ class Bench:
                 with torch.cuda.graph(g):
                     getattr(self, s)()
                 self._graphs[s] = g
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for s in self.STAGES:
+                    getattr(self, s)()
+            self._graphs["step"] = g
             torch.cuda.synchronize()
         return self._graphs
 
     def run(self, steps, warmup, flush):
+        """Whole-step times (one graph per step) and per-stage times (one graph per
+        stage), each step after an L2 flush and a GPU sleep that keeps the host ahead."""
         torch = self.torch
         stream = torch.cuda.current_stream()
         graphs = self.graphs()
         for _ in range(warmup):
-            for s in self.STAGES:
-                graphs[s].replay()
+            graphs["step"].replay()
         torch.cuda.synchronize()
-        ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in self.STAGES] for _ in range(steps)]
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
         torch.cuda.nvtx.range_push("timed")
         for i in range(steps):
             if flush is not None:
                 flush.zero_()
-            for j, s in enumerate(self.STAGES):
-                ev[i][j][0].record(stream)
-                graphs[s].replay()
-                ev[i][j][1].record(stream)
+            torch.cuda._sleep(1_000_000)
+            ev[i][0].record(stream)
+            graphs["step"].replay()
+            ev[i][1].record(stream)
         torch.cuda.nvtx.range_pop()
         torch.cuda.synchronize()
-        per = {s: [ev[i][j][0].elapsed_time(ev[i][j][1]) for i in range(steps)] for j, s in enumerate(self.STAGES)}
-        return per
+        step_ms = [a.elapsed_time(b) for a, b in ev]
+        evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in self.STAGES] for _ in range(steps)]
+        for i in range(steps):
+            if flush is not None:
+                flush.zero_()
+            torch.cuda._sleep(1_000_000)
+            for j, s in enumerate(self.STAGES):
+                evs[i][j][0].record(stream)
+                graphs[s].replay()
+                evs[i][j][1].record(stream)
+        torch.cuda.synchronize()
+        per = {s: [evs[i][j][0].elapsed_time(evs[i][j][1]) for i in range(steps)] for j, s in enumerate(self.STAGES)}
+        return step_ms, per
 
     def check_against_forward(self):
         """The staged step and the single moesq_moe_forward call give identical bytes."""
@@ -387,12 +404,12 @@ def run_ours(args, rank, world, local_rank):
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
-        per = b.run(args.steps, max(args.warmup, 3), flush)
+        step_ms, per = b.run(args.steps, max(args.warmup, 3), flush)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
     clocks = clk.summary()
-    total_ms = sum(sum(v) for v in per.values())
+    total_ms = sum(step_ms)
     if world > 1:
         t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -466,12 +483,13 @@ def run_ours(args, rank, world, local_rank):
             if T == args.tokens:
                 continue
             bb = Bench(cfg, T, dev, lin=b.lin)
-            per_t = bb.run(10, 3, flush)
+            st_t, per_t = bb.run(10, 3, flush)
             a = {s: sum(v) / len(v) for s, v in per_t.items()}
             f2 = step_flops(bb.S, H, I)
             y2 = step_bytes(bb.S, T, H, I, bb.n_touched)
-            row = {"tokens": T, "ms_per_step": sum(a.values()),
-                   "TFLOPs": (f2["gate_up"] + f2["down"]) / (sum(a.values()) * 1e-3) / 1e12}
+            ms_t = sum(st_t) / len(st_t)
+            row = {"tokens": T, "ms_per_step": ms_t,
+                   "TFLOPs": (f2["gate_up"] + f2["down"]) / (ms_t * 1e-3) / 1e12}
             for s, k in (("gemm_gate_up", "gate_up"), ("gemm_down", "down")):
                 d = a[s] * 1e-3
                 row[k] = {"ms": a[s], "TFLOPs": f2[k] / d / 1e12, "GBps": y2[k] / d / 1e9,

@@ -41,8 +41,7 @@ constexpr int B_BYTES = BN * BK / 2;       // token codes: 128 B per row (SW128)
 constexpr int E_BYTES = BM * 16;           // metadata: 16 B per row
 constexpr int SF_BYTES = 2 * 512;          // two 512-byte scale blocks
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + E_BYTES + 2 * SF_BYTES;  // 28672
-constexpr int EPI_LD = 65;                 // floats per staged accumulator row (64 + pad)
-constexpr int EPI_BYTES = BM * EPI_LD * 4;
+constexpr int EPI_BYTES = 4 * 2 * 32 * 32 * 4;  // SwiGLU gate/up exchange blocks (4 warp pairs)
 constexpr int MAX_E = 1024;
 constexpr int EPI_WARPS = 8;
 constexpr int EPI_THREADS = 32 * EPI_WARPS;
@@ -281,96 +280,130 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncwarp();
   } else {
     // ================================================================ epilogue
-    // 8 warps, two per TMEM lane quarter; per 64-column chunk each warp moves its
-    // 32 rows x 32 columns to shared memory (x alpha), then all 256 threads
-    // finish one (column, row-range) item each.
+    // 8 warps, two per TMEM lane quarter q (rows 32q..32q+31); warp half hh owns
+    // token columns [64hh, 64hh+64).  Lane = accumulator row = output feature.
     const int ew = warp - 2;            // 0..7
     const int q = warp & 3;             // TMEM lane quarter this warp may access
-    const int hh = ew >> 2;             // which 32-column half of the chunk
-    const int et = threadIdx.x - 64;    // 0..255
+    const int hh = ew >> 2;             // column half
     uint32_t acc_phase[2] = {0u, 0u};
     int buf = 0;
     const int I = p.M / 2;
+    // SwiGLU exchange: gate quarter q (0,1) pairs with up quarter q+2 on the same
+    // column half; each side hands the other a 32x32 block (column-major, lane-fast).
+    const int pair = (q & 1) + 2 * hh;  // 0..3
+    float* xch = epi + pair * 2 * 32 * 32;  // [2][32 cols][32 lanes]
     for (int id = blockIdx.x; id < total; id += gridDim.x) {
       const Tile t = decode_tile(S, id, MT, E, off);
       const float alpha = __fmul_rn(p.g_act[t.e], p.alpha_w[t.e]);
       mbar_wait(&S.acc_full[buf], acc_phase[buf], abort, p.d_status);
       tc_fence_after();
-      for (int c0 = 0; c0 < t.n_rows; c0 += 64) {
-        {  // phase 1
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(tmem + TM_ACC + buf * BN + c0 + 32 * hh + ((uint32_t)(32 * q) << 16), r);
+      const uint32_t tbase = tmem + TM_ACC + buf * BN + ((uint32_t)(32 * q) << 16);
+      const int c_lo = 64 * hh;                 // first column of this warp's half
+      const bool live = c_lo < t.n_rows;        // any valid token column in the half
+      if (p.epi == MOESQ_EPI_SWIGLU_NVFP4) {
+        const bool is_gate = q < 2;
+        // gate warp finishes columns [c_lo, c_lo+32), up warp [c_lo+32, c_lo+64)
+        uint32_t mine[32], other[32];
+        if (live) {
+          tmem_ld_32x32b_x32(tbase + c_lo + (is_gate ? 0 : 32), mine);
+          tmem_ld_32x32b_x32(tbase + c_lo + (is_gate ? 32 : 0), other);
           tmem_ld_wait();
-          float* row = epi + (32 * q + lane) * EPI_LD + 32 * hh;
-#pragma unroll
-          for (int j = 0; j < 32; ++j) row[j] = __fmul_rn(__uint_as_float(r[j]), alpha);
         }
-        if (c0 + 64 >= t.n_rows) {  // accumulator fully read: hand it back to the MMA warp
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&S.acc_empty[buf]);
-        }
-        named_bar_sync(1, EPI_THREADS);
-        if (p.epi == MOESQ_EPI_SWIGLU_NVFP4) {
-          // item: column j, 32-feature group g, half pp of the group (partner = lane ^ 1)
-          const int pp = et & 1, j = (et >> 1) & 63, g = et >> 7;
-          const int n = t.nt * BN + c0 + j;
-          float h[16];
-          float amax = 0.0f;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.acc_empty[buf]);
+        float* give = xch + (is_gate ? 0 : 1) * 1024;
+        const float* take = xch + (is_gate ? 1 : 0) * 1024;
+        if (live) {
 #pragma unroll
-          for (int f = 0; f < 16; ++f) {
-            const int r = 32 * g + 16 * pp + f;
-            h[f] = __fmul_rn(silu_fast(epi[r * EPI_LD + j]), epi[(64 + r) * EPI_LD + j]);
-            amax = fmaxf(amax, fabsf(h[f]));
+          for (int c = 0; c < 32; ++c) give[c * 32 + lane] = __fmul_rn(__uint_as_float(other[c]), alpha);
+        }
+        named_bar_sync(2 + pair, 64);
+        const int cb = c_lo + (is_gate ? 0 : 32);   // first tile column handled here
+        if (live && cb < t.n_rows) {
+          float hv[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float a = __fmul_rn(__uint_as_float(mine[c]), alpha);
+            const float b = take[c * 32 + lane];
+            const float gv = is_gate ? a : b, uv = is_gate ? b : a;
+            hv[c] = __fmul_rn(silu_fast(gv), uv);
           }
-          amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-          if (c0 + j < t.n_rows) {
-            const GroupScale gs = nvfp4_group_scale(amax, p.g_next[t.e]);
-            const uint2 o = make_uint2(nvfp4_word(h, gs.inv), nvfp4_word(h + 8, gs.inv));
-            const int64_t prow = (int64_t)p.pad_offsets[t.e] + n;
-            const int fb = 64 * t.mt + 32 * g;  // first feature of this group
+          // group amax of each token column over the warp's 32 features (lanes)
+          float my_amax = 0.0f;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const uint32_t r = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(hv[c])));
+            if (lane == c) my_amax = __uint_as_float(r);
+          }
+          const GroupScale gs = nvfp4_group_scale(my_amax, p.g_next[t.e]);  // lane c: column c
+          const int fb = 64 * t.mt + 32 * (q & 1);  // first feature of the group
+          const int64_t prow0 = (int64_t)p.pad_offsets[t.e] + t.nt * BN + cb;
+          uint8_t* codes = (uint8_t*)p.out;
+          const int nvalid = t.n_rows - cb;        // columns cb + c valid for c < nvalid
+#pragma unroll
+          for (int c4 = 0; c4 < 32; c4 += 4) {
+            float v[4], vp[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float inv = __shfl_sync(0xffffffffu, gs.inv, c4 + u);
+              v[u] = inv == 0.0f ? 0.0f : __fmul_rn(hv[c4 + u], inv);
+              vp[u] = __shfl_xor_sync(0xffffffffu, v[u], 1);
+            }
+            // even lanes: byte u = codes of features (lane, lane+1) of column c4+u
+            const uint32_t w = e2m1x8(v[0], vp[0], v[1], vp[1], v[2], vp[2], v[3], vp[3]);
+            if ((lane & 1) == 0) {
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const int64_t prow = prow0 + c4 + u;
+                if (c4 + u < nvalid && prow < p.P_cap)
+                  codes[prow * (I / 2) + fb / 2 + lane / 2] = (uint8_t)(w >> (8 * u));
+              }
+            }
+          }
+          if (lane < nvalid) {
+            const int64_t prow = prow0 + lane;
             if (prow >= 0 && prow < p.P_cap) {
-              uint8_t* codes = (uint8_t*)p.out;
-              *reinterpret_cast<uint2*>(codes + prow * (I / 2) + fb / 2 + 8 * pp) = o;
-              if (pp == 0) {
-                const int64_t blk = (prow / 128) * (I / 128) + fb / 128;
-                p.out_sf[blk * 512 + sf_block_offset((uint32_t)(prow % 128), (uint32_t)((fb / 32) % 4))] =
-                    (uint8_t)gs.sc;
-              }
+              const int64_t blk = (prow / 128) * (I / 128) + fb / 128;
+              p.out_sf[blk * 512 + sf_block_offset((uint32_t)(prow % 128), (uint32_t)((fb / 32) % 4))] =
+                  (uint8_t)gs.sc;
             }
           }
-        } else {
-          // item: column j, 32 consecutive accumulator rows seg*32 ..
-          const int j = et & 63, seg = et >> 6;
-          const int n = t.nt * BN + c0 + j;
-          const int64_t s = (int64_t)off[t.e] + n;
-          if (c0 + j < t.n_rows && s >= 0 && s < p.S) {
-            int col0;  // first output column of these 32 rows
-            if (p.gate_up) col0 = seg < 2 ? 64 * t.mt + 32 * seg : I + 64 * t.mt + 32 * (seg - 2);
-            else col0 = BM * t.mt + 32 * seg;
-            const float* src = epi + (32 * seg) * EPI_LD + j;
-            if (p.epi == MOESQ_EPI_F32) {
-              float* y = (float*)p.out + s * p.M + col0;
+        }
+        named_bar_sync(2 + pair, 64);  // the exchange block is free for the next tile
+      } else {
+        // row feature of this lane and its output column
+        const int r = 32 * q + lane;
+        int col;
+        if (p.gate_up) col = r < 64 ? 64 * t.mt + r : I + 64 * t.mt + (r - 64);
+        else col = BM * t.mt + r;
+        const int64_t s0 = (int64_t)off[t.e] + t.nt * BN;
 #pragma unroll
-              for (int c = 0; c < 8; ++c)
-                *reinterpret_cast<float4*>(y + 4 * c) =
-                    make_float4(src[(4 * c) * EPI_LD], src[(4 * c + 1) * EPI_LD],
-                                src[(4 * c + 2) * EPI_LD], src[(4 * c + 3) * EPI_LD]);
-            } else {
-              uint16_t* y = (uint16_t*)p.out + s * p.M + col0;
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int cb = c_lo + 32 * h2;
+          uint32_t acc[32];
+          const bool any = cb < t.n_rows;
+          if (any) {
+            tmem_ld_32x32b_x32(tbase + cb, acc);
+            tmem_ld_wait();
+          }
+          if (h2 == 1) {  // both column blocks read: accumulator free
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.acc_empty[buf]);
+          }
+          if (any) {
 #pragma unroll
-              for (int c = 0; c < 4; ++c) {
-                uint32_t w[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-                  w[u] = float_to_bf16_bits(src[(8 * c + 2 * u) * EPI_LD]) |
-                         (float_to_bf16_bits(src[(8 * c + 2 * u + 1) * EPI_LD]) << 16);
-                *reinterpret_cast<uint4*>(y + 8 * c) = make_uint4(w[0], w[1], w[2], w[3]);
+            for (int c = 0; c < 32; ++c) {
+              const int64_t s = s0 + cb + c;
+              if (cb + c < t.n_rows && s < p.S) {
+                const float v = __fmul_rn(__uint_as_float(acc[c]), alpha);
+                if (p.epi == MOESQ_EPI_F32) ((float*)p.out)[s * p.M + col] = v;
+                else ((uint16_t*)p.out)[s * p.M + col] = (uint16_t)float_to_bf16_bits(v);
               }
             }
           }
         }
-        named_bar_sync(1, EPI_THREADS);
       }
       acc_phase[buf] ^= 1;
       buf ^= 1;
