@@ -157,6 +157,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As above, but a thread whose phase is not complete is suspended in hardware
+// until the phase completes or `hint_ns` elapses, instead of spinning (waiting
+// warps then take no issue slots from the warps that do the work).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for the phase of `parity` to complete.  Gives up after
 // `limit_ns` (or at once when *abort is set), setting *abort and the timeout
 // flag; returns false then.  Every pipeline wait in the library goes through it.
@@ -166,8 +182,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   const uint64_t t0 = globaltimer_ns();
   uint32_t it = 0;
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (((++it) & 63u) == 0) {
+    if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
+    if (((++it) & 15u) == 0) {
       if (*abort) return false;
       if (globaltimer_ns() - t0 > limit_ns) {
         *abort = 1;

@@ -378,11 +378,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (p.gate_up) col = r < 64 ? 64 * t.mt + r : I + 64 * t.mt + (r - 64);
         else col = BM * t.mt + r;
         const int64_t s0 = (int64_t)off[t.e] + t.nt * BN;
+        int nvalid = t.n_rows;                     // valid columns of the tile
+        if (s0 + nvalid > p.S) nvalid = (int)(p.S - s0 > 0 ? p.S - s0 : 0);
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
           const int cb = c_lo + 32 * h2;
           uint32_t acc[32];
-          const bool any = cb < t.n_rows;
+          const bool any = cb < nvalid;
           if (any) {
             tmem_ld_32x32b_x32(tbase + cb, acc);
             tmem_ld_wait();
@@ -393,14 +395,17 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (lane == 0) mbar_arrive(&S.acc_empty[buf]);
           }
           if (any) {
+            const int nc = nvalid - cb < 32 ? nvalid - cb : 32;
+            if (p.epi == MOESQ_EPI_F32) {
+              float* yp = (float*)p.out + (s0 + cb) * p.M + col;
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              const int64_t s = s0 + cb + c;
-              if (cb + c < t.n_rows && s < p.S) {
-                const float v = __fmul_rn(__uint_as_float(acc[c]), alpha);
-                if (p.epi == MOESQ_EPI_F32) ((float*)p.out)[s * p.M + col] = v;
-                else ((uint16_t*)p.out)[s * p.M + col] = (uint16_t)float_to_bf16_bits(v);
-              }
+              for (int c = 0; c < 32; ++c)
+                if (c < nc) yp[(size_t)c * p.M] = __fmul_rn(__uint_as_float(acc[c]), alpha);
+            } else {
+              uint16_t* yp = (uint16_t*)p.out + (s0 + cb) * p.M + col;
+#pragma unroll
+              for (int c = 0; c < 32; ++c)
+                if (c < nc) yp[(size_t)c * p.M] = (uint16_t)float_to_bf16_bits(__fmul_rn(__uint_as_float(acc[c]), alpha));
             }
           }
         }
