@@ -62,9 +62,10 @@ __device__ __forceinline__ uint32_t nvfp4_word(const float* v, float inv) {
                 __fmul_rn(v[6], inv), __fmul_rn(v[7], inv));
 }
 
-// silu(x) = x / (1 + exp(-x)) with the fast exponential and reciprocal
+// silu(x) = x / (1 + exp(-x)) with the fast exponential and division (relative
+// error a few ulp; the denominator exceeds 2^126 only where silu rounds to 0)
 __device__ __forceinline__ float silu_fast(float x) {
-  return x * __frcp_rn(1.0f + __expf(-x));
+  return __fdividef(x, 1.0f + __expf(-x));
 }
 
 // E4M3 (finite, saturating) code of a nonnegative float32, nearest-even.

@@ -114,7 +114,7 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __maxnreg__(200)
     k_grouped_gemm_sp(const __grid_constant__ CUtensorMap tmap_a,
                       const __grid_constant__ CUtensorMap tmap_b,
                       const __grid_constant__ CUtensorMap tmap_b32, const Params p) {
@@ -313,7 +313,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.acc_empty[buf]);
         float* give = xch + (is_gate ? 0 : 1) * 1024;
-        const float* take = xch + (is_gate ? 1 : 0) * 1024;
+        const float* take = xch + (is_gate ? 1 : 0) * 1024;  // read here, then reused for the transpose
         if (live) {
 #pragma unroll
           for (int c = 0; c < 32; ++c) give[c * 32 + lane] = __fmul_rn(__uint_as_float(other[c]), alpha);
@@ -321,6 +321,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         named_bar_sync(2 + pair, 64);
         const int cb = c_lo + (is_gate ? 0 : 32);   // first tile column handled here
         if (live && cb < t.n_rows) {
+          // h for feature `lane` x 32 token columns, then a conflict-free transpose
+          // (XOR swizzle) through the block just read, so that each lane owns one
+          // token column's 32-feature group
           float hv[32];
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
@@ -329,41 +332,27 @@ __global__ void __launch_bounds__(THREADS, 1)
             const float gv = is_gate ? a : b, uv = is_gate ? b : a;
             hv[c] = __fmul_rn(silu_fast(gv), uv);
           }
-          // group amax of each token column over the warp's 32 features (lanes)
-          float my_amax = 0.0f;
+          __syncwarp();
+          float* tr = const_cast<float*>(take);
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const uint32_t r = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(hv[c])));
-            if (lane == c) my_amax = __uint_as_float(r);
+          for (int c = 0; c < 32; ++c) tr[c * 32 + (lane ^ c)] = hv[c];
+          __syncwarp();
+          float amax = 0.0f;
+#pragma unroll
+          for (int f = 0; f < 32; ++f) {
+            hv[f] = tr[lane * 32 + (f ^ lane)];   // column `lane`, feature f
+            amax = fmaxf(amax, fabsf(hv[f]));
           }
-          const GroupScale gs = nvfp4_group_scale(my_amax, p.g_next[t.e]);  // lane c: column c
-          const int fb = 64 * t.mt + 32 * (q & 1);  // first feature of the group
-          const int64_t prow0 = (int64_t)p.pad_offsets[t.e] + t.nt * BN + cb;
-          uint8_t* codes = (uint8_t*)p.out;
-          const int nvalid = t.n_rows - cb;        // columns cb + c valid for c < nvalid
-#pragma unroll
-          for (int c4 = 0; c4 < 32; c4 += 4) {
-            float v[4], vp[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float inv = __shfl_sync(0xffffffffu, gs.inv, c4 + u);
-              v[u] = inv == 0.0f ? 0.0f : __fmul_rn(hv[c4 + u], inv);
-              vp[u] = __shfl_xor_sync(0xffffffffu, v[u], 1);
-            }
-            // even lanes: byte u = codes of features (lane, lane+1) of column c4+u
-            const uint32_t w = e2m1x8(v[0], vp[0], v[1], vp[1], v[2], vp[2], v[3], vp[3]);
-            if ((lane & 1) == 0) {
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const int64_t prow = prow0 + c4 + u;
-                if (c4 + u < nvalid && prow < p.P_cap)
-                  codes[prow * (I / 2) + fb / 2 + lane / 2] = (uint8_t)(w >> (8 * u));
-              }
-            }
-          }
+          const int nvalid = t.n_rows - cb;
           if (lane < nvalid) {
-            const int64_t prow = prow0 + lane;
+            const GroupScale gs = nvfp4_group_scale(amax, p.g_next[t.e]);
+            const int fb = 64 * t.mt + 32 * (q & 1);  // first feature of the group
+            const int64_t prow = (int64_t)p.pad_offsets[t.e] + t.nt * BN + cb + lane;
             if (prow >= 0 && prow < p.P_cap) {
+              uint8_t* codes = (uint8_t*)p.out;
+              *reinterpret_cast<uint4*>(codes + prow * (I / 2) + fb / 2) =
+                  make_uint4(nvfp4_word(hv, gs.inv), nvfp4_word(hv + 8, gs.inv),
+                             nvfp4_word(hv + 16, gs.inv), nvfp4_word(hv + 24, gs.inv));
               const int64_t blk = (prow / 128) * (I / 128) + fb / 128;
               p.out_sf[blk * 512 + sf_block_offset((uint32_t)(prow % 128), (uint32_t)((fb / 32) % 4))] =
                   (uint8_t)gs.sc;
