@@ -45,7 +45,9 @@ constexpr int EPI_BYTES = 4 * 2 * 32 * 32 * 4;  // SwiGLU gate/up exchange block
 constexpr int MAX_E = 1024;
 constexpr int EPI_WARPS = 8;
 constexpr int EPI_THREADS = 32 * EPI_WARPS;
-constexpr int THREADS = 64 + EPI_THREADS;   // producer warp, MMA warp, epilogue warps
+// producer warp, MMA warp, epilogue warps.  10 warps put 3 on two SM sub-partitions,
+// whose 16K-register slices then cap a thread at 168 registers.
+constexpr int THREADS = 64 + EPI_THREADS;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_ACC = 0, TM_E = 256, TM_SFA = 264, TM_SFB = 272;
 
@@ -114,7 +116,7 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(THREADS, 1)
     k_grouped_gemm_sp(const __grid_constant__ CUtensorMap tmap_a,
                       const __grid_constant__ CUtensorMap tmap_b,
                       const __grid_constant__ CUtensorMap tmap_b32, const Params p) {
