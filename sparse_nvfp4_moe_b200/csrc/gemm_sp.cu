@@ -41,7 +41,7 @@ constexpr int B_BYTES = BN * BK / 2;       // token codes: 128 B per row (SW128)
 constexpr int E_BYTES = BM * 16;           // metadata: 16 B per row
 constexpr int SF_BYTES = 2 * 512;          // two 512-byte scale blocks
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + E_BYTES + 2 * SF_BYTES;  // 28672
-constexpr int EPI_BYTES = 4 * 2 * 32 * 32 * 4;  // SwiGLU gate/up exchange blocks (4 warp pairs)
+constexpr int EPI_BYTES = 8 * 32 * 32 * 4;  // one 32x32 fp32 block per epilogue warp (exchange/transpose)
 constexpr int MAX_E = 1024;
 constexpr int EPI_WARPS = 8;
 constexpr int EPI_THREADS = 32 * EPI_WARPS;
@@ -116,6 +116,7 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+template <int EPI>
 __global__ void __launch_bounds__(THREADS, 1)
     k_grouped_gemm_sp(const __grid_constant__ CUtensorMap tmap_a,
                       const __grid_constant__ CUtensorMap tmap_b,
@@ -302,7 +303,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t tbase = tmem + TM_ACC + buf * BN + ((uint32_t)(32 * q) << 16);
       const int c_lo = 64 * hh;                 // first column of this warp's half
       const bool live = c_lo < t.n_rows;        // any valid token column in the half
-      if (p.epi == MOESQ_EPI_SWIGLU_NVFP4) {
+      if constexpr (EPI == MOESQ_EPI_SWIGLU_NVFP4) {
         const bool is_gate = q < 2;
         // gate warp finishes columns [c_lo, c_lo+32), up warp [c_lo+32, c_lo+64)
         uint32_t mine[32], other[32];
@@ -363,15 +364,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         named_bar_sync(2 + pair, 64);  // the exchange block is free for the next tile
       } else {
-        // row feature of this lane and its output column
-        const int r = 32 * q + lane;
-        int col;
-        if (p.gate_up) col = r < 64 ? 64 * t.mt + r : I + 64 * t.mt + (r - 64);
-        else col = BM * t.mt + r;
+        // per 32x32 block: TMEM (lane = feature) -> swizzled transpose in this
+        // warp's shared block -> lane = token, 32 consecutive output features:
+        // one 64-byte (bf16) or 128-byte (f32) row segment per lane
+        float* tr = epi + ew * 1024;
+        const int col0 = p.gate_up ? (q < 2 ? 64 * t.mt + 32 * q : I + 64 * t.mt + 32 * (q - 2))
+                                   : BM * t.mt + 32 * q;
         const int64_t s0 = (int64_t)off[t.e] + t.nt * BN;
         int nvalid = t.n_rows;                     // valid columns of the tile
         if (s0 + nvalid > p.S) nvalid = (int)(p.S - s0 > 0 ? p.S - s0 : 0);
-#pragma unroll
+#pragma unroll 1
         for (int h2 = 0; h2 < 2; ++h2) {
           const int cb = c_lo + 32 * h2;
           uint32_t acc[32];
@@ -386,18 +388,38 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (lane == 0) mbar_arrive(&S.acc_empty[buf]);
           }
           if (any) {
-            const int nc = nvalid - cb < 32 ? nvalid - cb : 32;
-            if (p.epi == MOESQ_EPI_F32) {
-              float* yp = (float*)p.out + (s0 + cb) * p.M + col;
 #pragma unroll
-              for (int c = 0; c < 32; ++c)
-                if (c < nc) yp[(size_t)c * p.M] = __fmul_rn(__uint_as_float(acc[c]), alpha);
-            } else {
-              uint16_t* yp = (uint16_t*)p.out + (s0 + cb) * p.M + col;
+            for (int c = 0; c < 32; ++c) tr[c * 32 + (lane ^ c)] = __uint_as_float(acc[c]);
+            __syncwarp();
+            if (lane < nvalid - cb) {
+              const int64_t s = s0 + cb + lane;
+              if constexpr (EPI == MOESQ_EPI_F32) {
+                float4* y = reinterpret_cast<float4*>((float*)p.out + s * p.M + col0);
+                const float* row = tr + lane * 32;
+#pragma unroll 1
+                for (int u = 0; u < 8; ++u) {
+                  float v[4];
 #pragma unroll
-              for (int c = 0; c < 32; ++c)
-                if (c < nc) yp[(size_t)c * p.M] = (uint16_t)float_to_bf16_bits(__fmul_rn(__uint_as_float(acc[c]), alpha));
+                  for (int z = 0; z < 4; ++z) v[z] = __fmul_rn(row[(4 * u + z) ^ lane], alpha);
+                  y[u] = make_float4(v[0], v[1], v[2], v[3]);
+                }
+              } else {
+                uint4* y = reinterpret_cast<uint4*>((uint16_t*)p.out + s * p.M + col0);
+                const float* row = tr + lane * 32;
+#pragma unroll 1
+                for (int u = 0; u < 4; ++u) {
+                  uint32_t w[4];
+#pragma unroll
+                  for (int z = 0; z < 4; ++z) {
+                    const float a = __fmul_rn(row[(8 * u + 2 * z) ^ lane], alpha);
+                    const float b = __fmul_rn(row[(8 * u + 2 * z + 1) ^ lane], alpha);
+                    w[z] = float_to_bf16_bits(a) | (float_to_bf16_bits(b) << 16);
+                  }
+                  y[u] = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+              }
             }
+            __syncwarp();
           }
         }
       }
@@ -521,8 +543,12 @@ extern "C" moesq_status moesq_grouped_gemm(const moesq_linear* W, const uint8_t*
 
   static int attr_done[64] = {0};
   if (dev < 64 && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(sp::k_grouped_gemm_sp, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)sp::SMEM_BYTES) != cudaSuccess)
+    if (cudaFuncSetAttribute(sp::k_grouped_gemm_sp<MOESQ_EPI_F32>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(sp::k_grouped_gemm_sp<MOESQ_EPI_BF16>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(sp::k_grouped_gemm_sp<MOESQ_EPI_SWIGLU_NVFP4>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp::SMEM_BYTES) != cudaSuccess)
       return MOESQ_ERR_CUDA;
     attr_done[dev] = 1;
   }
@@ -545,7 +571,17 @@ extern "C" moesq_status moesq_grouped_gemm(const moesq_linear* W, const uint8_t*
   prm.gate_up = gate_up ? 1 : 0;
   prm.S = S;
   prm.P_cap = P_cap;
-  sp::k_grouped_gemm_sp<<<sms, sp::THREADS, sp::SMEM_BYTES, (cudaStream_t)stream>>>(ta, tb, tb32, prm);
+  cudaStream_t st = (cudaStream_t)stream;
+  switch (epilogue) {
+    case MOESQ_EPI_F32:
+      sp::k_grouped_gemm_sp<MOESQ_EPI_F32><<<sms, sp::THREADS, sp::SMEM_BYTES, st>>>(ta, tb, tb32, prm);
+      break;
+    case MOESQ_EPI_BF16:
+      sp::k_grouped_gemm_sp<MOESQ_EPI_BF16><<<sms, sp::THREADS, sp::SMEM_BYTES, st>>>(ta, tb, tb32, prm);
+      break;
+    default:
+      sp::k_grouped_gemm_sp<MOESQ_EPI_SWIGLU_NVFP4><<<sms, sp::THREADS, sp::SMEM_BYTES, st>>>(ta, tb, tb32, prm);
+  }
   MOESQ_CHECK_LAUNCH();
   return MOESQ_OK;
 }
