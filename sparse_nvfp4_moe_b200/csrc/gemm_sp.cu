@@ -373,20 +373,20 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int64_t s0 = (int64_t)off[t.e] + t.nt * BN;
         int nvalid = t.n_rows;                     // valid columns of the tile
         if (s0 + nvalid > p.S) nvalid = (int)(p.S - s0 > 0 ? p.S - s0 : 0);
-#pragma unroll 1
+        // both 32-column blocks are read before one wait, then the accumulator is
+        // released to the MMA warp before any conversion or store
+        uint32_t accs[2][32];
+        if (c_lo < nvalid) tmem_ld_32x32b_x32(tbase + c_lo, accs[0]);
+        if (c_lo + 32 < nvalid) tmem_ld_32x32b_x32(tbase + c_lo + 32, accs[1]);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.acc_empty[buf]);
+#pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
           const int cb = c_lo + 32 * h2;
-          uint32_t acc[32];
+          const uint32_t* acc = accs[h2];
           const bool any = cb < nvalid;
-          if (any) {
-            tmem_ld_32x32b_x32(tbase + cb, acc);
-            tmem_ld_wait();
-          }
-          if (h2 == 1) {  // both column blocks read: accumulator free
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&S.acc_empty[buf]);
-          }
           if (any) {
 #pragma unroll
             for (int c = 0; c < 32; ++c) tr[c * 32 + (lane ^ c)] = __uint_as_float(acc[c]);
