@@ -204,7 +204,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const bool b32 = t.n_rows <= 32;
         const uint32_t b_bytes = b32 ? 32 * 128 : B_BYTES;
         for (int kb = 0; kb < nkb; ++kb) {
-          mbar_wait(&S.empty[stage], phase ^ 1, abort, p.d_status);
+          mbar_wait_spin(&S.empty[stage], phase ^ 1, abort, p.d_status);
           const int nk = (kb128 - 2 * kb) >= 2 ? 2 : 1;
           uint8_t* st = smem + stage * STAGE_BYTES;
           mbar_arrive_expect_tx(&S.full[stage], A_BYTES + b_bytes + E_BYTES + 2 * nk * 512);
@@ -248,7 +248,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         mbar_wait(&S.acc_empty[buf], acc_phase[buf] ^ 1, abort, p.d_status);
         tc_fence_after();
         for (int kb = 0; kb < nkb; ++kb) {
-          mbar_wait(&S.full[stage], phase, abort, p.d_status);
+          mbar_wait_spin(&S.full[stage], phase, abort, p.d_status);
           tc_fence_after();
           const int nk = (kb128 - 2 * kb) >= 2 ? 2 : 1;
           const uint32_t st = smem_u32(smem + stage * STAGE_BYTES);
