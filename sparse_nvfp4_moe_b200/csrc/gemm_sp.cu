@@ -239,6 +239,16 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t phase = 0;
       uint32_t acc_phase[2] = {0u, 0u};
       int buf = 0;
+      // Shared-memory descriptors of stage 0; a stage (or a K offset inside it)
+      // only moves the 14-bit start-address field, so every later descriptor is
+      // one add.  All stage addresses stay below 256 KB, so the field never carries.
+      const uint32_t s0 = smem_u32(smem);
+      const uint64_t dA0 = smem_desc(s0, 16, 512, SWZ_64B);
+      const uint64_t dB0 = smem_desc(s0 + A_BYTES, 16, 1024, SWZ_128B);
+      const uint64_t dE0 = smem_desc(s0 + A_BYTES + B_BYTES, 16, 128, SWZ_NONE);
+      const uint64_t dSFA0 = smem_desc(s0 + A_BYTES + B_BYTES + E_BYTES, 16, 128, SWZ_NONE);
+      const uint64_t dSFB0 = dSFA0 + (SF_BYTES >> 4);
+      const uint32_t tE = tmem + TM_E, tSFA = tmem + TM_SFA, tSFB = tmem + TM_SFB;
       for (int id = blockIdx.x; id < total; id += gridDim.x) {
         const Tile t = decode_tile(S, id, MT, E, off);
         int n_mma = (t.n_rows + 15) / 16 * 16;
@@ -249,22 +259,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
         for (int kb = 0; kb < nkb; ++kb) {
           mbar_wait_spin(&S.full[stage], phase, abort, p.d_status);
-          tc_fence_after();
-          const int nk = (kb128 - 2 * kb) >= 2 ? 2 : 1;
-          const uint32_t st = smem_u32(smem + stage * STAGE_BYTES);
-          const uint32_t sA = st, sB = st + A_BYTES, sE = sB + B_BYTES, sSFA = sE + E_BYTES,
-                         sSFB = sSFA + SF_BYTES;
-          tc_cp_128x128b(tmem + TM_E, smem_desc(sE, 16, 128, SWZ_NONE));
-          for (int kk = 0; kk < nk; ++kk) {
-            tc_cp_32x128b_warpx4(tmem + TM_SFA + 4 * kk, smem_desc(sSFA + 512 * kk, 16, 128, SWZ_NONE));
-            tc_cp_32x128b_warpx4(tmem + TM_SFB + 4 * kk, smem_desc(sSFB + 512 * kk, 16, 128, SWZ_NONE));
-          }
-          for (int kk = 0; kk < nk; ++kk) {
-            const uint64_t adesc = smem_desc(sA + 32 * kk, 16, 512, SWZ_64B);
-            const uint64_t bdesc = smem_desc(sB + 64 * kk, 16, 1024, SWZ_128B);
-            tc_mma_sp_nvf4(d_tmem, adesc, bdesc, tmem + TM_E + 2 * kk, idesc,
-                           tmem + TM_SFA + 4 * kk, tmem + TM_SFB + 4 * kk,
-                           (kb > 0 || kk > 0) ? 1u : 0u);
+          const uint64_t so = (uint64_t)((stage * STAGE_BYTES) >> 4);
+          tc_cp_128x128b(tE, dE0 + so);
+          tc_cp_32x128b_warpx4(tSFA, dSFA0 + so);
+          tc_cp_32x128b_warpx4(tSFB, dSFB0 + so);
+          tc_mma_sp_nvf4(d_tmem, dA0 + so, dB0 + so, tE, idesc, tSFA, tSFB, kb > 0 ? 1u : 0u);
+          if (2 * kb + 1 < kb128) {  // second 128-deep K block of the stage
+            tc_cp_32x128b_warpx4(tSFA + 4, dSFA0 + so + (512 >> 4));
+            tc_cp_32x128b_warpx4(tSFB + 4, dSFB0 + so + (512 >> 4));
+            tc_mma_sp_nvf4(d_tmem, dA0 + so + (32 >> 4), dB0 + so + (64 >> 4), tE + 2, idesc, tSFA + 4,
+                           tSFB + 4, 1u);
           }
           tc_commit(&S.empty[stage]);
           if (++stage == STAGES) {
