@@ -67,8 +67,12 @@ struct Params {
   int64_t S, P_cap;
 };
 
+static_assert(STAGES % 2 == 0, "stages are released to the producer in pairs");
+
 struct Smem {
-  uint64_t full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], done;
+  // full[s]: stage s landed.  empty[s/2]: both stages of pair s/2 consumed (one
+  // tcgen05.commit per pair halves the commits, the costliest issue step).
+  uint64_t full[STAGES], empty[STAGES / 2], acc_full[2], acc_empty[2], done;
   uint32_t tmem_base;
   int abort;
   int tile_start[MAX_E + 1];
@@ -133,10 +137,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   // ---- set-up: barriers, tile prefix, TMEM
   if (threadIdx.x == 0) {
-    for (int i = 0; i < STAGES; ++i) {
-      mbar_init(&S.full[i], 1);
-      mbar_init(&S.empty[i], 1);
-    }
+    for (int i = 0; i < STAGES; ++i) mbar_init(&S.full[i], 1);
+    for (int i = 0; i < STAGES / 2; ++i) mbar_init(&S.empty[i], 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.acc_full[i], 1);
       mbar_init(&S.acc_empty[i], EPI_WARPS);
@@ -204,7 +206,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const bool b32 = t.n_rows <= 32;
         const uint32_t b_bytes = b32 ? 32 * 128 : B_BYTES;
         for (int kb = 0; kb < nkb; ++kb) {
-          mbar_wait_spin(&S.empty[stage], phase ^ 1, abort, p.d_status);
+          if ((stage & 1) == 0) mbar_wait_spin(&S.empty[stage >> 1], phase ^ 1, abort, p.d_status);
           const int nk = (kb128 - 2 * kb) >= 2 ? 2 : 1;
           uint8_t* st = smem + stage * STAGE_BYTES;
           mbar_arrive_expect_tx(&S.full[stage], A_BYTES + b_bytes + E_BYTES + 2 * nk * 512);
@@ -270,7 +272,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc_mma_sp_nvf4(d_tmem, dA0 + so + (32 >> 4), dB0 + so + (64 >> 4), tE + 2, idesc, tSFA + 4,
                            tSFB + 4, 1u);
           }
-          tc_commit(&S.empty[stage]);
+          if (stage & 1) tc_commit(&S.empty[stage >> 1]);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
