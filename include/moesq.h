@@ -68,7 +68,9 @@ typedef enum moesq_status {
   MOESQ_ERR_CUDA = 4,              /* a CUDA runtime/driver call failed (launch, tensor map) */
   MOESQ_ERR_TIMEOUT = 5,           /* reserved for callers that translate MOESQ_DFLAG_TIMEOUT */
   MOESQ_ERR_WORKSPACE = 6,         /* workspace pointer NULL or smaller than required */
-  MOESQ_ERR_DEVICE = 7             /* current device is not sm_100 */
+  MOESQ_ERR_DEVICE = 7,            /* current device is not sm_100 */
+  MOESQ_ERR_CAPACITY = 8           /* request larger than the fixed scratch of an
+                                      allocation-free entry point */
 } moesq_status;
 
 /* bits OR-ed into *d_status by the device */
@@ -178,6 +180,30 @@ moesq_status moesq_permute(const int32_t* topk_ids, int64_t T, int32_t k, int32_
                            int32_t* token_slot, void* ws, size_t ws_bytes, int32_t* d_status,
                            moesq_stream_t stream);
 moesq_status moesq_permute_workspace_size(int64_t T, int32_t k, int32_t E, size_t* bytes);
+
+/* Allocation-free variant of moesq_permute (the pages have no counterpart: this is a
+ * library convenience).  Same arguments, outputs and device flags as moesq_permute,
+ * minus the workspace: its scratch is a fixed 1 MiB array in device memory that the
+ * library declares statically, so it never calls cudaMalloc, cudaFree or any other
+ * allocating routine.  It is for callers that cannot allocate device memory when
+ * they route a batch -- a serving engine that reserves all device memory up front
+ * and forbids later allocations (a late cudaMalloc can fail or stall every stream
+ * on the device), or a plugin interface that hands the kernel only its bound input
+ * and output buffers.
+ *   Limit: ceil(T*k / 1024) * E <= MOESQ_PERMUTE_NOALLOC_MAX_COUNTS, else
+ *   MOESQ_ERR_CAPACITY is returned and nothing is enqueued (e.g. E = 512 allows
+ *   T*k up to 524288).
+ *   The first call on a device looks up the array's device address with that device
+ *   current (cudaGetSymbolAddress) and caches it; make that first call before any
+ *   stream capture.  Every GPU that loads the library holds the array until the
+ *   process exits.  All calls share it, and each call overwrites the parts it reads,
+ *   so calls whose executions overlap on the GPU (other streams, other host threads)
+ *   race and must be ordered by the caller. */
+#define MOESQ_PERMUTE_NOALLOC_MAX_COUNTS 262144
+moesq_status moesq_permute_noalloc(const int32_t* topk_ids, int64_t T, int32_t k, int32_t E,
+                                   int32_t* expert_offsets, int32_t* pad_offsets,
+                                   int32_t* slot_token, int32_t* token_slot, int32_t* d_status,
+                                   moesq_stream_t stream);
 
 /* Upper bound of the padded row count for S slots over E experts. */
 int64_t moesq_padded_rows(int64_t S, int32_t E);

@@ -50,6 +50,7 @@ _SIGS = {
     "moesq_permute": (ctypes.c_int, [c_vp, c_i64, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz,
                                      c_vp, c_vp]),
     "moesq_permute_workspace_size": (ctypes.c_int, [c_i64, c_i32, c_i32, ctypes.POINTER(c_sz)]),
+    "moesq_permute_noalloc": (ctypes.c_int, [c_vp, c_i64, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
     "moesq_padded_rows": (c_i64, [c_i64, c_i32]),
     "moesq_unpermute": (ctypes.c_int, [c_vp, c_vp, c_vp, c_i64, c_i32, c_i64, c_vp, c_vp]),
     "moesq_quant_act": (ctypes.c_int, [c_vp, c_i64, c_vp, c_vp, c_vp, c_i32, c_vp, c_i64, c_i32, c_vp,
@@ -181,6 +182,17 @@ def moesq_permute(topk_ids, T, k, E, expert_offsets, pad_offsets, slot_token, to
     _check("moesq_permute", lib().moesq_permute(_p(topk_ids), T, k, E, _p(expert_offsets),
                                                 _p(pad_offsets), _p(slot_token), _p(token_slot),
                                                 _p(ws), ws_bytes, _p(d_status), _stream(stream)))
+
+
+def moesq_permute_noalloc(topk_ids, T, k, E, expert_offsets, pad_offsets, slot_token, token_slot,
+                          d_status=None, stream=None):
+    """moesq_permute without a workspace argument (fixed device scratch; see the header)."""
+    _check("moesq_permute_noalloc", lib().moesq_permute_noalloc(
+        _p(topk_ids), T, k, E, _p(expert_offsets), _p(pad_offsets), _p(slot_token), _p(token_slot),
+        _p(d_status), _stream(stream)))
+
+
+PERMUTE_NOALLOC_MAX_COUNTS = 262144
 
 
 def moesq_unpermute(y, token_slot, topk_w, T, k, H, out, stream=None):

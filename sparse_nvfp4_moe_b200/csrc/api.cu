@@ -64,6 +64,7 @@ extern "C" const char* moesq_status_string(int status) {
     case MOESQ_ERR_TIMEOUT: return "a bounded device wait gave up";
     case MOESQ_ERR_WORKSPACE: return "workspace missing or too small";
     case MOESQ_ERR_DEVICE: return "current device is not sm_100";
+    case MOESQ_ERR_CAPACITY: return "request exceeds the fixed scratch of an allocation-free entry point";
     default: return "unknown status";
   }
 }

@@ -9,6 +9,8 @@
 // place in the padded GEMM operand buffers (pad_offsets).
 #include "common.cuh"
 
+#include <mutex>
+
 namespace moesq {
 
 constexpr int PERM_CHUNK = 1024;   // flattened (token, j) entries per block
@@ -248,5 +250,75 @@ extern "C" moesq_status moesq_unpermute(const uint16_t* y, const int32_t* token_
   if (g > 148 * 16) g = 148 * 16;
   k_unpermute<<<(int)g, 256, 0, (cudaStream_t)stream>>>(y, token_slot, topk_w, T, k, H, out);
   MOESQ_CHECK_LAUNCH();
+  return MOESQ_OK;
+}
+
+// ---------------------------------------------------------------------------
+// moesq_permute_noalloc: moesq_permute for callers that cannot allocate.
+//
+// Its only scratch (the per-chunk expert counts) lives in a fixed file-scope
+// device array, so the caller passes inputs and outputs only.  Every GPU that
+// loads this library keeps the array (1 MiB) until the process exits.  All calls
+// share it: calls whose executions overlap on the GPU (different streams, or
+// different host threads on one device) race on it and must be serialised by
+// the caller.  Every word a call reads is first written by that same call, so
+// nothing needs clearing between calls.
+static __device__ __align__(256) int32_t g_perm_noalloc_scratch[MOESQ_PERMUTE_NOALLOC_MAX_COUNTS];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+int32_t* g_noalloc_ptr[kMaxDevices] = {nullptr};
+
+// Device address of the scratch array for the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up once
+// per device (with that device current) and cached.
+moesq_status noalloc_scratch(int32_t** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOESQ_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MOESQ_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_perm_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      (void)cudaGetLastError();
+      return MOESQ_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = (int32_t*)p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return MOESQ_OK;
+}
+}  // namespace
+
+extern "C" moesq_status moesq_permute_noalloc(const int32_t* topk_ids, int64_t T, int32_t k,
+                                              int32_t E, int32_t* expert_offsets,
+                                              int32_t* pad_offsets, int32_t* slot_token,
+                                              int32_t* token_slot, int32_t* d_status,
+                                              moesq_stream_t stream) {
+  MOESQ_REQUIRE(expert_offsets && pad_offsets, MOESQ_ERR_INVALID_ARG);
+  MOESQ_REQUIRE(T >= 0 && k >= 1 && k <= 32 && E >= 1 && E <= 4096, MOESQ_ERR_INVALID_ARG);
+  const int64_t S = T * k;
+  MOESQ_REQUIRE(S < (1ll << 31), MOESQ_ERR_UNSUPPORTED_SHAPE);
+  MOESQ_REQUIRE(S == 0 || (topk_ids && slot_token && token_slot), MOESQ_ERR_INVALID_ARG);
+  const int64_t nchunks = (S + PERM_CHUNK - 1) / PERM_CHUNK;
+  MOESQ_REQUIRE(nchunks * E <= MOESQ_PERMUTE_NOALLOC_MAX_COUNTS, MOESQ_ERR_CAPACITY);
+  int32_t* counts = nullptr;
+  const moesq_status st = noalloc_scratch(&counts);
+  if (st != MOESQ_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t shm = (size_t)E * sizeof(int32_t);
+  if (nchunks > 0) {
+    k_perm_count<<<(int)nchunks, PERM_THREADS, shm, s>>>(topk_ids, S, E, (int)nchunks, counts,
+                                                        d_status);
+    MOESQ_CHECK_LAUNCH();
+  }
+  k_perm_scan<<<1, PERM_THREADS, shm, s>>>(counts, (int)nchunks, E, expert_offsets, pad_offsets);
+  MOESQ_CHECK_LAUNCH();
+  if (nchunks > 0) {
+    k_perm_scatter<<<(int)nchunks, PERM_THREADS, shm, s>>>(topk_ids, S, k, E, counts,
+                                                           expert_offsets, slot_token, token_slot);
+    MOESQ_CHECK_LAUNCH();
+  }
   return MOESQ_OK;
 }
