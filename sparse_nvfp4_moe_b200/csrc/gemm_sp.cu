@@ -180,11 +180,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (warp == 0) {
     // ================================================================ producer
-    // Lane 0 waits for a free slot and posts the expected bytes; lanes 0..5 then
-    // issue the stage's six copies in parallel (a single thread issuing them one
-    // after another was the pipeline's slowest loop).  A copy may complete before
-    // the expected-bytes arrival: the phase cannot complete before that arrival.
-    {
+    if (elect_one()) {
       int stage = 0;
       uint32_t phase = 0;
       long fills = 0;
@@ -200,7 +196,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         int prow = p.pad_offsets[t.e] + t.nt * BN;
         if (prow < 0 || (int64_t)prow + BN > p.P_cap) {  // inconsistent offsets: stay in bounds
-          if (lane == 0) flag(p.d_status, MOESQ_DFLAG_CAPACITY);
+          flag(p.d_status, MOESQ_DFLAG_CAPACITY);
           prow = 0;
         }
         const uint8_t* meta = p.meta + (size_t)(t.e * MT + t.mt) * nkb * 2048;
@@ -210,30 +206,19 @@ __global__ void __launch_bounds__(THREADS, 1)
         const bool b32 = t.n_rows <= 32;
         const uint32_t b_bytes = b32 ? 32 * 128 : B_BYTES;
         for (int kb = 0; kb < nkb; ++kb) {
+          if ((stage & 1) == 0) mbar_wait_spin(&S.empty[stage >> 1], phase ^ 1, abort, p.d_status);
           const int nk = (kb128 - 2 * kb) >= 2 ? 2 : 1;
           uint8_t* st = smem + stage * STAGE_BYTES;
-          uint64_t* fb = &S.full[stage];
-          if (lane == 0) {
-            if ((stage & 1) == 0) mbar_wait_spin(&S.empty[stage >> 1], phase ^ 1, abort, p.d_status);
-            mbar_arrive_expect_tx(fb, A_BYTES + b_bytes + E_BYTES + 2 * nk * 512);
-          }
-          __syncwarp();
-          switch (lane) {
-            case 0: tma_load_2d(st, &tmap_a, kb * 64, r0, fb); break;
-            case 1: tma_load_2d(st + A_BYTES / 2, &tmap_a, kb * 64, r1, fb); break;
-            case 2:
-              tma_load_2d(st + A_BYTES, b32 ? (const void*)&tmap_b32 : (const void*)&tmap_b, kb * 128,
-                          prow, fb);
-              break;
-            case 3: bulk_load(st + A_BYTES + B_BYTES, meta + (size_t)kb * 2048, E_BYTES, fb); break;
-            case 4:
-              bulk_load(st + A_BYTES + B_BYTES + E_BYTES, sfa + (size_t)kb * 1024, nk * 512, fb);
-              break;
-            case 5:
-              bulk_load(st + A_BYTES + B_BYTES + E_BYTES + SF_BYTES, sfb + (size_t)kb * 1024, nk * 512, fb);
-              break;
-            default: break;
-          }
+          mbar_arrive_expect_tx(&S.full[stage], A_BYTES + b_bytes + E_BYTES + 2 * nk * 512);
+          tma_load_2d(st, &tmap_a, kb * 64, r0, &S.full[stage]);
+          tma_load_2d(st + A_BYTES / 2, &tmap_a, kb * 64, r1, &S.full[stage]);
+          tma_load_2d(st + A_BYTES, b32 ? (const void*)&tmap_b32 : (const void*)&tmap_b, kb * 128, prow,
+                      &S.full[stage]);
+          bulk_load(st + A_BYTES + B_BYTES, meta + (size_t)kb * 2048, E_BYTES, &S.full[stage]);
+          bulk_load(st + A_BYTES + B_BYTES + E_BYTES, sfa + (size_t)kb * 1024, nk * 512,
+                    &S.full[stage]);
+          bulk_load(st + A_BYTES + B_BYTES + E_BYTES + SF_BYTES, sfb + (size_t)kb * 1024,
+                    nk * 512, &S.full[stage]);
           ++fills;
           if (++stage == STAGES) {
             stage = 0;
@@ -242,15 +227,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       // drain: every slot's last fill must have landed before the CTA exits
-      if (lane == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-          if (fills > s) {
-            const long u = s + (long)STAGES * ((fills - 1 - s) / STAGES);
-            drain_wait(&S.full[s], (uint32_t)((u / STAGES) & 1));
-          }
+      for (int s = 0; s < STAGES; ++s) {
+        if (fills > s) {
+          const long u = s + (long)STAGES * ((fills - 1 - s) / STAGES);
+          drain_wait(&S.full[s], (uint32_t)((u / STAGES) & 1));
         }
       }
-      __syncwarp();
     }
   } else if (warp == 1) {
     // ================================================================ MMA issuer
