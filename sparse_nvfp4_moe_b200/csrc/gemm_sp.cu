@@ -15,10 +15,11 @@
 //     weight tile) work items built on the device from the routing offsets, so
 //     empty experts cost nothing;
 //   * is warp-specialised: warp 0 issues TMA (values and tokens) and bulk copies
-//     (metadata, block scales) into a 6-stage shared-memory ring; warp 1 owns
-//     TMEM, copies metadata and scales smem->TMEM (tcgen05.cp) and issues the
-//     MMAs (dense K = 128 each, two per stage); warps 2..9 drain the
-//     double-buffered FP32 accumulators (tcgen05.ld) while the next tile runs;
+//     (metadata, block scales) into a 3-stage shared-memory ring of 512-deep K
+//     blocks; warp 1 owns TMEM, copies metadata and scales smem->TMEM
+//     (tcgen05.cp) and issues the MMAs (dense K = 128 each, four per stage);
+//     warps 2..9 drain the double-buffered FP32 accumulators (tcgen05.ld) while
+//     the next tile runs;
 //   * fuses the epilogue: FP32 or bf16 output per slot, or SwiGLU followed by
 //     NVFP4 requantisation written straight into the next GEMM's B operand
 //     layout (codes + 512-byte scale blocks).
@@ -34,13 +35,18 @@ namespace sp {
 
 constexpr int BM = 128;           // weight rows per tile
 constexpr int BN = 128;           // max tokens per tile
-constexpr int BK = 256;           // dense K per pipeline stage (two MMAs)
-constexpr int STAGES = 6;
-constexpr int A_BYTES = BM * BK / 4;       // compressed values: 64 B per row (SW64)
-constexpr int B_BYTES = BN * BK / 2;       // token codes: 128 B per row (SW128)
-constexpr int E_BYTES = BM * 16;           // metadata: 16 B per row
-constexpr int SF_BYTES = 2 * 512;          // two 512-byte scale blocks
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES + E_BYTES + 2 * SF_BYTES;  // 28672
+// A pipeline stage covers 512 dense K: four MMAs.  Every copy instruction costs
+// the single issuing thread about the same whatever its size, so a stage is
+// moved by few, large copies: one TMA for the weight tile, two for the token
+// tile, one bulk copy each for metadata and the two scale blocks.
+constexpr int BK = 512;
+constexpr int STAGES = 3;
+constexpr int A_BYTES = BM * BK / 4;       // compressed values: 128 B per row (SW128)
+constexpr int B_CHUNK = BN * 128;          // 256 dense K of token codes: 128 B per row (SW128)
+constexpr int B_BYTES = 2 * B_CHUNK;
+constexpr int E_BYTES = 2 * BM * 16;       // metadata: 16 B per row per 256 dense K
+constexpr int SF_BYTES = 4 * 512;          // one 512-byte scale block per 128 dense K
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + E_BYTES + 2 * SF_BYTES;  // 57344
 constexpr int EPI_BYTES = 8 * 32 * 32 * 4;  // one 32x32 fp32 block per epilogue warp (exchange/transpose)
 constexpr int MAX_E = 1024;
 constexpr int EPI_WARPS = 8;
@@ -49,7 +55,7 @@ constexpr int EPI_THREADS = 32 * EPI_WARPS;
 // whose 16K-register slices then cap a thread at 168 registers.
 constexpr int THREADS = 64 + EPI_THREADS;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TM_ACC = 0, TM_E = 256, TM_SFA = 264, TM_SFB = 272;
+constexpr uint32_t TM_ACC = 0, TM_E = 256, TM_SFA = 264, TM_SFB = 280;
 
 struct Params {
   const uint8_t* meta;
@@ -67,18 +73,21 @@ struct Params {
   int64_t S, P_cap;
 };
 
-static_assert(STAGES % 2 == 0, "stages are released to the producer in pairs");
-
 struct Smem {
-  // full[s]: stage s landed.  empty[s/2]: both stages of pair s/2 consumed (one
-  // tcgen05.commit per pair halves the commits, the costliest issue step).
-  uint64_t full[STAGES], empty[STAGES / 2], acc_full[2], acc_empty[2], done;
+  // full[s]: stage s landed.  empty[s]: stage s consumed by the tensor core.
+  uint64_t full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], done;
   uint32_t tmem_base;
   int abort;
+  // per-expert tables, read from global memory once at set-up so that no role
+  // waits on a global load between tiles: first token tile of each expert,
+  // routed-slot offsets, padded-row offsets
   int tile_start[MAX_E + 1];
+  int eoff[MAX_E + 1];
+  int epad[MAX_E];
 };
 
 constexpr size_t SMEM_BYTES = 1024 /*align*/ + (size_t)STAGES * STAGE_BYTES + EPI_BYTES + sizeof(Smem);
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 
 __device__ __forceinline__ uint32_t make_idesc(uint32_t n) {
   return (1u << 2)            // sparse
@@ -93,8 +102,7 @@ struct Tile {
   int e, nt, mt, n_rows;
 };
 
-__device__ __forceinline__ Tile decode_tile(const Smem& s, int id, int MT, int E,
-                                            const int32_t* __restrict__ off) {
+__device__ __forceinline__ Tile decode_tile(const Smem& s, int id, int MT, int E) {
   Tile t;
   const int q = id / MT;
   t.mt = id % MT;
@@ -106,7 +114,7 @@ __device__ __forceinline__ Tile decode_tile(const Smem& s, int id, int MT, int E
   }
   t.e = lo;
   t.nt = q - s.tile_start[lo];
-  const int te = off[lo + 1] - off[lo];
+  const int te = s.eoff[lo + 1] - s.eoff[lo];
   const int r = te - t.nt * BN;
   t.n_rows = r < BN ? r : BN;
   return t;
@@ -137,8 +145,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   // ---- set-up: barriers, tile prefix, TMEM
   if (threadIdx.x == 0) {
-    for (int i = 0; i < STAGES; ++i) mbar_init(&S.full[i], 1);
-    for (int i = 0; i < STAGES / 2; ++i) mbar_init(&S.empty[i], 1);
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&S.full[i], 1);
+      mbar_init(&S.empty[i], 1);
+    }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.acc_full[i], 1);
       mbar_init(&S.acc_empty[i], EPI_WARPS);
@@ -167,6 +177,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     if (lane == 0) S.tile_start[E] = run;
   }
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+    S.eoff[e] = off[e];
+    if (e < E) S.epad[e] = p.pad_offsets[e];
+  }
   if (warp == 1) {
     tmem_alloc(&S.tmem_base, TMEM_COLS);
     tmem_relinquish();
@@ -184,41 +198,38 @@ __global__ void __launch_bounds__(THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       long fills = 0;
+      const int nkb256 = (p.K + 255) / 256;
       for (int id = blockIdx.x; id < total; id += gridDim.x) {
-        const Tile t = decode_tile(S, id, MT, E, off);
-        int r0, r1;
-        if (p.gate_up) {
-          r0 = t.e * p.M + 64 * t.mt;
-          r1 = t.e * p.M + p.M / 2 + 64 * t.mt;
-        } else {
-          r0 = t.e * p.M + BM * t.mt;
-          r1 = r0 + 64;
-        }
-        int prow = p.pad_offsets[t.e] + t.nt * BN;
+        const Tile t = decode_tile(S, id, MT, E);
+        int prow = S.epad[t.e] + t.nt * BN;
         if (prow < 0 || (int64_t)prow + BN > p.P_cap) {  // inconsistent offsets: stay in bounds
           flag(p.d_status, MOESQ_DFLAG_CAPACITY);
           prow = 0;
         }
-        const uint8_t* meta = p.meta + (size_t)(t.e * MT + t.mt) * nkb * 2048;
-        const uint8_t* sfa = p.sfw + (size_t)(t.e * MT + t.mt) * kb128 * 512;
+        const size_t wt = (size_t)t.e * MT + t.mt;  // weight tile
+        const uint8_t* meta = p.meta + wt * nkb256 * 2048;
+        const uint8_t* sfa = p.sfw + wt * kb128 * 512;
         const uint8_t* sfb = p.act_sf + (size_t)(prow / 128) * kb128 * 512;
-        // a tile of <= 32 tokens loads a 32-row B box (decode-sized groups)
+        // a tile of <= 32 tokens loads 32-row B boxes (decode-sized groups)
         const bool b32 = t.n_rows <= 32;
-        const uint32_t b_bytes = b32 ? 32 * 128 : B_BYTES;
+        const void* tb = b32 ? (const void*)&tmap_b32 : (const void*)&tmap_b;
+        const uint32_t b_chunk = b32 ? 32 * 128 : B_CHUNK;
         for (int kb = 0; kb < nkb; ++kb) {
-          if ((stage & 1) == 0) mbar_wait_spin(&S.empty[stage >> 1], phase ^ 1, abort, p.d_status);
-          const int nk = (kb128 - 2 * kb) >= 2 ? 2 : 1;
+          mbar_wait_spin(&S.empty[stage], phase ^ 1, abort, p.d_status);
+          const int nk = min(4, kb128 - 4 * kb);  // 128-deep MMAs in this stage
+          const int nc = (nk + 1) >> 1;           // 256-deep chunks in this stage
           uint8_t* st = smem + stage * STAGE_BYTES;
-          mbar_arrive_expect_tx(&S.full[stage], A_BYTES + b_bytes + E_BYTES + 2 * nk * 512);
-          tma_load_2d(st, &tmap_a, kb * 64, r0, &S.full[stage]);
-          tma_load_2d(st + A_BYTES / 2, &tmap_a, kb * 64, r1, &S.full[stage]);
-          tma_load_2d(st + A_BYTES, b32 ? (const void*)&tmap_b32 : (const void*)&tmap_b, kb * 128, prow,
-                      &S.full[stage]);
-          bulk_load(st + A_BYTES + B_BYTES, meta + (size_t)kb * 2048, E_BYTES, &S.full[stage]);
-          bulk_load(st + A_BYTES + B_BYTES + E_BYTES, sfa + (size_t)kb * 1024, nk * 512,
-                    &S.full[stage]);
-          bulk_load(st + A_BYTES + B_BYTES + E_BYTES + SF_BYTES, sfb + (size_t)kb * 1024,
-                    nk * 512, &S.full[stage]);
+          uint64_t* bar = &S.full[stage];
+          mbar_arrive_expect_tx(bar, A_BYTES + nc * (b_chunk + BM * 16) + 2 * nk * 512);
+          // weight tile: gate rows 64mt.. and up rows I+64mt.. in one 4-D box,
+          // or 128 consecutive down rows
+          if (p.gate_up) tma_load_4d(st, &tmap_a, kb * 128, 64 * t.mt, 0, t.e, bar);
+          else tma_load_2d(st, &tmap_a, kb * 128, t.e * p.M + BM * t.mt, bar);
+          tma_load_2d(st + A_BYTES, tb, kb * 256, prow, bar);
+          if (nc > 1) tma_load_2d(st + A_BYTES + B_CHUNK, tb, kb * 256 + 128, prow, bar);
+          bulk_load(st + A_BYTES + B_BYTES, meta + (size_t)kb * 4096, nc * BM * 16, bar);
+          bulk_load(st + A_BYTES + B_BYTES + E_BYTES, sfa + (size_t)kb * 2048, nk * 512, bar);
+          bulk_load(st + A_BYTES + B_BYTES + E_BYTES + SF_BYTES, sfb + (size_t)kb * 2048, nk * 512, bar);
           ++fills;
           if (++stage == STAGES) {
             stage = 0;
@@ -245,14 +256,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       // only moves the 14-bit start-address field, so every later descriptor is
       // one add.  All stage addresses stay below 256 KB, so the field never carries.
       const uint32_t s0 = smem_u32(smem);
-      const uint64_t dA0 = smem_desc(s0, 16, 512, SWZ_64B);
+      const uint64_t dA0 = smem_desc(s0, 16, 1024, SWZ_128B);
       const uint64_t dB0 = smem_desc(s0 + A_BYTES, 16, 1024, SWZ_128B);
       const uint64_t dE0 = smem_desc(s0 + A_BYTES + B_BYTES, 16, 128, SWZ_NONE);
       const uint64_t dSFA0 = smem_desc(s0 + A_BYTES + B_BYTES + E_BYTES, 16, 128, SWZ_NONE);
       const uint64_t dSFB0 = dSFA0 + (SF_BYTES >> 4);
       const uint32_t tE = tmem + TM_E, tSFA = tmem + TM_SFA, tSFB = tmem + TM_SFB;
       for (int id = blockIdx.x; id < total; id += gridDim.x) {
-        const Tile t = decode_tile(S, id, MT, E, off);
+        const Tile t = decode_tile(S, id, MT, E);
         int n_mma = (t.n_rows + 15) / 16 * 16;
         if (n_mma < 16) n_mma = 16;
         const uint32_t idesc = make_idesc((uint32_t)n_mma);
@@ -262,17 +273,23 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int kb = 0; kb < nkb; ++kb) {
           mbar_wait_spin(&S.full[stage], phase, abort, p.d_status);
           const uint64_t so = (uint64_t)((stage * STAGE_BYTES) >> 4);
-          tc_cp_128x128b(tE, dE0 + so);
-          tc_cp_32x128b_warpx4(tSFA, dSFA0 + so);
-          tc_cp_32x128b_warpx4(tSFB, dSFB0 + so);
-          tc_mma_sp_nvf4(d_tmem, dA0 + so, dB0 + so, tE, idesc, tSFA, tSFB, kb > 0 ? 1u : 0u);
-          if (2 * kb + 1 < kb128) {  // second 128-deep K block of the stage
-            tc_cp_32x128b_warpx4(tSFA + 4, dSFA0 + so + (512 >> 4));
-            tc_cp_32x128b_warpx4(tSFB + 4, dSFB0 + so + (512 >> 4));
-            tc_mma_sp_nvf4(d_tmem, dA0 + so + (32 >> 4), dB0 + so + (64 >> 4), tE + 2, idesc, tSFA + 4,
-                           tSFB + 4, 1u);
+          const int nk = min(4, kb128 - 4 * kb);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (j < nk) {
+              // metadata of 256 dense K per copy (MMA j reads columns tE + 2j),
+              // one scale block per MMA and operand
+              if ((j & 1) == 0) tc_cp_128x128b(tE + 2 * j, dE0 + so + (uint64_t)((j >> 1) * (BM * 16 >> 4)));
+              tc_cp_32x128b_warpx4(tSFA + 4 * j, dSFA0 + so + (uint64_t)(j * (512 >> 4)));
+              tc_cp_32x128b_warpx4(tSFB + 4 * j, dSFB0 + so + (uint64_t)(j * (512 >> 4)));
+              // A: +32 B per 128 dense K inside the 128-byte swizzle row; B: 64 B
+              // per 128 dense K inside a 256-deep chunk
+              tc_mma_sp_nvf4(d_tmem, dA0 + so + (uint64_t)(j * 2),
+                             dB0 + so + (uint64_t)((j >> 1) * (B_CHUNK >> 4) + (j & 1) * 4), tE + 2 * j,
+                             idesc, tSFA + 4 * j, tSFB + 4 * j, (kb > 0 || j > 0) ? 1u : 0u);
+            }
           }
-          if (stage & 1) tc_commit(&S.empty[stage >> 1]);
+          tc_commit(&S.empty[stage]);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
@@ -302,7 +319,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int pair = (q & 1) + 2 * hh;  // 0..3
     float* xch = epi + pair * 2 * 32 * 32;  // [2][32 cols][32 lanes]
     for (int id = blockIdx.x; id < total; id += gridDim.x) {
-      const Tile t = decode_tile(S, id, MT, E, off);
+      const Tile t = decode_tile(S, id, MT, E);
       const float alpha = __fmul_rn(p.g_act[t.e], p.alpha_w[t.e]);
       mbar_wait(&S.acc_full[buf], acc_phase[buf], abort, p.d_status);
       tc_fence_after();
@@ -356,7 +373,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (lane < nvalid) {
             const GroupScale gs = nvfp4_group_scale(amax, p.g_next[t.e]);
             const int fb = 64 * t.mt + 32 * (q & 1);  // first feature of the group
-            const int64_t prow = (int64_t)p.pad_offsets[t.e] + t.nt * BN + cb + lane;
+            const int64_t prow = (int64_t)S.epad[t.e] + t.nt * BN + cb + lane;
             if (prow >= 0 && prow < p.P_cap) {
               uint8_t* codes = (uint8_t*)p.out;
               *reinterpret_cast<uint4*>(codes + prow * (I / 2) + fb / 2) =
@@ -376,7 +393,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         float* tr = epi + ew * 1024;
         const int col0 = p.gate_up ? (q < 2 ? 64 * t.mt + 32 * q : I + 64 * t.mt + 32 * (q - 2))
                                    : BM * t.mt + 32 * q;
-        const int64_t s0 = (int64_t)off[t.e] + t.nt * BN;
+        const int64_t s0 = (int64_t)S.eoff[t.e] + t.nt * BN;
         int nvalid = t.n_rows;                     // valid columns of the tile
         if (s0 + nvalid > p.S) nvalid = (int)(p.S - s0 > 0 ? p.S - s0 : 0);
         // both 32-column blocks are read before one wait, then the accumulator is
@@ -464,17 +481,23 @@ static PFN_encodeTiled get_encode_fn() {
   return fn;
 }
 
-static bool make_tmap_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
-                         uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swz) {
+// byte tensor of `rank` dims (innermost first); strides in bytes of dims 1..rank-1
+static bool make_tmap_u8(CUtensorMap* m, const void* base, uint32_t rank, const cuuint64_t* dims,
+                         const cuuint64_t* strides, const cuuint32_t* box, CUtensorMapSwizzle swz) {
   PFN_encodeTiled enc = get_encode_fn();
   if (!enc) return false;
-  cuuint64_t dims[2] = {inner, rows};
-  cuuint64_t strides[1] = {inner};
-  cuuint32_t box[2] = {box_inner, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static bool make_tmap_rows(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                           uint32_t box_inner, uint32_t box_rows) {
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {inner};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  return make_tmap_u8(m, base, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 static int device_sms(int* dev_out) {
@@ -536,15 +559,22 @@ extern "C" moesq_status moesq_grouped_gemm(const moesq_linear* W, const uint8_t*
   if (sms < 0) return MOESQ_ERR_CUDA;
   if (sms == 0) return MOESQ_ERR_DEVICE;
 
+  // Weight tile: 512 dense K = 128 compressed bytes per row.  gate_up tiles take
+  // 64 gate rows and the 64 up rows of the same features: a 4-D view
+  // (byte, row in half, half, expert) loads both halves with one copy.
   CUtensorMap ta, tb, tb32;
-  if (!make_tmap_u8(&ta, W->packed, (uint64_t)(W->K / 4), (uint64_t)(W->E * W->out), 64, 64,
-                    CU_TENSOR_MAP_SWIZZLE_64B))
+  const uint64_t rowA = (uint64_t)(W->K / 4);
+  if (gate_up) {
+    const cuuint64_t dims[4] = {rowA, (uint64_t)(W->out / 2), 2, (uint64_t)W->E};
+    const cuuint64_t strides[3] = {rowA, rowA * (uint64_t)(W->out / 2), rowA * (uint64_t)W->out};
+    const cuuint32_t box[4] = {128, 64, 2, 1};
+    if (!make_tmap_u8(&ta, W->packed, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return MOESQ_ERR_CUDA;
+  } else if (!make_tmap_rows(&ta, W->packed, rowA, (uint64_t)(W->E * W->out), 128, 128)) {
     return MOESQ_ERR_CUDA;
-  if (!make_tmap_u8(&tb, act_codes, (uint64_t)(W->K / 2), (uint64_t)P_cap, 128, 128,
-                    CU_TENSOR_MAP_SWIZZLE_128B))
-    return MOESQ_ERR_CUDA;
-  if (!make_tmap_u8(&tb32, act_codes, (uint64_t)(W->K / 2), (uint64_t)P_cap, 128, 32,
-                    CU_TENSOR_MAP_SWIZZLE_128B))
+  }
+  if (!make_tmap_rows(&tb, act_codes, (uint64_t)(W->K / 2), (uint64_t)P_cap, 128, 128) ||
+      !make_tmap_rows(&tb32, act_codes, (uint64_t)(W->K / 2), (uint64_t)P_cap, 128, 32))
     return MOESQ_ERR_CUDA;
 
   static int attr_done[64] = {0};
