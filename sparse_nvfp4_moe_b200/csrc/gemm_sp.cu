@@ -386,6 +386,46 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         }
         named_bar_sync(2 + pair, 64);  // the exchange block is free for the next tile
+      } else if constexpr (EPI == MOESQ_EPI_BF16) {
+        // lane = feature: scale and round to bf16, write each token's 32 features
+        // (64 B) into the shared staging tile [token][128 tile features]; then the
+        // eight warps copy whole output rows out, 512 contiguous bytes per store
+        // instruction (two 256-byte rows)
+        uint16_t* stg = reinterpret_cast<uint16_t*>(epi);  // 128 x 128 bf16
+        const int64_t s0 = (int64_t)S.eoff[t.e] + t.nt * BN;
+        int nvalid = t.n_rows;
+        if (s0 + nvalid > p.S) nvalid = (int)(p.S - s0 > 0 ? p.S - s0 : 0);
+        uint32_t accs[2][32];
+        if (c_lo < nvalid) tmem_ld_32x32b_x32(tbase + c_lo, accs[0]);
+        if (c_lo + 32 < nvalid) tmem_ld_32x32b_x32(tbase + c_lo + 32, accs[1]);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.acc_empty[buf]);
+        named_bar_sync(1, EPI_THREADS);  // the previous tile's rows have been copied out
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int cb = c_lo + 32 * h2;
+          if (cb < nvalid) {
+            uint16_t* col = stg + 32 * q + lane;
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              col[(cb + c) * 128] = (uint16_t)float_to_bf16_bits(__fmul_rn(__uint_as_float(accs[h2][c]), alpha));
+          }
+        }
+        named_bar_sync(1, EPI_THREADS);  // staging tile complete
+        // rows of this warp: 16ew .. 16ew+15, two per instruction; lanes 0-7 and
+        // 8-15 take the two 128-byte halves of one row (tile features 0-63, 64-127)
+        const int half = (lane >> 3) & 1;
+        const int colh = p.gate_up ? (half ? I + 64 * t.mt : 64 * t.mt) : BM * t.mt + 64 * half;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = 16 * ew + 2 * i + (lane >> 4);
+          if (r < nvalid) {
+            const uint4 v = *reinterpret_cast<const uint4*>(stg + r * 128 + 64 * half + 8 * (lane & 7));
+            *reinterpret_cast<uint4*>((uint16_t*)p.out + (s0 + r) * p.M + colh + 8 * (lane & 7)) = v;
+          }
+        }
       } else {
         // per 32x32 block: TMEM (lane = feature) -> swizzled transpose in this
         // warp's shared block -> lane = token, 32 consecutive output features:

@@ -120,6 +120,21 @@ def test_gate_up_f32_within_tolerance(layer):
     assert (err <= lim).all(), f"max err/lim {np.max(err / lim):.3g} at {np.unravel_index(np.argmax(err / lim), err.shape)}"
 
 
+def test_gate_up_bf16_within_tolerance(layer):
+    """bf16 output of the gate_up GEMM: gate and up halves of a tile land in separate column ranges."""
+    L = layer
+    eo, po, st, ts = L.device_routing()
+    codes, sf = L.device_act(eo, po, st)
+    out = torch.full((L.S, 2 * L.cfg.I), float("nan"), dtype=torch.bfloat16, device="cuda")
+    M.moesq_grouped_gemm(L.dgu.struct, codes, sf, cuda(L.g_in_gu), eo, po, L.S, L.P, M.EPI_BF16, None,
+                         out.view(torch.uint16), None)
+    y = out.float().cpu().numpy().astype(np.float64)
+    lim = TOL * L.bound_gu + bf16_ulp(L.acc_gu) + 1e-30
+    assert np.isfinite(y).all()
+    err = np.abs(y - L.acc_gu)
+    assert (err <= lim).all(), f"max err/lim {np.max(err / lim):.3g}"
+
+
 def test_down_bf16_within_tolerance(layer):
     """down GEMM on NVFP4 activations quantised from a synthetic h (one row per slot)."""
     L = layer
