@@ -6,20 +6,23 @@
 // Blackwell sparse NVFP4 MMA takes one scale per 32 dense K = 16 kept values
 // ("Compression details", same card).  This kernel:
 //
-//   * puts the weights on the sparse operand A of tcgen05.mma.sp (M = 128
-//     weight rows per tile) and the routed tokens of one expert on B (N <= 128),
-//     so the compressed weight bytes are the streamed operand and the weight
-//     values are read exactly as stored (weight_sparse_packed is the compressed
-//     A operand: kept elements in K order);
-//   * is persistent: one CTA per SM walks a static list of (expert, token tile,
-//     weight tile) work items built on the device from the routing offsets, so
-//     empty experts cost nothing;
-//   * is warp-specialised: warp 0 issues TMA (values and tokens) and bulk copies
-//     (metadata, block scales) into a 3-stage shared-memory ring of 512-deep K
-//     blocks; warp 1 owns TMEM, copies metadata and scales smem->TMEM
-//     (tcgen05.cp) and issues the MMAs (dense K = 128 each, four per stage);
-//     warps 2..9 drain the double-buffered FP32 accumulators (tcgen05.ld) while
-//     the next tile runs;
+//   * puts the weights on the sparse operand A of tcgen05.mma.sp and the routed
+//     tokens of one expert on B (N <= 128), so the compressed weight bytes are
+//     the streamed operand and the weight values are read exactly as stored
+//     (weight_sparse_packed is the compressed A operand: kept elements in K order);
+//   * runs on CTA pairs (clusters of 2 on two SMs, cta_group::2): one MMA covers
+//     256 weight rows, 128 per CTA, and each CTA stages only half of the token
+//     tile, which halves the token bytes every SM loads and reads per MMA (the
+//     shared-memory operand reads bound a single-CTA sparse MMA);
+//   * is persistent: each pair walks a static list of (expert, token tile,
+//     weight-tile pair) work items built on the device from the routing
+//     offsets, so empty experts cost nothing;
+//   * is warp-specialised: warp 0 of each CTA issues the TMA copies (values,
+//     tokens, metadata, block scales) into a 4-stage shared-memory ring of
+//     512-deep K blocks; warp 1 of the first CTA copies metadata and scales
+//     smem->TMEM (tcgen05.cp) and issues the MMAs (dense K = 128 each, four per
+//     stage); warps 2..9 of each CTA drain its double-buffered FP32
+//     accumulators (tcgen05.ld) while the next tile runs;
 //   * fuses the epilogue: FP32 or bf16 output per slot, or SwiGLU followed by
 //     NVFP4 requantisation written straight into the next GEMM's B operand
 //     layout (codes + 512-byte scale blocks).
@@ -37,16 +40,16 @@ constexpr int BM = 128;           // weight rows per tile
 constexpr int BN = 128;           // max tokens per tile
 // A pipeline stage covers 512 dense K: four MMAs.  Every copy instruction costs
 // the single issuing thread about the same whatever its size, so a stage is
-// moved by few, large copies: one TMA for the weight tile, two for the token
-// tile, one bulk copy each for metadata and the two scale blocks.
+// moved by few, large copies: one for the weight tile, two for the token tile,
+// one each for metadata and the two scale blocks.
 constexpr int BK = 512;
-constexpr int STAGES = 3;
+constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK / 4;       // compressed values: 128 B per row (SW128)
-constexpr int B_CHUNK = BN * 128;          // 256 dense K of token codes: 128 B per row (SW128)
+constexpr int B_CHUNK = (BN / 2) * 128;    // this CTA's half of the tokens, 256 dense K: 128 B per row (SW128)
 constexpr int B_BYTES = 2 * B_CHUNK;
 constexpr int E_BYTES = 2 * BM * 16;       // metadata: 16 B per row per 256 dense K
 constexpr int SF_BYTES = 4 * 512;          // one 512-byte scale block per 128 dense K
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES + E_BYTES + 2 * SF_BYTES;  // 57344
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + E_BYTES + 2 * SF_BYTES;  // 40960
 constexpr int EPI_BYTES = 8 * 32 * 32 * 4;  // one 32x32 fp32 block per epilogue warp (exchange/transpose)
 constexpr int MAX_E = 1024;
 constexpr int EPI_WARPS = 8;
@@ -95,7 +98,7 @@ __device__ __forceinline__ uint32_t make_idesc(uint32_t n) {
          | (1u << 10)         // B: E2M1
          | ((n >> 3) << 17)   // N
          | (0u << 23)         // scale factors UE4M3
-         | ((uint32_t)(BM >> 4) << 24);
+         | ((uint32_t)(2 * BM >> 4) << 24);  // M = 256 over the CTA pair
 }
 
 struct Tile {
@@ -129,36 +132,44 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 }
 
 template <int EPI>
-__global__ void __launch_bounds__(THREADS, 1)
-    k_grouped_gemm_sp(const __grid_constant__ CUtensorMap tmap_a,
-                      const __grid_constant__ CUtensorMap tmap_b,
-                      const __grid_constant__ CUtensorMap tmap_b32, const Params p) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    k_grouped_gemm_sp(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                      const __grid_constant__ CUtensorMap tmap_b16, const __grid_constant__ CUtensorMap tmap_e,
+                      const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
+                      const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   float* epi = (float*)(smem + STAGES * STAGE_BYTES);
   Smem& S = *(Smem*)(smem + STAGES * STAGE_BYTES + EPI_BYTES);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int E = p.E, MT = p.M / BM;
-  const int nkb = (p.K + BK - 1) / BK, kb128 = p.K / 128;
+  const uint32_t rank = cluster_ctarank();  // 0: issues the pair's MMAs
+  const bool lead = rank == 0;
+  const int E = p.E, MT = p.M / BM, MT2 = (MT + 1) / 2;
+  const int nkb = (p.K + BK - 1) / BK, kb128 = p.K / 128, nkb256 = (p.K + 255) / 256;
   const int32_t* off = p.expert_offsets;
+  const int pair_id = blockIdx.x >> 1, npairs = gridDim.x >> 1;
 
-  // ---- set-up: barriers, tile prefix, TMEM
+  // ---- set-up: barriers, tables, TMEM (both CTAs), then a cluster barrier so
+  // that no CTA signals a barrier of its peer before the peer initialised it
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
-      mbar_init(&S.full[i], 1);
-      mbar_init(&S.empty[i], 1);
+      mbar_init(&S.full[i], 1);   // used in CTA 0: its producer's arrival + both CTAs' bytes
+      mbar_init(&S.empty[i], 1);  // one multicast commit per use, in both CTAs
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.acc_full[i], 1);
-      mbar_init(&S.acc_empty[i], EPI_WARPS);
+      mbar_init(&S.acc_empty[i], 2 * EPI_WARPS);  // used in CTA 0: every epilogue warp of the pair
     }
     mbar_init(&S.done, 1);
     S.abort = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmap_a);
     tma_prefetch_desc(&tmap_b);
-    tma_prefetch_desc(&tmap_b32);
+    tma_prefetch_desc(&tmap_b16);
+    tma_prefetch_desc(&tmap_e);
+    tma_prefetch_desc(&tmap_sfa);
+    tma_prefetch_desc(&tmap_sfb);
   }
   if (warp == 0) {  // tile_start[e] = sum over e' < e of ceil(T_e' / BN)
     int run = 0;
@@ -182,54 +193,59 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (e < E) S.epad[e] = p.pad_offsets[e];
   }
   if (warp == 1) {
-    tmem_alloc(&S.tmem_base, TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_pair(&S.tmem_base, TMEM_COLS);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem = S.tmem_base;
-  const int total = S.tile_start[E] * MT;
+  const int total = S.tile_start[E] * MT2;
   volatile int* abort = &S.abort;
 
   if (warp == 0) {
     // ================================================================ producer
+    // Both CTAs load their own weight rows, their half of the token rows and the
+    // full token scale block into their own shared memory; every copy completes
+    // on CTA 0's full barrier, where CTA 0 posts the pair's byte count.
     if (elect_one()) {
       int stage = 0;
       uint32_t phase = 0;
       long fills = 0;
-      const int nkb256 = (p.K + 255) / 256;
-      for (int id = blockIdx.x; id < total; id += gridDim.x) {
-        const Tile t = decode_tile(S, id, MT, E);
+      for (int id = pair_id; id < total; id += npairs) {
+        const Tile t = decode_tile(S, id, MT2, E);
+        const int mt = min(2 * t.mt + (int)rank, MT - 1);  // an odd last tile is loaded twice
         int prow = S.epad[t.e] + t.nt * BN;
         if (prow < 0 || (int64_t)prow + BN > p.P_cap) {  // inconsistent offsets: stay in bounds
           flag(p.d_status, MOESQ_DFLAG_CAPACITY);
           prow = 0;
         }
-        const size_t wt = (size_t)t.e * MT + t.mt;  // weight tile
-        const uint8_t* meta = p.meta + wt * nkb256 * 2048;
-        const uint8_t* sfa = p.sfw + wt * kb128 * 512;
-        const uint8_t* sfb = p.act_sf + (size_t)(prow / 128) * kb128 * 512;
-        // a tile of <= 32 tokens loads 32-row B boxes (decode-sized groups)
-        const bool b32 = t.n_rows <= 32;
-        const void* tb = b32 ? (const void*)&tmap_b32 : (const void*)&tmap_b;
-        const uint32_t b_chunk = b32 ? 32 * 128 : B_CHUNK;
+        const int n_mma = max(16, (t.n_rows + 15) / 16 * 16);
+        const int brow = prow + (int)rank * (n_mma / 2);  // this CTA's half of the token rows
+        const int wt = t.e * MT + mt;                   // weight tile
+        // a tile of <= 32 tokens loads 16-row B boxes (decode-sized groups)
+        const bool small = n_mma <= 32;
+        const void* tb = small ? (const void*)&tmap_b16 : (const void*)&tmap_b;
+        const uint32_t b_box = small ? 16 * 128 : B_CHUNK;
         for (int kb = 0; kb < nkb; ++kb) {
           mbar_wait_spin(&S.empty[stage], phase ^ 1, abort, p.d_status);
           const int nk = min(4, kb128 - 4 * kb);  // 128-deep MMAs in this stage
           const int nc = (nk + 1) >> 1;           // 256-deep chunks in this stage
           uint8_t* st = smem + stage * STAGE_BYTES;
-          uint64_t* bar = &S.full[stage];
-          mbar_arrive_expect_tx(bar, A_BYTES + nc * (b_chunk + BM * 16) + 2 * nk * 512);
+          const uint32_t bar = cluster_map(&S.full[stage], 0);
+          if (lead) mbar_arrive_expect_tx(&S.full[stage], 2u * (A_BYTES + nc * b_box + E_BYTES + 2 * SF_BYTES));
           // weight tile: gate rows 64mt.. and up rows I+64mt.. in one 4-D box,
           // or 128 consecutive down rows
-          if (p.gate_up) tma_load_4d(st, &tmap_a, kb * 128, 64 * t.mt, 0, t.e, bar);
-          else tma_load_2d(st, &tmap_a, kb * 128, t.e * p.M + BM * t.mt, bar);
-          tma_load_2d(st + A_BYTES, tb, kb * 256, prow, bar);
-          if (nc > 1) tma_load_2d(st + A_BYTES + B_CHUNK, tb, kb * 256 + 128, prow, bar);
-          bulk_load(st + A_BYTES + B_BYTES, meta + (size_t)kb * 4096, nc * BM * 16, bar);
-          bulk_load(st + A_BYTES + B_BYTES + E_BYTES, sfa + (size_t)kb * 2048, nk * 512, bar);
-          bulk_load(st + A_BYTES + B_BYTES + E_BYTES + SF_BYTES, sfb + (size_t)kb * 2048, nk * 512, bar);
+          if (p.gate_up) tma_load_4d_pair(st, &tmap_a, kb * 128, 64 * mt, 0, t.e, bar);
+          else tma_load_2d_pair(st, &tmap_a, kb * 128, t.e * p.M + BM * mt, bar);
+          tma_load_2d_pair(st + A_BYTES, tb, kb * 256, brow, bar);
+          if (nc > 1) tma_load_2d_pair(st + A_BYTES + B_CHUNK, tb, kb * 256 + 128, brow, bar);
+          // metadata (2 KB per 256 dense K) and scale blocks (512 B per 128 dense K)
+          // as 256-byte rows; a stage always moves 4 KB + 2 KB + 2 KB
+          tma_load_2d_pair(st + A_BYTES + B_BYTES, &tmap_e, 0, (wt * nkb256 + 2 * kb) * 8, bar);
+          tma_load_2d_pair(st + A_BYTES + B_BYTES + E_BYTES, &tmap_sfa, 0, (wt * kb128 + 4 * kb) * 2, bar);
+          tma_load_2d_pair(st + A_BYTES + B_BYTES + E_BYTES + SF_BYTES, &tmap_sfb, 0,
+                           ((prow / 128) * kb128 + 4 * kb) * 2, bar);
           ++fills;
           if (++stage == STAGES) {
             stage = 0;
@@ -237,24 +253,28 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         }
       }
-      // drain: every slot's last fill must have landed before the CTA exits
+      // drain: CTA 0 waits until every fill of the pair has landed; CTA 1 until
+      // the tensor core has consumed (hence received) its last fill of each slot
       for (int s = 0; s < STAGES; ++s) {
         if (fills > s) {
           const long u = s + (long)STAGES * ((fills - 1 - s) / STAGES);
-          drain_wait(&S.full[s], (uint32_t)((u / STAGES) & 1));
+          const uint32_t par = (uint32_t)((u / STAGES) & 1);
+          if (lead) drain_wait(&S.full[s], par);
+          else drain_wait(&S.empty[s], par);
         }
       }
     }
+    __syncwarp();
   } else if (warp == 1) {
-    // ================================================================ MMA issuer
-    if (elect_one()) {
+    // ================================================================ MMA issuer (CTA 0)
+    if (lead && elect_one()) {
       int stage = 0;
       uint32_t phase = 0;
       uint32_t acc_phase[2] = {0u, 0u};
       int buf = 0;
-      // Shared-memory descriptors of stage 0; a stage (or a K offset inside it)
-      // only moves the 14-bit start-address field, so every later descriptor is
-      // one add.  All stage addresses stay below 256 KB, so the field never carries.
+      // Shared-memory descriptors of stage 0 (the same offsets hold the peer's
+      // operands); a stage or a K offset only moves the 14-bit start-address
+      // field, and all stage addresses stay below 256 KB, so it never carries.
       const uint32_t s0 = smem_u32(smem);
       const uint64_t dA0 = smem_desc(s0, 16, 1024, SWZ_128B);
       const uint64_t dB0 = smem_desc(s0 + A_BYTES, 16, 1024, SWZ_128B);
@@ -262,16 +282,16 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint64_t dSFA0 = smem_desc(s0 + A_BYTES + B_BYTES + E_BYTES, 16, 128, SWZ_NONE);
       const uint64_t dSFB0 = dSFA0 + (SF_BYTES >> 4);
       const uint32_t tE = tmem + TM_E, tSFA = tmem + TM_SFA, tSFB = tmem + TM_SFB;
-      for (int id = blockIdx.x; id < total; id += gridDim.x) {
-        const Tile t = decode_tile(S, id, MT, E);
-        int n_mma = (t.n_rows + 15) / 16 * 16;
-        if (n_mma < 16) n_mma = 16;
+      for (int id = pair_id; id < total; id += npairs) {
+        const Tile t = decode_tile(S, id, MT2, E);
+        const int n_mma = max(16, (t.n_rows + 15) / 16 * 16);
         const uint32_t idesc = make_idesc((uint32_t)n_mma);
         const uint32_t d_tmem = tmem + TM_ACC + buf * BN;
-        mbar_wait(&S.acc_empty[buf], acc_phase[buf] ^ 1, abort, p.d_status);
+        mbar_wait_spin(&S.acc_empty[buf], acc_phase[buf] ^ 1, abort, p.d_status);
         tc_fence_after();
         for (int kb = 0; kb < nkb; ++kb) {
           mbar_wait_spin(&S.full[stage], phase, abort, p.d_status);
+          tc_fence_after();
           const uint64_t so = (uint64_t)((stage * STAGE_BYTES) >> 4);
           const int nk = min(4, kb128 - 4 * kb);
 #pragma unroll
@@ -279,28 +299,28 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (j < nk) {
               // metadata of 256 dense K per copy (MMA j reads columns tE + 2j),
               // one scale block per MMA and operand
-              if ((j & 1) == 0) tc_cp_128x128b(tE + 2 * j, dE0 + so + (uint64_t)((j >> 1) * (BM * 16 >> 4)));
-              tc_cp_32x128b_warpx4(tSFA + 4 * j, dSFA0 + so + (uint64_t)(j * (512 >> 4)));
-              tc_cp_32x128b_warpx4(tSFB + 4 * j, dSFB0 + so + (uint64_t)(j * (512 >> 4)));
+              if ((j & 1) == 0) tc_cp_pair_128x128b(tE + 2 * j, dE0 + so + (uint64_t)((j >> 1) * (BM * 16 >> 4)));
+              tc_cp_pair_32x128b_warpx4(tSFA + 4 * j, dSFA0 + so + (uint64_t)(j * (512 >> 4)));
+              tc_cp_pair_32x128b_warpx4(tSFB + 4 * j, dSFB0 + so + (uint64_t)(j * (512 >> 4)));
               // A: +32 B per 128 dense K inside the 128-byte swizzle row; B: 64 B
               // per 128 dense K inside a 256-deep chunk
-              tc_mma_sp_nvf4(d_tmem, dA0 + so + (uint64_t)(j * 2),
-                             dB0 + so + (uint64_t)((j >> 1) * (B_CHUNK >> 4) + (j & 1) * 4), tE + 2 * j,
-                             idesc, tSFA + 4 * j, tSFB + 4 * j, (kb > 0 || j > 0) ? 1u : 0u);
+              tc_mma_pair_sp_nvf4(d_tmem, dA0 + so + (uint64_t)(j * 2),
+                                  dB0 + so + (uint64_t)((j >> 1) * (B_CHUNK >> 4) + (j & 1) * 4), tE + 2 * j,
+                                  idesc, tSFA + 4 * j, tSFB + 4 * j, (kb > 0 || j > 0) ? 1u : 0u);
             }
           }
-          tc_commit(&S.empty[stage]);
+          tc_commit_pair_mc(&S.empty[stage], 0x3);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
-        tc_commit(&S.acc_full[buf]);
+        tc_commit_pair_mc(&S.acc_full[buf], 0x3);
         acc_phase[buf] ^= 1;
         buf ^= 1;
       }
-      // drain: all tensor-core work of this CTA complete before TMEM is freed
-      tc_commit(&S.done);
+      // drain: all tensor-core work of the pair complete before TMEM is freed
+      tc_commit_pair_mc(&S.done, 0x1);
       drain_wait(&S.done, 0);
     }
     __syncwarp();
@@ -308,20 +328,30 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ================================================================ epilogue
     // 8 warps, two per TMEM lane quarter q (rows 32q..32q+31); warp half hh owns
     // token columns [64hh, 64hh+64).  Lane = accumulator row = output feature.
+    // Each CTA drains its own 128 rows of the pair's accumulator.
     const int ew = warp - 2;            // 0..7
     const int q = warp & 3;             // TMEM lane quarter this warp may access
     const int hh = ew >> 2;             // column half
     uint32_t acc_phase[2] = {0u, 0u};
     int buf = 0;
     const int I = p.M / 2;
+    // accumulator buffer released to CTA 0's MMA warp: a local arrive in CTA 0,
+    // a remote one from CTA 1
+    const uint32_t acc_empty_lead0 = cluster_map(&S.acc_empty[0], 0), acc_empty_lead1 = cluster_map(&S.acc_empty[1], 0);
+    auto release_acc = [&](int b) {
+      if (lead) mbar_arrive(&S.acc_empty[b]);
+      else mbar_arrive_remote(b ? acc_empty_lead1 : acc_empty_lead0);
+    };
     // SwiGLU exchange: gate quarter q (0,1) pairs with up quarter q+2 on the same
     // column half; each side hands the other a 32x32 block (column-major, lane-fast).
     const int pair = (q & 1) + 2 * hh;  // 0..3
     float* xch = epi + pair * 2 * 32 * 32;  // [2][32 cols][32 lanes]
-    for (int id = blockIdx.x; id < total; id += gridDim.x) {
-      const Tile t = decode_tile(S, id, MT, E);
+    for (int id = pair_id; id < total; id += npairs) {
+      const Tile t = decode_tile(S, id, MT2, E);
+      const int mt = 2 * t.mt + (int)rank;  // this CTA's weight tile
+      const bool own_tile = mt < MT;          // false: the duplicate of an odd last tile
       const float alpha = __fmul_rn(p.g_act[t.e], p.alpha_w[t.e]);
-      mbar_wait(&S.acc_full[buf], acc_phase[buf], abort, p.d_status);
+      mbar_wait_poll(&S.acc_full[buf], acc_phase[buf], abort, p.d_status);
       tc_fence_after();
       const uint32_t tbase = tmem + TM_ACC + buf * BN + ((uint32_t)(32 * q) << 16);
       const int c_lo = 64 * hh;                 // first column of this warp's half
@@ -337,7 +367,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&S.acc_empty[buf]);
+        if (lane == 0) release_acc(buf);
         float* give = xch + (is_gate ? 0 : 1) * 1024;
         const float* take = xch + (is_gate ? 1 : 0) * 1024;  // read here, then reused for the transpose
         if (live) {
@@ -372,7 +402,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           const int nvalid = t.n_rows - cb;
           if (lane < nvalid) {
             const GroupScale gs = nvfp4_group_scale(amax, p.g_next[t.e]);
-            const int fb = 64 * t.mt + 32 * (q & 1);  // first feature of the group
+            const int fb = 64 * mt + 32 * (q & 1);  // first feature of the group
             const int64_t prow = (int64_t)S.epad[t.e] + t.nt * BN + cb + lane;
             if (prow >= 0 && prow < p.P_cap) {
               uint8_t* codes = (uint8_t*)p.out;
@@ -401,7 +431,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&S.acc_empty[buf]);
+        if (lane == 0) release_acc(buf);
         named_bar_sync(1, EPI_THREADS);  // the previous tile's rows have been copied out
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
@@ -417,22 +447,21 @@ __global__ void __launch_bounds__(THREADS, 1)
         // rows of this warp: 16ew .. 16ew+15, two per instruction; lanes 0-7 and
         // 8-15 take the two 128-byte halves of one row (tile features 0-63, 64-127)
         const int half = (lane >> 3) & 1;
-        const int colh = p.gate_up ? (half ? I + 64 * t.mt : 64 * t.mt) : BM * t.mt + 64 * half;
+        const int colh = p.gate_up ? (half ? I + 64 * mt : 64 * mt) : BM * mt + 64 * half;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int r = 16 * ew + 2 * i + (lane >> 4);
-          if (r < nvalid) {
+          if (own_tile && r < nvalid) {
             const uint4 v = *reinterpret_cast<const uint4*>(stg + r * 128 + 64 * half + 8 * (lane & 7));
             *reinterpret_cast<uint4*>((uint16_t*)p.out + (s0 + r) * p.M + colh + 8 * (lane & 7)) = v;
           }
         }
       } else {
-        // per 32x32 block: TMEM (lane = feature) -> swizzled transpose in this
-        // warp's shared block -> lane = token, 32 consecutive output features:
-        // one 64-byte (bf16) or 128-byte (f32) row segment per lane
+        // f32: per 32x32 block, TMEM (lane = feature) -> swizzled transpose in this
+        // warp's shared block -> lane = token, one 128-byte row segment per lane
         float* tr = epi + ew * 1024;
-        const int col0 = p.gate_up ? (q < 2 ? 64 * t.mt + 32 * q : I + 64 * t.mt + 32 * (q - 2))
-                                   : BM * t.mt + 32 * q;
+        const int col0 = p.gate_up ? (q < 2 ? 64 * mt + 32 * q : I + 64 * mt + 32 * (q - 2))
+                                   : BM * mt + 32 * q;
         const int64_t s0 = (int64_t)S.eoff[t.e] + t.nt * BN;
         int nvalid = t.n_rows;                     // valid columns of the tile
         if (s0 + nvalid > p.S) nvalid = (int)(p.S - s0 > 0 ? p.S - s0 : 0);
@@ -444,7 +473,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&S.acc_empty[buf]);
+        if (lane == 0) release_acc(buf);
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
           const int cb = c_lo + 32 * h2;
@@ -454,32 +483,16 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int c = 0; c < 32; ++c) tr[c * 32 + (lane ^ c)] = __uint_as_float(acc[c]);
             __syncwarp();
-            if (lane < nvalid - cb) {
+            if (own_tile && lane < nvalid - cb) {
               const int64_t s = s0 + cb + lane;
-              if constexpr (EPI == MOESQ_EPI_F32) {
-                float4* y = reinterpret_cast<float4*>((float*)p.out + s * p.M + col0);
-                const float* row = tr + lane * 32;
+              float4* y = reinterpret_cast<float4*>((float*)p.out + s * p.M + col0);
+              const float* row = tr + lane * 32;
 #pragma unroll 1
-                for (int u = 0; u < 8; ++u) {
-                  float v[4];
+              for (int u = 0; u < 8; ++u) {
+                float v[4];
 #pragma unroll
-                  for (int z = 0; z < 4; ++z) v[z] = __fmul_rn(row[(4 * u + z) ^ lane], alpha);
-                  y[u] = make_float4(v[0], v[1], v[2], v[3]);
-                }
-              } else {
-                uint4* y = reinterpret_cast<uint4*>((uint16_t*)p.out + s * p.M + col0);
-                const float* row = tr + lane * 32;
-#pragma unroll 1
-                for (int u = 0; u < 4; ++u) {
-                  uint32_t w[4];
-#pragma unroll
-                  for (int z = 0; z < 4; ++z) {
-                    const float a = __fmul_rn(row[(8 * u + 2 * z) ^ lane], alpha);
-                    const float b = __fmul_rn(row[(8 * u + 2 * z + 1) ^ lane], alpha);
-                    w[z] = float_to_bf16_bits(a) | (float_to_bf16_bits(b) << 16);
-                  }
-                  y[u] = make_uint4(w[0], w[1], w[2], w[3]);
-                }
+                for (int z = 0; z < 4; ++z) v[z] = __fmul_rn(row[(4 * u + z) ^ lane], alpha);
+                y[u] = make_float4(v[0], v[1], v[2], v[3]);
               }
             }
             __syncwarp();
@@ -491,11 +504,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   }
 
+  // no CTA of the pair frees TMEM or exits while its peer may still use it
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
+    tmem_dealloc_pair(tmem, TMEM_COLS);
   }
 }
 
@@ -533,11 +547,11 @@ static bool make_tmap_u8(CUtensorMap* m, const void* base, uint32_t rank, const 
 }
 
 static bool make_tmap_rows(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
-                           uint32_t box_inner, uint32_t box_rows) {
+                           uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swz) {
   const cuuint64_t dims[2] = {inner, rows};
   const cuuint64_t strides[1] = {inner};
   const cuuint32_t box[2] = {box_inner, box_rows};
-  return make_tmap_u8(m, base, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+  return make_tmap_u8(m, base, 2, dims, strides, box, swz);
 }
 
 static int device_sms(int* dev_out) {
@@ -602,31 +616,54 @@ extern "C" moesq_status moesq_grouped_gemm(const moesq_linear* W, const uint8_t*
   // Weight tile: 512 dense K = 128 compressed bytes per row.  gate_up tiles take
   // 64 gate rows and the 64 up rows of the same features: a 4-D view
   // (byte, row in half, half, expert) loads both halves with one copy.
-  CUtensorMap ta, tb, tb32;
+  CUtensorMap ta, tb, tb16, te, tsfa, tsfb;
   const uint64_t rowA = (uint64_t)(W->K / 4);
+  const int64_t MT = W->out / 128, kb128 = W->K / 128, nkb256 = (W->K + 255) / 256;
   if (gate_up) {
     const cuuint64_t dims[4] = {rowA, (uint64_t)(W->out / 2), 2, (uint64_t)W->E};
     const cuuint64_t strides[3] = {rowA, rowA * (uint64_t)(W->out / 2), rowA * (uint64_t)W->out};
     const cuuint32_t box[4] = {128, 64, 2, 1};
     if (!make_tmap_u8(&ta, W->packed, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
       return MOESQ_ERR_CUDA;
-  } else if (!make_tmap_rows(&ta, W->packed, rowA, (uint64_t)(W->E * W->out), 128, 128)) {
+  } else if (!make_tmap_rows(&ta, W->packed, rowA, (uint64_t)(W->E * W->out), 128, 128,
+                             CU_TENSOR_MAP_SWIZZLE_128B)) {
     return MOESQ_ERR_CUDA;
   }
-  if (!make_tmap_rows(&tb, act_codes, (uint64_t)(W->K / 2), (uint64_t)P_cap, 128, 128) ||
-      !make_tmap_rows(&tb32, act_codes, (uint64_t)(W->K / 2), (uint64_t)P_cap, 128, 32))
+  // token codes: a CTA stages 64 (or, for tiles of <= 32 tokens, 16) rows
+  if (!make_tmap_rows(&tb, act_codes, (uint64_t)(W->K / 2), (uint64_t)P_cap, 128, 64,
+                      CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_rows(&tb16, act_codes, (uint64_t)(W->K / 2), (uint64_t)P_cap, 128, 16,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+    return MOESQ_ERR_CUDA;
+  // metadata and scale blocks seen as 256-byte rows (no swizzle: contiguous copies)
+  if (!make_tmap_rows(&te, W->meta, 256, (uint64_t)(W->E * MT * nkb256 * 8), 256, 16,
+                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_tmap_rows(&tsfa, W->sf, 256, (uint64_t)(W->E * MT * kb128 * 2), 256, 8, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_tmap_rows(&tsfb, act_sf, 256, (uint64_t)(P_cap / 128 * kb128 * 2), 256, 8,
+                      CU_TENSOR_MAP_SWIZZLE_NONE))
     return MOESQ_ERR_CUDA;
 
-  static int attr_done[64] = {0};
-  if (dev < 64 && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(sp::k_grouped_gemm_sp<MOESQ_EPI_F32>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp::SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(sp::k_grouped_gemm_sp<MOESQ_EPI_BF16>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp::SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(sp::k_grouped_gemm_sp<MOESQ_EPI_SWIGLU_NVFP4>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp::SMEM_BYTES) != cudaSuccess)
+  // clusters of 2 CTAs, one CTA per SM: as many pairs as the device can hold at once
+  static int pairs_cache[64][3] = {{0}};
+  const int ei = epilogue - MOESQ_EPI_F32;
+  int pairs = dev < 64 ? pairs_cache[dev][ei] : 0;
+  if (pairs == 0) {
+    const void* fn = epilogue == MOESQ_EPI_F32 ? (const void*)sp::k_grouped_gemm_sp<MOESQ_EPI_F32>
+                     : epilogue == MOESQ_EPI_BF16 ? (const void*)sp::k_grouped_gemm_sp<MOESQ_EPI_BF16>
+                                                  : (const void*)sp::k_grouped_gemm_sp<MOESQ_EPI_SWIGLU_NVFP4>;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp::SMEM_BYTES) != cudaSuccess)
       return MOESQ_ERR_CUDA;
-    attr_done[dev] = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(sms & ~1));
+    cfg.blockDim = dim3(sp::THREADS);
+    cfg.dynamicSmemBytes = sp::SMEM_BYTES;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess || n < 1) {
+      (void)cudaGetLastError();
+      return MOESQ_ERR_CUDA;
+    }
+    pairs = n < sms / 2 ? n : sms / 2;
+    if (dev < 64) pairs_cache[dev][ei] = pairs;
   }
   sp::Params prm;
   prm.meta = W->meta;
@@ -648,15 +685,17 @@ extern "C" moesq_status moesq_grouped_gemm(const moesq_linear* W, const uint8_t*
   prm.S = S;
   prm.P_cap = P_cap;
   cudaStream_t st = (cudaStream_t)stream;
+  const dim3 grid((unsigned)(2 * pairs));
   switch (epilogue) {
     case MOESQ_EPI_F32:
-      sp::k_grouped_gemm_sp<MOESQ_EPI_F32><<<sms, sp::THREADS, sp::SMEM_BYTES, st>>>(ta, tb, tb32, prm);
+      sp::k_grouped_gemm_sp<MOESQ_EPI_F32><<<grid, sp::THREADS, sp::SMEM_BYTES, st>>>(ta, tb, tb16, te, tsfa, tsfb, prm);
       break;
     case MOESQ_EPI_BF16:
-      sp::k_grouped_gemm_sp<MOESQ_EPI_BF16><<<sms, sp::THREADS, sp::SMEM_BYTES, st>>>(ta, tb, tb32, prm);
+      sp::k_grouped_gemm_sp<MOESQ_EPI_BF16><<<grid, sp::THREADS, sp::SMEM_BYTES, st>>>(ta, tb, tb16, te, tsfa, tsfb, prm);
       break;
     default:
-      sp::k_grouped_gemm_sp<MOESQ_EPI_SWIGLU_NVFP4><<<sms, sp::THREADS, sp::SMEM_BYTES, st>>>(ta, tb, tb32, prm);
+      sp::k_grouped_gemm_sp<MOESQ_EPI_SWIGLU_NVFP4><<<grid, sp::THREADS, sp::SMEM_BYTES, st>>>(ta, tb, tb16, te, tsfa, tsfb,
+                                                                                              prm);
   }
   MOESQ_CHECK_LAUNCH();
   return MOESQ_OK;
