@@ -50,13 +50,14 @@ constexpr int B_BYTES = 2 * B_CHUNK;
 constexpr int E_BYTES = 2 * BM * 16;       // metadata: 16 B per row per 256 dense K
 constexpr int SF_BYTES = 4 * 512;          // one 512-byte scale block per 128 dense K
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + E_BYTES + 2 * SF_BYTES;  // 40960
-constexpr int EPI_BYTES = 8 * 32 * 32 * 4;  // one 32x32 fp32 block per epilogue warp (exchange/transpose)
+constexpr int EPI_BYTES = 32768;  // epilogue exchange / transpose / staging space
 constexpr int MAX_E = 1024;
-constexpr int EPI_WARPS = 8;
+// Sixteen epilogue warps, four per sub-partition: the epilogue is latency-bound
+// (TMEM loads, shared-memory transposes, MUFU-heavy SiLU), so it wants warps;
+// 18 warps leave 112 registers a thread.
+constexpr int EPI_WARPS = 16;
 constexpr int EPI_THREADS = 32 * EPI_WARPS;
-// producer warp, MMA warp, epilogue warps.  10 warps put 3 on two SM sub-partitions,
-// whose 16K-register slices then cap a thread at 168 registers.
-constexpr int THREADS = 64 + EPI_THREADS;
+constexpr int THREADS = 64 + EPI_THREADS;  // producer warp, MMA warp, epilogue warps
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_ACC = 0, TM_E = 256, TM_SFA = 264, TM_SFB = 280;
 
@@ -87,6 +88,8 @@ struct Smem {
   int tile_start[MAX_E + 1];
   int eoff[MAX_E + 1];
   int epad[MAX_E];
+  float alpha[MAX_E];  // g_act[e] * alpha_w[e]: the accumulator's scale
+  float gnext[MAX_E];  // global scale of the requantised output (SwiGLU epilogue)
 };
 
 constexpr size_t SMEM_BYTES = 1024 /*align*/ + (size_t)STAGES * STAGE_BYTES + EPI_BYTES + sizeof(Smem);
@@ -105,16 +108,16 @@ struct Tile {
   int e, nt, mt, n_rows;
 };
 
-__device__ __forceinline__ Tile decode_tile(const Smem& s, int id, int MT, int E) {
+// Work item `id` -> (expert, token tile, weight tile).  Every role walks its
+// items in increasing order, so the expert is found by stepping `e` forward
+// from the previous item's (tile_start is non-decreasing; empty experts are
+// stepped over).
+__device__ __forceinline__ Tile decode_tile(const Smem& s, int id, int MT, int E, int& e) {
   Tile t;
   const int q = id / MT;
   t.mt = id % MT;
-  int lo = 0, hi = E - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (s.tile_start[mid] <= q) lo = mid;
-    else hi = mid - 1;
-  }
+  while (e + 1 < E && s.tile_start[e + 1] <= q) ++e;
+  const int lo = e;
   t.e = lo;
   t.nt = q - s.tile_start[lo];
   const int te = s.eoff[lo + 1] - s.eoff[lo];
@@ -190,7 +193,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   }
   for (int e = threadIdx.x; e <= E; e += blockDim.x) {
     S.eoff[e] = off[e];
-    if (e < E) S.epad[e] = p.pad_offsets[e];
+    if (e < E) {
+      S.epad[e] = p.pad_offsets[e];
+      S.alpha[e] = __fmul_rn(p.g_act[e], p.alpha_w[e]);
+      S.gnext[e] = p.g_next ? p.g_next[e] : 0.0f;
+    }
   }
   if (warp == 1) {
     tmem_alloc_pair(&S.tmem_base, TMEM_COLS);
@@ -212,8 +219,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       long fills = 0;
+      int e_cur = 0;
       for (int id = pair_id; id < total; id += npairs) {
-        const Tile t = decode_tile(S, id, MT2, E);
+        const Tile t = decode_tile(S, id, MT2, E, e_cur);
         const int mt = min(2 * t.mt + (int)rank, MT - 1);  // an odd last tile is loaded twice
         int prow = S.epad[t.e] + t.nt * BN;
         if (prow < 0 || (int64_t)prow + BN > p.P_cap) {  // inconsistent offsets: stay in bounds
@@ -282,8 +290,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       const uint64_t dSFA0 = smem_desc(s0 + A_BYTES + B_BYTES + E_BYTES, 16, 128, SWZ_NONE);
       const uint64_t dSFB0 = dSFA0 + (SF_BYTES >> 4);
       const uint32_t tE = tmem + TM_E, tSFA = tmem + TM_SFA, tSFB = tmem + TM_SFB;
+      int e_cur = 0;
       for (int id = pair_id; id < total; id += npairs) {
-        const Tile t = decode_tile(S, id, MT2, E);
+        const Tile t = decode_tile(S, id, MT2, E, e_cur);
         const int n_mma = max(16, (t.n_rows + 15) / 16 * 16);
         const uint32_t idesc = make_idesc((uint32_t)n_mma);
         const uint32_t d_tmem = tmem + TM_ACC + buf * BN;
@@ -326,12 +335,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     __syncwarp();
   } else {
     // ================================================================ epilogue
-    // 8 warps, two per TMEM lane quarter q (rows 32q..32q+31); warp half hh owns
-    // token columns [64hh, 64hh+64).  Lane = accumulator row = output feature.
-    // Each CTA drains its own 128 rows of the pair's accumulator.
-    const int ew = warp - 2;            // 0..7
+    // 16 warps, four per TMEM lane quarter q (rows 32q..32q+31); warp k of a
+    // quarter owns token columns [32k, 32k+32).  Lane = accumulator row = output
+    // feature.  Each CTA drains its own 128 rows of the pair's accumulator.
+    const int ew = warp - 2;            // 0..15
     const int q = warp & 3;             // TMEM lane quarter this warp may access
-    const int hh = ew >> 2;             // column half
+    const int kb = ew >> 2;             // column block
+    const int c_lo = 32 * kb;           // first column of this warp's block
     uint32_t acc_phase[2] = {0u, 0u};
     int buf = 0;
     const int I = p.M / 2;
@@ -343,75 +353,77 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       else mbar_arrive_remote(b ? acc_empty_lead1 : acc_empty_lead0);
     };
     // SwiGLU exchange: gate quarter q (0,1) pairs with up quarter q+2 on the same
-    // column half; each side hands the other a 32x32 block (column-major, lane-fast).
-    const int pair = (q & 1) + 2 * hh;  // 0..3
-    float* xch = epi + pair * 2 * 32 * 32;  // [2][32 cols][32 lanes]
+    // column block; each side hands the other a 16x32 block (column-major, lane-fast).
+    const int pair = (q & 1) + 2 * kb;           // 0..7
+    float* xch = epi + pair * 2 * 16 * 32;       // [2][16 cols][32 lanes]
+    int e_cur = 0;
     for (int id = pair_id; id < total; id += npairs) {
-      const Tile t = decode_tile(S, id, MT2, E);
+      const Tile t = decode_tile(S, id, MT2, E, e_cur);
       const int mt = 2 * t.mt + (int)rank;  // this CTA's weight tile
       const bool own_tile = mt < MT;          // false: the duplicate of an odd last tile
-      const float alpha = __fmul_rn(p.g_act[t.e], p.alpha_w[t.e]);
+      const float alpha = S.alpha[t.e];
       mbar_wait_poll(&S.acc_full[buf], acc_phase[buf], abort, p.d_status);
       tc_fence_after();
       const uint32_t tbase = tmem + TM_ACC + buf * BN + ((uint32_t)(32 * q) << 16);
-      const int c_lo = 64 * hh;                 // first column of this warp's half
-      const bool live = c_lo < t.n_rows;        // any valid token column in the half
+      const bool live = c_lo < t.n_rows;        // any valid token column in the block
       if constexpr (EPI == MOESQ_EPI_SWIGLU_NVFP4) {
         const bool is_gate = q < 2;
-        // gate warp finishes columns [c_lo, c_lo+32), up warp [c_lo+32, c_lo+64)
-        uint32_t mine[32], other[32];
+        // gate warp finishes columns [c_lo, c_lo+16), up warp [c_lo+16, c_lo+32)
+        uint32_t mine[16], other[16];
         if (live) {
-          tmem_ld_32x32b_x32(tbase + c_lo + (is_gate ? 0 : 32), mine);
-          tmem_ld_32x32b_x32(tbase + c_lo + (is_gate ? 32 : 0), other);
+          tmem_ld_32x32b_x16(tbase + c_lo + (is_gate ? 16 : 0), other);
+          tmem_ld_32x32b_x16(tbase + c_lo + (is_gate ? 0 : 16), mine);
           tmem_ld_wait();
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) release_acc(buf);
-        float* give = xch + (is_gate ? 0 : 1) * 1024;
-        const float* take = xch + (is_gate ? 1 : 0) * 1024;  // read here, then reused for the transpose
+        float* give = xch + (is_gate ? 0 : 1) * 512;
+        float* take = xch + (is_gate ? 1 : 0) * 512;  // read here, then reused for the transpose
         if (live) {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) give[c * 32 + lane] = __fmul_rn(__uint_as_float(other[c]), alpha);
+          for (int c = 0; c < 16; ++c) give[c * 32 + lane] = __fmul_rn(__uint_as_float(other[c]), alpha);
         }
         named_bar_sync(2 + pair, 64);
-        const int cb = c_lo + (is_gate ? 0 : 32);   // first tile column handled here
+        const int cb = c_lo + (is_gate ? 0 : 16);   // first tile column finished here
         if (live && cb < t.n_rows) {
-          // h for feature `lane` x 32 token columns, then a conflict-free transpose
-          // (XOR swizzle) through the block just read, so that each lane owns one
-          // token column's 32-feature group
-          float hv[32];
+          // h for feature `lane` x 16 token columns, then a conflict-free transpose
+          // (XOR swizzle) through the block just read: lane = (token column
+          // lane&15, feature half lane>>4), 16 features each
+          float hv[16];
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
+          for (int c = 0; c < 16; ++c) {
             const float a = __fmul_rn(__uint_as_float(mine[c]), alpha);
             const float b = take[c * 32 + lane];
             const float gv = is_gate ? a : b, uv = is_gate ? b : a;
             hv[c] = __fmul_rn(silu_fast(gv), uv);
           }
           __syncwarp();
-          float* tr = const_cast<float*>(take);
 #pragma unroll
-          for (int c = 0; c < 32; ++c) tr[c * 32 + (lane ^ c)] = hv[c];
+          for (int c = 0; c < 16; ++c) take[c * 32 + (lane ^ c)] = hv[c];
           __syncwarp();
+          const int tok = lane & 15, fh = lane >> 4;
           float amax = 0.0f;
 #pragma unroll
-          for (int f = 0; f < 32; ++f) {
-            hv[f] = tr[lane * 32 + (f ^ lane)];   // column `lane`, feature f
-            amax = fmaxf(amax, fabsf(hv[f]));
+          for (int i = 0; i < 16; ++i) {
+            const int f = 16 * fh + i;
+            hv[i] = take[tok * 32 + (f ^ tok)];   // token column tok, feature f
+            amax = fmaxf(amax, fabsf(hv[i]));
           }
-          const int nvalid = t.n_rows - cb;
-          if (lane < nvalid) {
-            const GroupScale gs = nvfp4_group_scale(amax, p.g_next[t.e]);
+          amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 16));
+          if (tok < t.n_rows - cb) {
+            const GroupScale gs = nvfp4_group_scale(amax, S.gnext[t.e]);
             const int fb = 64 * mt + 32 * (q & 1);  // first feature of the group
-            const int64_t prow = (int64_t)S.epad[t.e] + t.nt * BN + cb + lane;
+            const int64_t prow = (int64_t)S.epad[t.e] + t.nt * BN + cb + tok;
             if (prow >= 0 && prow < p.P_cap) {
               uint8_t* codes = (uint8_t*)p.out;
-              *reinterpret_cast<uint4*>(codes + prow * (I / 2) + fb / 2) =
-                  make_uint4(nvfp4_word(hv, gs.inv), nvfp4_word(hv + 8, gs.inv),
-                             nvfp4_word(hv + 16, gs.inv), nvfp4_word(hv + 24, gs.inv));
-              const int64_t blk = (prow / 128) * (I / 128) + fb / 128;
-              p.out_sf[blk * 512 + sf_block_offset((uint32_t)(prow % 128), (uint32_t)((fb / 32) % 4))] =
-                  (uint8_t)gs.sc;
+              *reinterpret_cast<uint2*>(codes + prow * (I / 2) + fb / 2 + 8 * fh) =
+                  make_uint2(nvfp4_word(hv, gs.inv), nvfp4_word(hv + 8, gs.inv));
+              if (fh == 0) {
+                const int64_t blk = (prow / 128) * (I / 128) + fb / 128;
+                p.out_sf[blk * 512 + sf_block_offset((uint32_t)(prow % 128), (uint32_t)((fb / 32) % 4))] =
+                    (uint8_t)gs.sc;
+              }
             }
           }
         }
@@ -419,71 +431,67 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       } else if constexpr (EPI == MOESQ_EPI_BF16) {
         // lane = feature: scale and round to bf16, write each token's 32 features
         // (64 B) into the shared staging tile [token][128 tile features]; then the
-        // eight warps copy whole output rows out, 512 contiguous bytes per store
+        // sixteen warps copy whole output rows out, 512 contiguous bytes per store
         // instruction (two 256-byte rows)
         uint16_t* stg = reinterpret_cast<uint16_t*>(epi);  // 128 x 128 bf16
         const int64_t s0 = (int64_t)S.eoff[t.e] + t.nt * BN;
         int nvalid = t.n_rows;
         if (s0 + nvalid > p.S) nvalid = (int)(p.S - s0 > 0 ? p.S - s0 : 0);
-        uint32_t accs[2][32];
-        if (c_lo < nvalid) tmem_ld_32x32b_x32(tbase + c_lo, accs[0]);
-        if (c_lo + 32 < nvalid) tmem_ld_32x32b_x32(tbase + c_lo + 32, accs[1]);
-        tmem_ld_wait();
+        uint32_t acc[32];
+        if (c_lo < nvalid) {
+          tmem_ld_32x32b_x32(tbase + c_lo, acc);
+          tmem_ld_wait();
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) release_acc(buf);
         named_bar_sync(1, EPI_THREADS);  // the previous tile's rows have been copied out
+        if (c_lo < nvalid) {
+          uint16_t* col = stg + 32 * q + lane;
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          const int cb = c_lo + 32 * h2;
-          if (cb < nvalid) {
-            uint16_t* col = stg + 32 * q + lane;
-#pragma unroll
-            for (int c = 0; c < 32; ++c)
-              col[(cb + c) * 128] = (uint16_t)float_to_bf16_bits(__fmul_rn(__uint_as_float(accs[h2][c]), alpha));
-          }
+          for (int c = 0; c < 32; ++c)
+            col[(c_lo + c) * 128] = (uint16_t)float_to_bf16_bits(__fmul_rn(__uint_as_float(acc[c]), alpha));
         }
         named_bar_sync(1, EPI_THREADS);  // staging tile complete
-        // rows of this warp: 16ew .. 16ew+15, two per instruction; lanes 0-7 and
-        // 8-15 take the two 128-byte halves of one row (tile features 0-63, 64-127)
-        const int half = (lane >> 3) & 1;
-        const int colh = p.gate_up ? (half ? I + 64 * mt : 64 * mt) : BM * mt + 64 * half;
+        // 16-byte chunk i of the tile: row i >> 4, half (i >> 3) & 1 (tile features
+        // 0-63 / 64-127), eight bf16 each
+        const int et = threadIdx.x - 64;  // 0..511
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int r = 16 * ew + 2 * i + (lane >> 4);
+        for (int i0 = 0; i0 < 4; ++i0) {
+          const int i = et + EPI_THREADS * i0;
+          const int r = i >> 4, half = (i >> 3) & 1, w = i & 7;
           if (own_tile && r < nvalid) {
-            const uint4 v = *reinterpret_cast<const uint4*>(stg + r * 128 + 64 * half + 8 * (lane & 7));
-            *reinterpret_cast<uint4*>((uint16_t*)p.out + (s0 + r) * p.M + colh + 8 * (lane & 7)) = v;
+            const int colh = p.gate_up ? (half ? I + 64 * mt : 64 * mt) : BM * mt + 64 * half;
+            const uint4 v = *reinterpret_cast<const uint4*>(stg + r * 128 + 64 * half + 8 * w);
+            *reinterpret_cast<uint4*>((uint16_t*)p.out + (s0 + r) * p.M + colh + 8 * w) = v;
           }
         }
       } else {
-        // f32: per 32x32 block, TMEM (lane = feature) -> swizzled transpose in this
-        // warp's shared block -> lane = token, one 128-byte row segment per lane
-        float* tr = epi + ew * 1024;
+        // f32: per 16-column half of the block, TMEM (lane = feature) -> swizzled
+        // transpose in this warp's shared block -> lanes 0-15 = tokens, one
+        // 128-byte row segment each
+        float* tr = epi + ew * 512;
         const int col0 = p.gate_up ? (q < 2 ? 64 * mt + 32 * q : I + 64 * mt + 32 * (q - 2))
                                    : BM * mt + 32 * q;
         const int64_t s0 = (int64_t)S.eoff[t.e] + t.nt * BN;
         int nvalid = t.n_rows;                     // valid columns of the tile
         if (s0 + nvalid > p.S) nvalid = (int)(p.S - s0 > 0 ? p.S - s0 : 0);
-        // both 32-column blocks are read before one wait, then the accumulator is
-        // released to the MMA warp before any conversion or store
-        uint32_t accs[2][32];
-        if (c_lo < nvalid) tmem_ld_32x32b_x32(tbase + c_lo, accs[0]);
-        if (c_lo + 32 < nvalid) tmem_ld_32x32b_x32(tbase + c_lo + 32, accs[1]);
-        tmem_ld_wait();
+        uint32_t acc[32];
+        if (c_lo < nvalid) {
+          tmem_ld_32x32b_x32(tbase + c_lo, acc);
+          tmem_ld_wait();
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) release_acc(buf);
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
-          const int cb = c_lo + 32 * h2;
-          const uint32_t* acc = accs[h2];
-          const bool any = cb < nvalid;
-          if (any) {
+          const int cb = c_lo + 16 * h2;
+          if (cb < nvalid) {
 #pragma unroll
-            for (int c = 0; c < 32; ++c) tr[c * 32 + (lane ^ c)] = __uint_as_float(acc[c]);
+            for (int c = 0; c < 16; ++c) tr[c * 32 + (lane ^ c)] = __uint_as_float(acc[16 * h2 + c]);
             __syncwarp();
-            if (own_tile && lane < nvalid - cb) {
+            if (own_tile && lane < 16 && lane < nvalid - cb) {
               const int64_t s = s0 + cb + lane;
               float4* y = reinterpret_cast<float4*>((float*)p.out + s * p.M + col0);
               const float* row = tr + lane * 32;
