@@ -139,7 +139,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     k_grouped_gemm_sp(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                       const __grid_constant__ CUtensorMap tmap_b16, const __grid_constant__ CUtensorMap tmap_e,
                       const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
-                      const Params p) {
+                      const __grid_constant__ CUtensorMap tmap_y, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   float* epi = (float*)(smem + STAGES * STAGE_BYTES);
@@ -429,11 +429,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
         named_bar_sync(2 + pair, 64);  // the exchange block is free for the next tile
       } else if constexpr (EPI == MOESQ_EPI_BF16) {
-        // lane = feature: scale and round to bf16, write each token's 32 features
-        // (64 B) into the shared staging tile [token][128 tile features]; then the
-        // sixteen warps copy whole output rows out, 512 contiguous bytes per store
-        // instruction (two 256-byte rows)
-        uint16_t* stg = reinterpret_cast<uint16_t*>(epi);  // 128 x 128 bf16
+        // Stage the bf16 tile as two 64-feature halves [128 token rows][128 B] in
+        // the TMA 128-byte swizzle (16-byte chunk j of row r at chunk j ^ (r & 7)),
+        // then write it with two TMA tensor stores (full tiles) or a row-bounded
+        // copy (a ragged last tile of an expert).  Lane = feature: adjacent lanes
+        // swap one value so that each lane stores a bf16 pair of neighbouring
+        // features as one word; even lanes take column c, odd lanes column c + 4,
+        // whose rows fall on the other half of the banks.
+        uint8_t* stg = reinterpret_cast<uint8_t*>(epi);  // 2 x 128 x 128 B
         const int64_t s0 = (int64_t)S.eoff[t.e] + t.nt * BN;
         int nvalid = t.n_rows;
         if (s0 + nvalid > p.S) nvalid = (int)(p.S - s0 > 0 ? p.S - s0 : 0);
@@ -445,25 +448,49 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) release_acc(buf);
-        named_bar_sync(1, EPI_THREADS);  // the previous tile's rows have been copied out
+        if (threadIdx.x == 64) bulk_wait_group_read0();  // the previous tile's stores have read the staging
+        named_bar_sync(1, EPI_THREADS);                  // and every copy of it is done
         if (c_lo < nvalid) {
-          uint16_t* col = stg + 32 * q + lane;
+          const int odd = lane & 1;
+          uint8_t* hb = stg + (q >> 1) * 16384;
+          const int w = 16 * (q & 1) + (lane >> 1);  // feature pair within the 64-feature half
 #pragma unroll
-          for (int c = 0; c < 32; ++c)
-            col[(c_lo + c) * 128] = (uint16_t)float_to_bf16_bits(__fmul_rn(__uint_as_float(acc[c]), alpha));
+          for (int c8 = 0; c8 < 32; c8 += 8) {
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+              const int c = c8 + c4;
+              const float v0 = __fmul_rn(__uint_as_float(acc[c]), alpha);
+              const float v1 = __fmul_rn(__uint_as_float(acc[c + 4]), alpha);
+              const float recv = __shfl_xor_sync(0xffffffffu, odd ? v0 : v1, 1);
+              const float lo = odd ? recv : v0, hi = odd ? v1 : recv;
+              const int row = c_lo + c + 4 * odd;
+              const __nv_bfloat162 pr = __floats2bfloat162_rn(lo, hi);
+              *reinterpret_cast<uint32_t*>(hb + row * 128 + (((w >> 2) ^ (row & 7)) << 4) + ((w & 3) << 2)) =
+                  *reinterpret_cast<const uint32_t*>(&pr);
+            }
+          }
         }
+        fence_proxy_async_smem();
         named_bar_sync(1, EPI_THREADS);  // staging tile complete
-        // 16-byte chunk i of the tile: row i >> 4, half (i >> 3) & 1 (tile features
-        // 0-63 / 64-127), eight bf16 each
-        const int et = threadIdx.x - 64;  // 0..511
+        const int x0 = p.gate_up ? 64 * mt : BM * mt;            // first column of half 0
+        const int x1 = p.gate_up ? I + 64 * mt : BM * mt + 64;   // and of half 1
+        if (own_tile && nvalid == BN) {
+          if (threadIdx.x == 64) {
+            tma_store_2d(&tmap_y, stg, x0, (int32_t)s0);
+            tma_store_2d(&tmap_y, stg + 16384, x1, (int32_t)s0);
+            bulk_commit_group();
+          }
+        } else if (own_tile) {
+          // 16-byte chunk i: row i >> 4, half (i >> 3) & 1, chunk i & 7 of the half row
+          const int et = threadIdx.x - 64;  // 0..511
 #pragma unroll
-        for (int i0 = 0; i0 < 4; ++i0) {
-          const int i = et + EPI_THREADS * i0;
-          const int r = i >> 4, half = (i >> 3) & 1, w = i & 7;
-          if (own_tile && r < nvalid) {
-            const int colh = p.gate_up ? (half ? I + 64 * mt : 64 * mt) : BM * mt + 64 * half;
-            const uint4 v = *reinterpret_cast<const uint4*>(stg + r * 128 + 64 * half + 8 * w);
-            *reinterpret_cast<uint4*>((uint16_t*)p.out + (s0 + r) * p.M + colh + 8 * w) = v;
+          for (int i0 = 0; i0 < 4; ++i0) {
+            const int i = et + EPI_THREADS * i0;
+            const int r = i >> 4, half = (i >> 3) & 1, j = i & 7;
+            if (r < nvalid) {
+              const uint4 v = *reinterpret_cast<const uint4*>(stg + half * 16384 + r * 128 + ((j ^ (r & 7)) << 4));
+              *reinterpret_cast<uint4*>((uint16_t*)p.out + (s0 + r) * p.M + (half ? x1 : x0) + 8 * j) = v;
+            }
           }
         }
       } else {
@@ -512,6 +539,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     }
   }
 
+  if constexpr (EPI == MOESQ_EPI_BF16) {
+    if (threadIdx.x == 64) bulk_wait_group0();  // the last tile's stores are complete
+  }
   // no CTA of the pair frees TMEM or exits while its peer may still use it
   tc_fence_before();
   cluster_sync_all();
@@ -651,6 +681,19 @@ extern "C" moesq_status moesq_grouped_gemm(const moesq_linear* W, const uint8_t*
                       CU_TENSOR_MAP_SWIZZLE_NONE))
     return MOESQ_ERR_CUDA;
 
+  // bf16 output [S rows x out columns]: 64-column x 128-row boxes, 128-byte swizzle
+  CUtensorMap ty = ta;
+  if (epilogue == MOESQ_EPI_BF16) {
+    PFN_encodeTiled enc = get_encode_fn();
+    const cuuint64_t dims[2] = {(uint64_t)W->out, (uint64_t)S};
+    const cuuint64_t strides[1] = {(uint64_t)W->out * 2};
+    const cuuint32_t box[2] = {64, 128}, estr[2] = {1, 1};
+    if (!enc || enc(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return MOESQ_ERR_CUDA;
+  }
+
   // clusters of 2 CTAs, one CTA per SM: as many pairs as the device can hold at once
   static int pairs_cache[64][3] = {{0}};
   const int ei = epilogue - MOESQ_EPI_F32;
@@ -696,14 +739,14 @@ extern "C" moesq_status moesq_grouped_gemm(const moesq_linear* W, const uint8_t*
   const dim3 grid((unsigned)(2 * pairs));
   switch (epilogue) {
     case MOESQ_EPI_F32:
-      sp::k_grouped_gemm_sp<MOESQ_EPI_F32><<<grid, sp::THREADS, sp::SMEM_BYTES, st>>>(ta, tb, tb16, te, tsfa, tsfb, prm);
+      sp::k_grouped_gemm_sp<MOESQ_EPI_F32><<<grid, sp::THREADS, sp::SMEM_BYTES, st>>>(ta, tb, tb16, te, tsfa, tsfb, ty, prm);
       break;
     case MOESQ_EPI_BF16:
-      sp::k_grouped_gemm_sp<MOESQ_EPI_BF16><<<grid, sp::THREADS, sp::SMEM_BYTES, st>>>(ta, tb, tb16, te, tsfa, tsfb, prm);
+      sp::k_grouped_gemm_sp<MOESQ_EPI_BF16><<<grid, sp::THREADS, sp::SMEM_BYTES, st>>>(ta, tb, tb16, te, tsfa, tsfb, ty, prm);
       break;
     default:
       sp::k_grouped_gemm_sp<MOESQ_EPI_SWIGLU_NVFP4><<<grid, sp::THREADS, sp::SMEM_BYTES, st>>>(ta, tb, tb16, te, tsfa, tsfb,
-                                                                                              prm);
+                                                                                              ty, prm);
   }
   MOESQ_CHECK_LAUNCH();
   return MOESQ_OK;
