@@ -248,6 +248,16 @@ __device__ __forceinline__ bool mbar_wait_poll(uint64_t* bar, uint32_t parity, v
   }
 }
 
+// ------------------------------------------------- programmatic launch ----
+// The kernels of the hot path are launched with programmatic stream
+// serialisation: a kernel may be scheduled while its predecessor in the stream
+// is still running, runs its input-independent prologue, and waits in
+// pdl_wait() until the predecessor has completed and its writes are visible.
+// pdl_trigger() lets the successor be scheduled once every CTA of this grid has
+// reached it (or exited).  Launched without the attribute, both are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------- TMA ----
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
@@ -523,3 +533,20 @@ __device__ __forceinline__ bool elect_one() {
   } while (0)
 
 static inline bool moesq_aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+// host: launch `kernel` on `stream` with programmatic stream serialisation
+template <typename... P, typename... A>
+static inline cudaError_t moesq_launch(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem,
+                                       cudaStream_t stream, A&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<A&&>(args)...);
+}

@@ -174,12 +174,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     tma_prefetch_desc(&tmap_sfa);
     tma_prefetch_desc(&tmap_sfb);
   }
+  if (warp == 1) {
+    tmem_alloc_pair(&S.tmem_base, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  // everything above is independent of the inputs; the routing offsets and the
+  // activations are written by the kernels before this one
+  pdl_wait();
+  pdl_trigger();
+  // per-expert tables: one round of parallel global loads
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+    S.eoff[e] = off[e];
+    if (e < E) {
+      S.epad[e] = p.pad_offsets[e];
+      S.alpha[e] = __fmul_rn(p.g_act[e], p.alpha_w[e]);
+      S.gnext[e] = p.g_next ? p.g_next[e] : 0.0f;
+    }
+  }
+  __syncthreads();
   if (warp == 0) {  // tile_start[e] = sum over e' < e of ceil(T_e' / BN)
     int run = 0;
     for (int e0 = 0; e0 < E; e0 += 32) {
       const int e = e0 + lane;
       int v = 0;
-      if (e < E) v = (off[e + 1] - off[e] + BN - 1) / BN;
+      if (e < E) v = (S.eoff[e + 1] - S.eoff[e] + BN - 1) / BN;
       int x = v;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -190,18 +208,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       run += __shfl_sync(0xffffffffu, x, 31);
     }
     if (lane == 0) S.tile_start[E] = run;
-  }
-  for (int e = threadIdx.x; e <= E; e += blockDim.x) {
-    S.eoff[e] = off[e];
-    if (e < E) {
-      S.epad[e] = p.pad_offsets[e];
-      S.alpha[e] = __fmul_rn(p.g_act[e], p.alpha_w[e]);
-      S.gnext[e] = p.g_next ? p.g_next[e] : 0.0f;
-    }
-  }
-  if (warp == 1) {
-    tmem_alloc_pair(&S.tmem_base, TMEM_COLS);
-    tmem_relinquish_pair();
   }
   tc_fence_before();
   cluster_sync_all();
@@ -737,17 +743,23 @@ extern "C" moesq_status moesq_grouped_gemm(const moesq_linear* W, const uint8_t*
   prm.P_cap = P_cap;
   cudaStream_t st = (cudaStream_t)stream;
   const dim3 grid((unsigned)(2 * pairs));
+  cudaError_t err;
   switch (epilogue) {
     case MOESQ_EPI_F32:
-      sp::k_grouped_gemm_sp<MOESQ_EPI_F32><<<grid, sp::THREADS, sp::SMEM_BYTES, st>>>(ta, tb, tb16, te, tsfa, tsfb, ty, prm);
+      err = moesq_launch(sp::k_grouped_gemm_sp<MOESQ_EPI_F32>, grid, dim3(sp::THREADS), sp::SMEM_BYTES, st, ta, tb,
+                         tb16, te, tsfa, tsfb, ty, prm);
       break;
     case MOESQ_EPI_BF16:
-      sp::k_grouped_gemm_sp<MOESQ_EPI_BF16><<<grid, sp::THREADS, sp::SMEM_BYTES, st>>>(ta, tb, tb16, te, tsfa, tsfb, ty, prm);
+      err = moesq_launch(sp::k_grouped_gemm_sp<MOESQ_EPI_BF16>, grid, dim3(sp::THREADS), sp::SMEM_BYTES, st, ta, tb,
+                         tb16, te, tsfa, tsfb, ty, prm);
       break;
     default:
-      sp::k_grouped_gemm_sp<MOESQ_EPI_SWIGLU_NVFP4><<<grid, sp::THREADS, sp::SMEM_BYTES, st>>>(ta, tb, tb16, te, tsfa, tsfb,
-                                                                                              ty, prm);
+      err = moesq_launch(sp::k_grouped_gemm_sp<MOESQ_EPI_SWIGLU_NVFP4>, grid, dim3(sp::THREADS), sp::SMEM_BYTES, st,
+                         ta, tb, tb16, te, tsfa, tsfb, ty, prm);
   }
-  MOESQ_CHECK_LAUNCH();
+  if (err != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MOESQ_ERR_CUDA;
+  }
   return MOESQ_OK;
 }

@@ -27,6 +27,8 @@ __global__ void k_quant_act(const uint16_t* __restrict__ x, int64_t K, const int
                             const int32_t* __restrict__ pad_offsets, int E,
                             const float* __restrict__ g_in, int64_t rows, int layout,
                             uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+  pdl_wait();  // the previous kernel's outputs are complete past here
+  pdl_trigger();
   const int64_t G = K / 32;
   const int64_t n = rows * G;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
@@ -77,6 +79,8 @@ __global__ void k_quant_act_routed(const uint16_t* __restrict__ x, int64_t T, in
                                    const int32_t* __restrict__ pad_offsets, int E,
                                    const float* __restrict__ g_in, uint8_t* __restrict__ codes,
                                    uint8_t* __restrict__ sf) {
+  pdl_wait();  // the previous kernel's outputs are complete past here
+  pdl_trigger();
   const int64_t G = K / 32;
   const int64_t n = T * G;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
@@ -133,10 +137,9 @@ extern "C" moesq_status moesq_quant_act_routed(const uint16_t* x, int64_t T, int
   const int64_t n = T * (K / 32);
   int64_t g = (n + 127) / 128;
   if (g > 148 * 32) g = 148 * 32;
-  k_quant_act_routed<<<(int)g, 128, 0, (cudaStream_t)stream>>>(x, T, K, topk_ids, token_slot, k,
-                                                              expert_offsets, pad_offsets, E, g_in,
-                                                              codes, sf);
-  MOESQ_CHECK_LAUNCH();
+  if (moesq_launch(k_quant_act_routed, dim3((unsigned)g), dim3(128), 0, (cudaStream_t)stream, x, T, K, topk_ids,
+                   token_slot, k, expert_offsets, pad_offsets, E, g_in, codes, sf) != cudaSuccess)
+    return MOESQ_ERR_CUDA;
   return MOESQ_OK;
 }
 
@@ -156,8 +159,8 @@ extern "C" moesq_status moesq_quant_act(const uint16_t* x, int64_t K, const int3
   const int64_t n = rows * (K / 32);
   int64_t g = (n + 127) / 128;
   if (g > 148 * 32) g = 148 * 32;
-  k_quant_act<<<(int)g, 128, 0, (cudaStream_t)stream>>>(x, K, gather, expert_offsets, pad_offsets,
-                                                       E, g_in, rows, layout, codes, sf);
-  MOESQ_CHECK_LAUNCH();
+  if (moesq_launch(k_quant_act, dim3((unsigned)g), dim3(128), 0, (cudaStream_t)stream, x, K, gather, expert_offsets,
+                   pad_offsets, E, g_in, rows, layout, codes, sf) != cudaSuccess)
+    return MOESQ_ERR_CUDA;
   return MOESQ_OK;
 }

@@ -29,6 +29,8 @@ __global__ void __launch_bounds__(PERM_THREADS) k_perm_count(const int32_t* __re
                                                              int64_t S, int E, int nchunks,
                                                              int32_t* __restrict__ counts,
                                                              int32_t* d_status) {
+  pdl_wait();  // the previous kernel's outputs are complete past here
+  pdl_trigger();
   extern __shared__ int32_t hist[];
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
@@ -72,6 +74,8 @@ __global__ void __launch_bounds__(PERM_THREADS) k_perm_scan(int32_t* __restrict_
                                                             int nchunks, int E,
                                                             int32_t* __restrict__ expert_offsets,
                                                             int32_t* __restrict__ pad_offsets) {
+  pdl_wait();  // the previous kernel's outputs are complete past here
+  pdl_trigger();
   extern __shared__ int32_t sm[];
   int32_t* tot = sm;  // [E]
   __shared__ int32_t warp_sums[32];
@@ -127,6 +131,8 @@ __global__ void __launch_bounds__(PERM_THREADS) k_perm_scatter(
     const int32_t* __restrict__ ids, int64_t S, int k, int E, const int32_t* __restrict__ chunk_base,
     const int32_t* __restrict__ expert_offsets, int32_t* __restrict__ slot_token,
     int32_t* __restrict__ token_slot) {
+  pdl_wait();  // the previous kernel's outputs are complete past here
+  pdl_trigger();
   extern __shared__ int32_t run[];  // [E] next free slot of each expert for this chunk
   for (int e = threadIdx.x; e < E; e += blockDim.x)
     run[e] = expert_offsets[e] + chunk_base[(int64_t)e * gridDim.x + blockIdx.x];
@@ -160,6 +166,8 @@ __global__ void __launch_bounds__(PERM_THREADS) k_perm_scatter(
 __global__ void k_unpermute(const uint16_t* __restrict__ y, const int32_t* __restrict__ token_slot,
                             const float* __restrict__ topk_w, int64_t T, int k, int64_t H,
                             uint16_t* __restrict__ out) {
+  pdl_wait();  // the previous kernel's outputs are complete past here
+  pdl_trigger();
   const int64_t vec = H / 8;
   const int64_t n = T * vec;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
@@ -224,15 +232,17 @@ extern "C" moesq_status moesq_permute(const int32_t* topk_ids, int64_t T, int32_
   int32_t* counts = (int32_t*)ws;
   const size_t shm = (size_t)E * sizeof(int32_t);
   if (nchunks > 0) {
-    k_perm_count<<<nchunks, PERM_THREADS, shm, s>>>(topk_ids, S, E, nchunks, counts, d_status);
-    MOESQ_CHECK_LAUNCH();
+    if (moesq_launch(k_perm_count, dim3(nchunks), dim3(PERM_THREADS), shm, s, topk_ids, S, E, nchunks, counts,
+                     d_status) != cudaSuccess)
+      return MOESQ_ERR_CUDA;
   }
-  k_perm_scan<<<1, PERM_THREADS, shm, s>>>(counts, nchunks, E, expert_offsets, pad_offsets);
-  MOESQ_CHECK_LAUNCH();
+  if (moesq_launch(k_perm_scan, dim3(1), dim3(PERM_THREADS), shm, s, counts, nchunks, E, expert_offsets,
+                   pad_offsets) != cudaSuccess)
+    return MOESQ_ERR_CUDA;
   if (nchunks > 0) {
-    k_perm_scatter<<<nchunks, PERM_THREADS, shm, s>>>(topk_ids, S, k, E, counts, expert_offsets,
-                                                       slot_token, token_slot);
-    MOESQ_CHECK_LAUNCH();
+    if (moesq_launch(k_perm_scatter, dim3(nchunks), dim3(PERM_THREADS), shm, s, topk_ids, S, k, E,
+                     (const int32_t*)counts, (const int32_t*)expert_offsets, slot_token, token_slot) != cudaSuccess)
+      return MOESQ_ERR_CUDA;
   }
   return MOESQ_OK;
 }
@@ -248,8 +258,9 @@ extern "C" moesq_status moesq_unpermute(const uint16_t* y, const int32_t* token_
   const int64_t n = T * (H / 8);
   int64_t g = (n + 255) / 256;
   if (g > 148 * 16) g = 148 * 16;
-  k_unpermute<<<(int)g, 256, 0, (cudaStream_t)stream>>>(y, token_slot, topk_w, T, k, H, out);
-  MOESQ_CHECK_LAUNCH();
+  if (moesq_launch(k_unpermute, dim3((unsigned)g), dim3(256), 0, (cudaStream_t)stream, y, token_slot, topk_w, T, k,
+                   H, out) != cudaSuccess)
+    return MOESQ_ERR_CUDA;
   return MOESQ_OK;
 }
 
