@@ -53,6 +53,9 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-slots", type=int, default=2048, help="slots in the CPU-baseline sample")
+    ap.add_argument("--storage", action="store_true",
+                    help="storage benchmark instead: decode / re-encode / repack every expert's "
+                         "pair-bitmask tensors of --config (default kimi_k2 with this flag)")
     return ap.parse_args()
 
 
@@ -535,8 +538,105 @@ def run_reference(args, rank, world):
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+# ------------------------------------------------------ storage benchmark ---
+# bytes per dense element moved by each storage kernel (in + out)
+STORAGE_BYTES = dict(decode=0.25 + 1 / 16 + 0.5,          # packed + mask -> dense codes
+                     encode=0.5 + 1 / 16 + 0.25 + 1 / 16,  # dense codes + mask hint -> packed + mask
+                     repack=1 / 16 + 1 / 32 + 1 / 16 + 1 / 32)  # mask + scales -> metadata + scale blocks
+
+
+def run_storage(args):
+    """Every expert linear of a layer (gate_up and down of all experts) exported to
+    pair-bitmask storage by the library, then per pass: decode to dense NVFP4
+    codes, re-encode (checked bit-exact against the stored bytes) and repack into
+    the GEMM layouts.  value = bytes moved per pass / pass time."""
+    import torch
+
+    import sparse_nvfp4_moe_b200 as M
+    import workloads as W
+    cfg_name = args.config if args.config != "qwen3_30b_a3b" else "kimi_k2"
+    cfg = W.CONFIGS[cfg_name]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    tensors = []
+    split = cfg.split_gate_up_global
+    for which, n_seg, kind in (("gate_up", 2 if split else 1, M.KIND_GATE_UP_SPLIT if split else M.KIND_GATE_UP),
+                               ("down", 1, M.KIND_DOWN)):
+        parts = []
+        for e0 in range(0, cfg.E, 64):
+            w = W.all_expert_weights_bf16(cfg, which, device=dev, experts=range(e0, min(cfg.E, e0 + 64)))
+            parts.append(M.quantize_expert_weights(w, n_seg))
+            del w
+        st = {k: torch.cat([p_[k] for p_ in parts]) for k in ("packed", "mask", "scale", "g_w")}
+        E, out, K = cfg.E, parts[0]["out"], parts[0]["K"]
+        del parts
+        torch.cuda.empty_cache()
+        mb, sb = M.repack_sizes(out, K)
+        u8 = dict(dtype=torch.uint8, device=dev)
+        tensors.append(dict(which=which, kind=kind, E=E, out=out, K=K,
+                            st=st, dense=torch.empty((E * out, K // 2), **u8),
+                            packed2=torch.empty_like(st["packed"]), mask2=torch.empty_like(st["mask"]),
+                            meta=torch.empty(E * mb, **u8), sf=torch.empty(E * sb, **u8),
+                            alpha=torch.empty(E, dtype=torch.float32, device=dev)))
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def op(name):
+        for t in tensors:
+            rows = t["E"] * t["out"]
+            if name == "decode":
+                M.moesq_decode(t["st"]["packed"], t["st"]["mask"], t["dense"], rows, t["K"], status)
+            elif name == "encode":
+                M.moesq_encode(t["dense"], t["st"]["mask"], t["packed2"], t["mask2"], rows, t["K"], status)
+            else:
+                M.moesq_repack_meta(t["st"]["mask"], t["st"]["scale"], t["st"]["g_w"], t["E"], t["out"], t["K"],
+                                    t["kind"], t["meta"], t["sf"], t["alpha"], status)
+
+    n_elem = sum(t["E"] * t["out"] * t["K"] for t in tensors)
+    for _ in range(max(args.warmup, 3)):
+        for name in STORAGE_BYTES:
+            op(name)
+    torch.cuda.synchronize()
+    exact = all(torch.equal(t["packed2"], t["st"]["packed"]) and torch.equal(t["mask2"], t["st"]["mask"])
+                for t in tensors)
+    per = {}
+    with ClockSampler(dev.index) as clk:
+        for name in STORAGE_BYTES:
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+            for a, b in ev:
+                a.record()
+                op(name)
+                b.record()
+            torch.cuda.synchronize()
+            ms = sum(a.elapsed_time(b) for a, b in ev) / len(ev)
+            gb = STORAGE_BYTES[name] * n_elem / 1e9
+            per[name] = {"ms": ms, "GB": gb, "GBps": gb / (ms * 1e-3), "hbm_frac": gb / (ms * 1e-3) / peaks["hbm_gbs"]}
+    clocks = clk.summary()
+    tot_ms = sum(v["ms"] for v in per.values())
+    tot_gb = sum(v["GB"] for v in per.values())
+    # the inputs are resident between passes and larger than L2 (no flush needed)
+    return {"metric": f"pair-bitmask storage decode + re-encode + repack GB/s, all {cfg.E} experts' "
+                      f"gate_up and down ({cfg.name}-shaped, 1 B200)",
+            "value": tot_gb / (tot_ms * 1e-3), "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": tot_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "u8 (E2M1 codes, pair bitmask, E4M3 scales)", "data": "synthetic",
+            "config": {"workload": f"{cfg.name} storage: {cfg.E} experts x (gate_up [{2 * cfg.I},{cfg.H}] + "
+                                   f"down [{cfg.H},{cfg.I}])", "dense_elements": n_elem,
+                       "l2": "not flushed: every pass moves > 10 GB"},
+            "round_trip_bit_exact": bool(exact), "per_op": per,
+            "roofline": {"bound": "hbm", "achieved": tot_gb / (tot_ms * 1e-3), "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": tot_gb / (tot_ms * 1e-3) / peaks["hbm_gbs"], "traffic": None},
+            "device_status": int(status.item()), "clocks": clocks,
+            # per step and tensor: decode 1, encode 1, repack 2 (metadata, scale blocks)
+            "gpu_launches": 4 * len(tensors) * args.steps}
+
+
 def main():
     args = parse_args()
+    if args.storage and args.impl == "ours":
+        print(json.dumps(run_storage(args)))
+        return 0
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

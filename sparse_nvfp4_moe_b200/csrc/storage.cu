@@ -12,9 +12,6 @@
 
 namespace moesq {
 
-// kept byte positions (p0 < p1) of a mask nibble; 0xFF for illegal nibbles
-__constant__ uint8_t c_pos0[16] = {255, 255, 255, 0, 255, 0, 1, 255, 255, 0, 1, 255, 2, 255, 255, 255};
-__constant__ uint8_t c_pos1[16] = {255, 255, 255, 1, 255, 2, 2, 255, 255, 3, 3, 255, 3, 255, 255, 255};
 
 static inline int grid_for(int64_t n, int block) {
   int64_t g = (n + block - 1) / block;
@@ -22,74 +19,127 @@ static inline int grid_for(int64_t n, int block) {
   return (int)(g < cap ? (g > 0 ? g : 1) : cap);
 }
 
+// kept byte positions of a legal mask nibble (exactly two bits set): lowest and
+// highest set bit; legality is popc == 2
+__device__ __forceinline__ bool nib_legal(uint32_t nib) { return __popc(nib) == 2; }
+__device__ __forceinline__ uint32_t nib_lo(uint32_t nib) { return __ffs(nib) - 1; }
+__device__ __forceinline__ uint32_t nib_hi(uint32_t nib) { return 31 - __clz(nib); }
+
+// one mask byte (two chunks) + its 4 packed bytes -> 8 dense bytes
+__device__ __forceinline__ uint2 decode_byte(uint32_t m, uint32_t pk, bool& bad) {
+  uint32_t out[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t nib = (m >> (4 * h)) & 0xF;
+    if (!nib_legal(nib)) {
+      bad = true;
+      out[h] = 0u;
+      continue;
+    }
+    const uint32_t b0 = (pk >> (16 * h)) & 0xFF, b1 = (pk >> (16 * h + 8)) & 0xFF;
+    out[h] = (b0 << (8 * nib_lo(nib))) | (b1 << (8 * nib_hi(nib)));
+  }
+  return make_uint2(out[0], out[1]);
+}
+
 // ------------------------------------------------------------------ decode --
-// thread per mask byte: 4 packed bytes in -> 8 dense bytes out
+// thread per 16 mask bytes: 16 B mask + 64 B packed in -> 128 B dense out (16-byte
+// vector accesses); a tail of < 16 mask bytes one byte per thread
 __global__ void k_decode(const uint8_t* __restrict__ packed, const uint8_t* __restrict__ mask,
                          uint8_t* __restrict__ dense, int64_t nbytes_mask, int32_t* d_status) {
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nbytes_mask;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const uint32_t m = mask[i];
-    const uint32_t pk = *reinterpret_cast<const uint32_t*>(packed + 4 * i);
-    uint32_t out[2] = {0u, 0u};
-    bool bad = false;
+  bool bad = false;
+  const int64_t n16 = nbytes_mask / 16;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n16; i += stride) {
+    const uint4 mv = reinterpret_cast<const uint4*>(mask)[i];
+    const uint32_t mw[4] = {mv.x, mv.y, mv.z, mv.w};
+    const uint4* pk = reinterpret_cast<const uint4*>(packed) + 4 * i;
+    uint4* out = reinterpret_cast<uint4*>(dense) + 8 * i;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const uint32_t nib = (m >> (4 * h)) & 0xF;
-      const uint32_t p0 = c_pos0[nib], p1 = c_pos1[nib];
-      if (p0 == 255) {
-        bad = true;
-        continue;
-      }
-      const uint32_t b0 = (pk >> (16 * h)) & 0xFF, b1 = (pk >> (16 * h + 8)) & 0xFF;
-      out[h] = (b0 << (8 * p0)) | (b1 << (8 * p1));
+    for (int q = 0; q < 4; ++q) {
+      const uint4 pv = pk[q];  // packed bytes of mask word q (4 mask bytes)
+      const uint32_t pw[4] = {pv.x, pv.y, pv.z, pv.w};
+      uint2 d[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) d[j] = decode_byte((mw[q] >> (8 * j)) & 0xFF, pw[j], bad);
+      out[2 * q] = make_uint4(d[0].x, d[0].y, d[1].x, d[1].y);
+      out[2 * q + 1] = make_uint4(d[2].x, d[2].y, d[3].x, d[3].y);
     }
-    if (bad) flag(d_status, MOESQ_DFLAG_BAD_SPARSITY);
-    *reinterpret_cast<uint2*>(dense + 8 * i) = make_uint2(out[0], out[1]);
   }
+  for (int64_t i = 16 * n16 + blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nbytes_mask; i += stride) {
+    const uint2 d = decode_byte(mask[i], *reinterpret_cast<const uint32_t*>(packed + 4 * i), bad);
+    *reinterpret_cast<uint2*>(dense + 8 * i) = d;
+  }
+  if (bad) flag(d_status, MOESQ_DFLAG_BAD_SPARSITY);
 }
 
 // ------------------------------------------------------------------ encode --
+// 8 dense bytes (two chunks) -> 4 packed bytes + 1 mask byte
+// returns (packed word, mask byte)
+__device__ __forceinline__ uint2 encode_byte(uint2 d, uint32_t hm, bool use_hint, bool& bad) {
+  uint32_t mk = 0, pk = 0;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t w = h ? d.y : d.x;
+    uint32_t nz = 0;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) nz |= (((w >> (8 * b)) & 0xFF) != 0) << b;
+    uint32_t nib;
+    if (use_hint) {
+      nib = (hm >> (4 * h)) & 0xF;
+      if (!nib_legal(nib) || (nz & ~nib)) bad = true;
+    } else {
+      nib = nz;
+      if (__popc(nib) > 2) bad = true;
+      // fill up to 2 kept bytes with the lowest-index zero bytes
+#pragma unroll
+      for (int b = 0; b < 4; ++b)
+        if (__popc(nib) < 2 && !((nib >> b) & 1)) nib |= 1u << b;
+    }
+    if (!nib_legal(nib)) nib = 3;  // only reachable when flagged: keep memory-safe output
+    const uint32_t b0 = (w >> (8 * nib_lo(nib))) & 0xFF, b1 = (w >> (8 * nib_hi(nib))) & 0xFF;
+    pk |= (b0 | (b1 << 8)) << (16 * h);
+    mk |= nib << (4 * h);
+  }
+  return make_uint2(pk, mk);
+}
+
+// thread per 16 mask bytes: 128 B dense (+ 16 B hint) in -> 64 B packed + 16 B mask out
 __global__ void k_encode(const uint8_t* __restrict__ dense, const uint8_t* __restrict__ hint,
                          uint8_t* __restrict__ packed, uint8_t* __restrict__ mask,
                          int64_t nbytes_mask, int32_t* d_status) {
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nbytes_mask;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const uint2 d = *reinterpret_cast<const uint2*>(dense + 8 * i);
-    const uint32_t hm = hint ? hint[i] : 0u;
-    uint32_t pk = 0, mk = 0;
-    bool bad = false;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const uint32_t w = h ? d.y : d.x;
-      uint32_t nz = 0;
-#pragma unroll
-      for (int b = 0; b < 4; ++b) nz |= (((w >> (8 * b)) & 0xFF) != 0) << b;
-      uint32_t nib;
-      if (hint) {
-        nib = (hm >> (4 * h)) & 0xF;
-        if (c_pos0[nib] == 255 || (nz & ~nib)) bad = true;
-      } else {
-        nib = nz;
-        if (__popc(nib) > 2) bad = true;
-        // fill up to 2 kept bytes with the lowest-index zero bytes
-#pragma unroll
-        for (int b = 0; b < 4; ++b)
-          if (__popc(nib) < 2 && !((nib >> b) & 1)) nib |= 1u << b;
-      }
-      uint32_t p0 = c_pos0[nib], p1 = c_pos1[nib];
-      if (p0 == 255) {  // only reachable when flagged: keep memory-safe output
-        p0 = 0;
-        p1 = 1;
-        nib = 3;
-      }
-      const uint32_t b0 = (w >> (8 * p0)) & 0xFF, b1 = (w >> (8 * p1)) & 0xFF;
-      pk |= (b0 | (b1 << 8)) << (16 * h);
-      mk |= nib << (4 * h);
+  bool bad = false;
+  const bool use_hint = hint != nullptr;
+  const int64_t n16 = nbytes_mask / 16;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n16; i += stride) {
+    uint32_t hw[4] = {0u, 0u, 0u, 0u};
+    if (use_hint) {
+      const uint4 hv = reinterpret_cast<const uint4*>(hint)[i];
+      hw[0] = hv.x, hw[1] = hv.y, hw[2] = hv.z, hw[3] = hv.w;
     }
-    if (bad) flag(d_status, MOESQ_DFLAG_BAD_SPARSITY);
-    *reinterpret_cast<uint32_t*>(packed + 4 * i) = pk;
-    mask[i] = (uint8_t)mk;
+    const uint4* dv = reinterpret_cast<const uint4*>(dense) + 8 * i;
+    uint4* pk_out = reinterpret_cast<uint4*>(packed) + 4 * i;
+    uint32_t mw[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 a = dv[2 * q], c = dv[2 * q + 1];
+      const uint2 d[4] = {make_uint2(a.x, a.y), make_uint2(a.z, a.w), make_uint2(c.x, c.y), make_uint2(c.z, c.w)};
+      uint2 r[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) r[j] = encode_byte(d[j], (hw[q] >> (8 * j)) & 0xFF, use_hint, bad);
+      mw[q] = r[0].y | (r[1].y << 8) | (r[2].y << 16) | (r[3].y << 24);
+      pk_out[q] = make_uint4(r[0].x, r[1].x, r[2].x, r[3].x);
+    }
+    reinterpret_cast<uint4*>(mask)[i] = make_uint4(mw[0], mw[1], mw[2], mw[3]);
   }
+  for (int64_t i = 16 * n16 + blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nbytes_mask; i += stride) {
+    const uint2 r = encode_byte(*reinterpret_cast<const uint2*>(dense + 8 * i), use_hint ? hint[i] : 0u, use_hint,
+                                bad);
+    *reinterpret_cast<uint32_t*>(packed + 4 * i) = r.x;
+    mask[i] = (uint8_t)r.y;
+  }
+  if (bad) flag(d_status, MOESQ_DFLAG_BAD_SPARSITY);
 }
 
 // ------------------------------------------------------------ weight export --
@@ -212,19 +262,32 @@ __global__ void k_quant_encode(const uint16_t* __restrict__ w, int64_t E, int64_
 }
 
 // ------------------------------------------------------------------- repack --
-// metadata: thread per (expert, tile, kb256, tile row): 16 mask bytes -> 16 metadata bytes
-__constant__ uint8_t c_meta_nib[16] = {0, 0, 0, 4, 0, 8, 9, 0, 0, 12, 13, 0, 14, 0, 0, 0};
-
+// metadata: thread per (expert, tile, kb256, tile row): 16 mask bytes -> 16 metadata
+// bytes.  The metadata nibble of a chunk is i0 | i1 << 2, its kept pair indices
+// (lowest and highest set bit of the mask nibble).
 __device__ __forceinline__ int64_t tile_src_row(int64_t tile, int64_t r, int64_t out, bool gate_up) {
   if (!gate_up) return 128 * tile + r;
   const int64_t I = out / 2;
   return r < 64 ? 64 * tile + r : I + 64 * tile + (r - 64);
 }
 
+__device__ __forceinline__ uint32_t meta_of_mask_word(uint32_t w, bool& bad) {
+  uint32_t o = 0;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint32_t nib = (w >> (4 * c)) & 0xF;
+    const bool ok = nib_legal(nib);
+    if (!ok) bad = true;
+    o |= (ok ? (nib_lo(nib) | (nib_hi(nib) << 2)) : 0u) << (4 * c);
+  }
+  return o;
+}
+
 __global__ void k_repack_meta(const uint8_t* __restrict__ mask, int64_t E, int64_t out, int64_t K,
                               bool gate_up, uint8_t* __restrict__ meta, int32_t* d_status) {
   const int64_t tiles = out / 128, nkb = (K + 255) / 256, mbytes_row = K / 16;
   const int64_t n = E * tiles * nkb * 128;
+  bool bad = false;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t r = i % 128;
@@ -233,50 +296,57 @@ __global__ void k_repack_meta(const uint8_t* __restrict__ mask, int64_t E, int64
     const int64_t e = i / (128 * nkb * tiles);
     const int64_t src = e * out + tile_src_row(t, r, out, gate_up);
     const uint8_t* m = mask + src * mbytes_row + kb * 16;
-    const int64_t avail = (mbytes_row - kb * 16) >= 16 ? 16 : (mbytes_row - kb * 16);
-    uint32_t o[4] = {0u, 0u, 0u, 0u};
-    bool bad = false;
-    for (int b = 0; b < 16; ++b) {
-      if (b >= avail) break;
-      const uint32_t mb = m[b];
-      const uint32_t lo = mb & 0xF, hi = mb >> 4;
-      if (c_pos0[lo] == 255 || c_pos0[hi] == 255) bad = true;
-      o[b >> 2] |= (uint32_t)(c_meta_nib[lo] | (c_meta_nib[hi] << 4)) << (8 * (b & 3));
-    }
-    if (bad) flag(d_status, MOESQ_DFLAG_BAD_SPARSITY);
+    // rows are K/16 bytes with K % 128 == 0: 8-byte aligned; the last 128 dense K
+    // of a row with K % 256 == 128 has 8 mask bytes and zero metadata after them
+    const bool full = mbytes_row - kb * 16 >= 16;
+    const uint2 m0 = *reinterpret_cast<const uint2*>(m);
+    const uint2 m1 = full ? *reinterpret_cast<const uint2*>(m + 8) : make_uint2(0u, 0u);
+    uint4 o;
+    o.x = meta_of_mask_word(m0.x, bad);
+    o.y = meta_of_mask_word(m0.y, bad);
+    o.z = full ? meta_of_mask_word(m1.x, bad) : 0u;
+    o.w = full ? meta_of_mask_word(m1.y, bad) : 0u;
     // block (e, t, kb) is 2048 bytes, row r at 16 r
-    *reinterpret_cast<uint4*>(meta + (((e * tiles + t) * nkb + kb) * 128 + r) * 16) =
-        make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint4*>(meta + (((e * tiles + t) * nkb + kb) * 128 + r) * 16) = o;
   }
+  if (bad) flag(d_status, MOESQ_DFLAG_BAD_SPARSITY);
 }
 
-// scale factors: thread per (expert, tile, kb128, tile row): 4 scale bytes, folded for up rows
+// scale factors: thread per (expert, tile, kb128, lane l of the block): the 4 scale
+// bytes of tile rows l, l+32, l+64, l+96 form the 16 bytes at 16 l of the
+// 512-byte block (row r, scale j at (r%32)*16 + (r/32)*4 + j), so a warp writes
+// one whole block; up rows of a split gate_up get the up/gate global ratio folded
 __global__ void k_repack_sf(const uint8_t* __restrict__ scale, const float* __restrict__ g_w,
                             int64_t E, int64_t out, int64_t K, int32_t kind,
                             uint8_t* __restrict__ sf, float* __restrict__ alpha_w) {
   const bool gate_up = kind != MOESQ_LINEAR_DOWN;
   const bool split = kind == MOESQ_LINEAR_GATE_UP_SPLIT;
   const int64_t tiles = out / 128, nkb = K / 128, sbytes_row = K / 32;
-  const int64_t n = E * tiles * nkb * 128;
+  const int64_t n = E * tiles * nkb * 32;
   const int64_t tid0 = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   if (tid0 < E) alpha_w[tid0] = split ? g_w[2 * tid0] : g_w[tid0];
   for (int64_t i = tid0; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t r = i % 128;
-    const int64_t kb = (i / 128) % nkb;
-    const int64_t t = (i / (128 * nkb)) % tiles;
-    const int64_t e = i / (128 * nkb * tiles);
-    const int64_t srow = tile_src_row(t, r, out, gate_up);
-    uint32_t s4 = *reinterpret_cast<const uint32_t*>(scale + (e * out + srow) * sbytes_row + 4 * kb);
-    if (split && srow >= out / 2) {
-      const float ratio = __fdiv_rn(g_w[2 * e + 1], g_w[2 * e]);
-      uint32_t f = 0;
+    const int64_t l = i % 32;
+    const int64_t kb = (i / 32) % nkb;
+    const int64_t t = (i / (32 * nkb)) % tiles;
+    const int64_t e = i / (32 * nkb * tiles);
+    uint32_t s4[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        f |= e4m3_code(__fmul_rn(e4m3_value((s4 >> (8 * j)) & 0xFF), ratio)) << (8 * j);
-      s4 = f;
+    for (int c = 0; c < 4; ++c) {
+      const int64_t srow = tile_src_row(t, l + 32 * c, out, gate_up);
+      uint32_t v = *reinterpret_cast<const uint32_t*>(scale + (e * out + srow) * sbytes_row + 4 * kb);
+      if (split && srow >= out / 2) {
+        const float ratio = __fdiv_rn(g_w[2 * e + 1], g_w[2 * e]);
+        uint32_t f = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          f |= e4m3_code(__fmul_rn(e4m3_value((v >> (8 * j)) & 0xFF), ratio)) << (8 * j);
+        v = f;
+      }
+      s4[c] = v;
     }
-    *reinterpret_cast<uint32_t*>(sf + ((e * tiles + t) * nkb + kb) * 512 +
-                                 sf_block_offset((uint32_t)r, 0)) = s4;
+    *reinterpret_cast<uint4*>(sf + ((e * tiles + t) * nkb + kb) * 512 + 16 * l) =
+        make_uint4(s4[0], s4[1], s4[2], s4[3]);
   }
 }
 
@@ -377,7 +447,7 @@ extern "C" moesq_status moesq_repack_meta(const uint8_t* mask, const uint8_t* sc
   k_repack_meta<<<grid_for(n1, 128), 128, 0, s>>>(mask, E, out, K, kind != MOESQ_LINEAR_DOWN, meta,
                                                   d_status);
   MOESQ_CHECK_LAUNCH();
-  const int64_t n2 = E * (out / 128) * (K / 128) * 128;
+  const int64_t n2 = E * (out / 128) * (K / 128) * 32;
   int g2 = grid_for(n2, 128);
   if ((int64_t)g2 * 128 < E) g2 = (int)((E + 127) / 128);
   k_repack_sf<<<g2, 128, 0, s>>>(scale, g_w, E, out, K, kind, sf, alpha_w);
