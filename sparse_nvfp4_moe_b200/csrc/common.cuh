@@ -54,6 +54,18 @@ __device__ __forceinline__ uint32_t e2m1x8(float a0, float a1, float a2, float a
   return out;
 }
 
+// Two float32 values -> one byte of E2M1 codes (lo in the low nibble), same
+// rounding rule as e2m1x8.
+__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b, %2, %1;\n\t"
+      "cvt.u32.u8 %0, b;\n\t}"
+      : "=r"(out)
+      : "f"(lo), "f"(hi));
+  return out;
+}
+
 // codes of v[0..7] under a group multiplier (inv == 0: the group is all zeros)
 __device__ __forceinline__ uint32_t nvfp4_word(const float* v, float inv) {
   if (inv == 0.0f) return 0u;

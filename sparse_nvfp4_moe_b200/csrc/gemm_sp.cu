@@ -393,9 +393,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         named_bar_sync(2 + pair, 64);
         const int cb = c_lo + (is_gate ? 0 : 16);   // first tile column finished here
         if (live && cb < t.n_rows) {
-          // h for feature `lane` x 16 token columns, then a conflict-free transpose
-          // (XOR swizzle) through the block just read: lane = (token column
-          // lane&15, feature half lane>>4), 16 features each
+          // h for feature `lane` x 16 token columns
           float hv[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
@@ -404,32 +402,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             const float gv = is_gate ? a : b, uv = is_gate ? b : a;
             hv[c] = __fmul_rn(silu_fast(gv), uv);
           }
-          __syncwarp();
+          // NVFP4 requant of each token column (lane = feature, the 32 lanes are
+          // the column's 32-feature group): group amax by a warp reduction; lane c
+          // (< 16) takes column c's scale; every lane scales its value by the
+          // column's multiplier; adjacent lanes pair into one code byte; the 16
+          // code bytes of each column are gathered through shared memory
+          uint32_t my_amax = 0u;
 #pragma unroll
-          for (int c = 0; c < 16; ++c) take[c * 32 + (lane ^ c)] = hv[c];
-          __syncwarp();
-          const int tok = lane & 15, fh = lane >> 4;
-          float amax = 0.0f;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int f = 16 * fh + i;
-            hv[i] = take[tok * 32 + (f ^ tok)];   // token column tok, feature f
-            amax = fmaxf(amax, fabsf(hv[i]));
+          for (int c = 0; c < 16; ++c) {
+            const uint32_t a = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(hv[c])));
+            if (lane == c) my_amax = a;
           }
-          amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 16));
-          if (tok < t.n_rows - cb) {
-            const GroupScale gs = nvfp4_group_scale(amax, S.gnext[t.e]);
+          GroupScale gs;
+          gs.sc = 0u;
+          gs.inv = 0.0f;
+          if (lane < 16) gs = nvfp4_group_scale(__uint_as_float(my_amax), S.gnext[t.e]);
+          uint32_t wd[4] = {0u, 0u, 0u, 0u};  // code bytes of features (lane, lane+1), columns 0..15
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float iv = __shfl_sync(0xffffffffu, gs.inv, c);
+            const float v = iv == 0.0f ? 0.0f : __fmul_rn(hv[c], iv);
+            const float nb = __shfl_xor_sync(0xffffffffu, v, 1);
+            wd[c >> 2] |= e2m1x2(v, nb) << (8 * (c & 3));
+          }
+          __syncwarp();
+          uint8_t* tb = reinterpret_cast<uint8_t*>(take);  // [16 columns][16 code bytes]
+          if ((lane & 1) == 0) {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) tb[c * 16 + (lane >> 1)] = (uint8_t)(wd[c >> 2] >> (8 * (c & 3)));
+          }
+          __syncwarp();
+          if (lane < 16 && lane < t.n_rows - cb) {
             const int fb = 64 * mt + 32 * (q & 1);  // first feature of the group
-            const int64_t prow = (int64_t)S.epad[t.e] + t.nt * BN + cb + tok;
+            const int64_t prow = (int64_t)S.epad[t.e] + t.nt * BN + cb + lane;
             if (prow >= 0 && prow < p.P_cap) {
               uint8_t* codes = (uint8_t*)p.out;
-              *reinterpret_cast<uint2*>(codes + prow * (I / 2) + fb / 2 + 8 * fh) =
-                  make_uint2(nvfp4_word(hv, gs.inv), nvfp4_word(hv + 8, gs.inv));
-              if (fh == 0) {
-                const int64_t blk = (prow / 128) * (I / 128) + fb / 128;
-                p.out_sf[blk * 512 + sf_block_offset((uint32_t)(prow % 128), (uint32_t)((fb / 32) % 4))] =
-                    (uint8_t)gs.sc;
-              }
+              *reinterpret_cast<uint4*>(codes + prow * (I / 2) + fb / 2) = *reinterpret_cast<const uint4*>(tb + lane * 16);
+              const int64_t blk = (prow / 128) * (I / 128) + fb / 128;
+              p.out_sf[blk * 512 + sf_block_offset((uint32_t)(prow % 128), (uint32_t)((fb / 32) % 4))] =
+                  (uint8_t)gs.sc;
             }
           }
         }
