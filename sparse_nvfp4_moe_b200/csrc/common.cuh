@@ -410,6 +410,14 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const void* tmap, in
       "l"(tmap), "r"(x), "r"(y), "r"(bar_cluster)
       : "memory");
 }
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const void* tmap, int32_t x, int32_t y,
+                                                 int32_t z, uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+      "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(bar_cluster)
+      : "memory");
+}
 __device__ __forceinline__ void tma_load_4d_pair(void* dst, const void* tmap, int32_t x, int32_t y,
                                                  int32_t z, int32_t w, uint32_t bar_cluster) {
   asm volatile(
@@ -458,6 +466,10 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
 // memory at the descriptor's offset goes to its own TMEM
 __device__ __forceinline__ void tc_cp_pair_128x128b(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+// 128 lanes x 32 bytes: two 16-byte core-matrix columns `LBO` bytes apart
+__device__ __forceinline__ void tc_cp_pair_128x256b(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 __device__ __forceinline__ void tc_cp_pair_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)

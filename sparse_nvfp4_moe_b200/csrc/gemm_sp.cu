@@ -139,7 +139,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     k_grouped_gemm_sp(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                       const __grid_constant__ CUtensorMap tmap_b16, const __grid_constant__ CUtensorMap tmap_e,
                       const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
-                      const __grid_constant__ CUtensorMap tmap_y, const Params p) {
+                      const __grid_constant__ CUtensorMap tmap_y, const __grid_constant__ CUtensorMap tmap_b_3d,
+                      const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   float* epi = (float*)(smem + STAGES * STAGE_BYTES);
@@ -173,6 +174,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     tma_prefetch_desc(&tmap_e);
     tma_prefetch_desc(&tmap_sfa);
     tma_prefetch_desc(&tmap_sfb);
+    tma_prefetch_desc(&tmap_b_3d);
   }
   if (warp == 1) {
     tmem_alloc_pair(&S.tmem_base, TMEM_COLS);
@@ -226,6 +228,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       uint32_t phase = 0;
       long fills = 0;
       int e_cur = 0;
+      uint32_t full_lead[STAGES];
+#pragma unroll
+      for (int i = 0; i < STAGES; ++i) full_lead[i] = cluster_map(&S.full[i], 0);
+      const bool b3d = (p.K % 256) == 0;  // both 256-deep token chunks of a stage in one 3-D box
       for (int id = pair_id; id < total; id += npairs) {
         const Tile t = decode_tile(S, id, MT2, E, e_cur);
         const int mt = min(2 * t.mt + (int)rank, MT - 1);  // an odd last tile is loaded twice
@@ -240,20 +246,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // a tile of <= 32 tokens loads 16-row B boxes (decode-sized groups)
         const bool small = n_mma <= 32;
         const void* tb = small ? (const void*)&tmap_b16 : (const void*)&tmap_b;
+        const void* tb3 = &tmap_b_3d;
         const uint32_t b_box = small ? 16 * 128 : B_CHUNK;
         for (int kb = 0; kb < nkb; ++kb) {
           mbar_wait_spin(&S.empty[stage], phase ^ 1, abort, p.d_status);
           const int nk = min(4, kb128 - 4 * kb);  // 128-deep MMAs in this stage
           const int nc = (nk + 1) >> 1;           // 256-deep chunks in this stage
           uint8_t* st = smem + stage * STAGE_BYTES;
-          const uint32_t bar = cluster_map(&S.full[stage], 0);
+          uint32_t bar = full_lead[0];
+#pragma unroll
+          for (int i = 1; i < STAGES; ++i)
+            if (stage == i) bar = full_lead[i];
           if (lead) mbar_arrive_expect_tx(&S.full[stage], 2u * (A_BYTES + nc * b_box + E_BYTES + 2 * SF_BYTES));
           // weight tile: gate rows 64mt.. and up rows I+64mt.. in one 4-D box,
           // or 128 consecutive down rows
           if (p.gate_up) tma_load_4d_pair(st, &tmap_a, kb * 128, 64 * mt, 0, t.e, bar);
           else tma_load_2d_pair(st, &tmap_a, kb * 128, t.e * p.M + BM * mt, bar);
-          tma_load_2d_pair(st + A_BYTES, tb, kb * 256, brow, bar);
-          if (nc > 1) tma_load_2d_pair(st + A_BYTES + B_CHUNK, tb, kb * 256 + 128, brow, bar);
+          if (b3d && nc > 1 && !small) {  // 64-row chunks: chunk 1 lands at B_CHUNK as the MMA expects
+            tma_load_3d_pair(st + A_BYTES, tb3, 0, brow, 2 * kb, bar);
+          } else {
+            tma_load_2d_pair(st + A_BYTES, tb, kb * 256, brow, bar);
+            if (nc > 1) tma_load_2d_pair(st + A_BYTES + B_CHUNK, tb, kb * 256 + 128, brow, bar);
+          }
           // metadata (2 KB per 256 dense K) and scale blocks (512 B per 128 dense K)
           // as 256-byte rows; a stage always moves 4 KB + 2 KB + 2 KB
           tma_load_2d_pair(st + A_BYTES + B_BYTES, &tmap_e, 0, (wt * nkb256 + 2 * kb) * 8, bar);
@@ -293,6 +307,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       const uint64_t dA0 = smem_desc(s0, 16, 1024, SWZ_128B);
       const uint64_t dB0 = smem_desc(s0 + A_BYTES, 16, 1024, SWZ_128B);
       const uint64_t dE0 = smem_desc(s0 + A_BYTES + B_BYTES, 16, 128, SWZ_NONE);
+      const uint64_t dE2 = smem_desc(s0 + A_BYTES + B_BYTES, BM * 16, 128, SWZ_NONE);  // LBO = chunk stride
       const uint64_t dSFA0 = smem_desc(s0 + A_BYTES + B_BYTES + E_BYTES, 16, 128, SWZ_NONE);
       const uint64_t dSFB0 = dSFA0 + (SF_BYTES >> 4);
       const uint32_t tE = tmem + TM_E, tSFA = tmem + TM_SFA, tSFB = tmem + TM_SFB;
@@ -309,6 +324,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           tc_fence_after();
           const uint64_t so = (uint64_t)((stage * STAGE_BYTES) >> 4);
           const int nk = min(4, kb128 - 4 * kb);
+          if (nk == 4) {
+            // metadata of both 256-deep chunks (2 KB apart) in one copy; MMA j
+            // reads columns tE + 2j
+            tc_cp_pair_128x256b(tE, dE2 + so);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              tc_cp_pair_32x128b_warpx4(tSFA + 4 * j, dSFA0 + so + (uint64_t)(j * (512 >> 4)));
+              tc_cp_pair_32x128b_warpx4(tSFB + 4 * j, dSFB0 + so + (uint64_t)(j * (512 >> 4)));
+              tc_mma_pair_sp_nvf4(d_tmem, dA0 + so + (uint64_t)(j * 2),
+                                  dB0 + so + (uint64_t)((j >> 1) * (B_CHUNK >> 4) + (j & 1) * 4), tE + 2 * j,
+                                  idesc, tSFA + 4 * j, tSFB + 4 * j, (kb > 0 || j > 0) ? 1u : 0u);
+            }
+          } else {
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             if (j < nk) {
@@ -323,6 +351,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                                   dB0 + so + (uint64_t)((j >> 1) * (B_CHUNK >> 4) + (j & 1) * 4), tE + 2 * j,
                                   idesc, tSFA + 4 * j, tSFB + 4 * j, (kb > 0 || j > 0) ? 1u : 0u);
             }
+          }
           }
           tc_commit_pair_mc(&S.empty[stage], 0x3);
           if (++stage == STAGES) {
@@ -690,6 +719,15 @@ extern "C" moesq_status moesq_grouped_gemm(const moesq_linear* W, const uint8_t*
       !make_tmap_rows(&tb16, act_codes, (uint64_t)(W->K / 2), (uint64_t)P_cap, 128, 16,
                       CU_TENSOR_MAP_SWIZZLE_128B))
     return MOESQ_ERR_CUDA;
+  // the same token codes as (128-byte chunk row, row, 256-deep chunk): both 64-row chunks
+  // of a 512-deep stage in one box; valid when K % 256 == 0 (else the 2-D boxes are used)
+  CUtensorMap tb3 = tb;
+  if (W->K % 256 == 0) {
+    const cuuint64_t dims[3] = {128, (uint64_t)P_cap, (uint64_t)(W->K / 256)};
+    const cuuint64_t strides[2] = {(uint64_t)(W->K / 2), 128};
+    const cuuint32_t box64[3] = {128, 64, 2};
+    if (!make_tmap_u8(&tb3, act_codes, 3, dims, strides, box64, CU_TENSOR_MAP_SWIZZLE_128B)) return MOESQ_ERR_CUDA;
+  }
   // metadata and scale blocks seen as 256-byte rows (no swizzle: contiguous copies)
   if (!make_tmap_rows(&te, W->meta, 256, (uint64_t)(W->E * MT * nkb256 * 8), 256, 16,
                       CU_TENSOR_MAP_SWIZZLE_NONE) ||
@@ -758,15 +796,15 @@ extern "C" moesq_status moesq_grouped_gemm(const moesq_linear* W, const uint8_t*
   switch (epilogue) {
     case MOESQ_EPI_F32:
       err = moesq_launch(sp::k_grouped_gemm_sp<MOESQ_EPI_F32>, grid, dim3(sp::THREADS), sp::SMEM_BYTES, st, ta, tb,
-                         tb16, te, tsfa, tsfb, ty, prm);
+                         tb16, te, tsfa, tsfb, ty, tb3, prm);
       break;
     case MOESQ_EPI_BF16:
       err = moesq_launch(sp::k_grouped_gemm_sp<MOESQ_EPI_BF16>, grid, dim3(sp::THREADS), sp::SMEM_BYTES, st, ta, tb,
-                         tb16, te, tsfa, tsfb, ty, prm);
+                         tb16, te, tsfa, tsfb, ty, tb3, prm);
       break;
     default:
       err = moesq_launch(sp::k_grouped_gemm_sp<MOESQ_EPI_SWIGLU_NVFP4>, grid, dim3(sp::THREADS), sp::SMEM_BYTES, st,
-                         ta, tb, tb16, te, tsfa, tsfb, ty, prm);
+                         ta, tb, tb16, te, tsfa, tsfb, ty, tb3, prm);
   }
   if (err != cudaSuccess) {
     (void)cudaGetLastError();

@@ -95,6 +95,8 @@ CASES = {
     "ragged_multi_tile": (W.LayerConfig("ragged", 41, 4, 2, 384, 128, (400,), "uniform", True), 400),
     "sparse_routing": (W.LayerConfig("sparse", 43, 16, 1, 256, 256, (9,), "zipf", True), 9),
     "mid_ktail": (W.LayerConfig("mid", 42, 16, 4, 384, 256, (300,), "uniform", True), 300),
+    # full 512-deep stages (one metadata copy per stage, 3-D token boxes), plus tiles of <= 32 tokens
+    "deep_k": (W.LayerConfig("deep", 44, 12, 2, 1024, 512, (150,), "zipf", True), 150),
 }
 
 
