@@ -78,6 +78,10 @@ struct Params {
 };
 
 struct Smem {
+  // SwiGLU epilogue staging, double-buffered over tiles: per 32-token column block
+  // the requantised codes (32 B = 64 features per token) and the scale pairs
+  alignas(128) uint8_t hstg[2][4][32][32];
+  alignas(16) uint8_t sstg[2][4][32][2];
   // full[s]: stage s landed.  empty[s]: stage s consumed by the tensor core.
   uint64_t full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], done;
   uint32_t tmem_base;
@@ -392,6 +396,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const int pair = (q & 1) + 2 * kb;           // 0..7
     float* xch = epi + pair * 2 * 16 * 32;       // [2][16 cols][32 lanes]
     int e_cur = 0;
+    int sb = 0;  // SwiGLU staging buffer of this tile
     for (int id = pair_id; id < total; id += npairs) {
       const Tile t = decode_tile(S, id, MT2, E, e_cur);
       const int mt = 2 * t.mt + (int)rank;  // this CTA's weight tile
@@ -431,49 +436,55 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             const float gv = is_gate ? a : b, uv = is_gate ? b : a;
             hv[c] = __fmul_rn(silu_fast(gv), uv);
           }
-          // NVFP4 requant of each token column (lane = feature, the 32 lanes are
-          // the column's 32-feature group): group amax by a warp reduction; lane c
-          // (< 16) takes column c's scale; every lane scales its value by the
-          // column's multiplier; adjacent lanes pair into one code byte; the 16
-          // code bytes of each column are gathered through shared memory
-          uint32_t my_amax = 0u;
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const uint32_t a = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(hv[c])));
-            if (lane == c) my_amax = a;
-          }
-          GroupScale gs;
-          gs.sc = 0u;
-          gs.inv = 0.0f;
-          if (lane < 16) gs = nvfp4_group_scale(__uint_as_float(my_amax), S.gnext[t.e]);
-          uint32_t wd[4] = {0u, 0u, 0u, 0u};  // code bytes of features (lane, lane+1), columns 0..15
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const float iv = __shfl_sync(0xffffffffu, gs.inv, c);
-            const float v = iv == 0.0f ? 0.0f : __fmul_rn(hv[c], iv);
-            const float nb = __shfl_xor_sync(0xffffffffu, v, 1);
-            wd[c >> 2] |= e2m1x2(v, nb) << (8 * (c & 3));
-          }
+          // NVFP4 requant of each token column.  Transpose through the block just
+          // read: column c is one 128-byte row (feature f in 16-byte chunk
+          // (f/4) ^ (c&7), so both the row writes and the chunk reads below spread
+          // over the banks); lane = (column lane&15, feature half lane>>4) then
+          // reads its 16 features with four 16-byte loads.  Each lane of a column
+          // pair computes the scale from the joint amax; codes of adjacent
+          // features pack in-thread.
           __syncwarp();
-          uint8_t* tb = reinterpret_cast<uint8_t*>(take);  // [16 columns][16 code bytes]
-          if ((lane & 1) == 0) {
 #pragma unroll
-            for (int c = 0; c < 16; ++c) tb[c * 16 + (lane >> 1)] = (uint8_t)(wd[c >> 2] >> (8 * (c & 3)));
-          }
+          for (int c = 0; c < 16; ++c) take[c * 32 + ((((lane >> 2) ^ c) & 7) << 2) + (lane & 3)] = hv[c];
           __syncwarp();
-          if (lane < 16 && lane < t.n_rows - cb) {
-            const int fb = 64 * mt + 32 * (q & 1);  // first feature of the group
-            const int64_t prow = (int64_t)S.epad[t.e] + t.nt * BN + cb + lane;
-            if (prow >= 0 && prow < p.P_cap) {
-              uint8_t* codes = (uint8_t*)p.out;
-              *reinterpret_cast<uint4*>(codes + prow * (I / 2) + fb / 2) = *reinterpret_cast<const uint4*>(tb + lane * 16);
-              const int64_t blk = (prow / 128) * (I / 128) + fb / 128;
-              p.out_sf[blk * 512 + sf_block_offset((uint32_t)(prow % 128), (uint32_t)((fb / 32) % 4))] =
-                  (uint8_t)gs.sc;
-            }
+          const int tok = lane & 15, fh = lane >> 4;
+          float amax = 0.0f;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int chunk = (4 * fh + k) ^ (tok & 7);
+            const float4 v = *reinterpret_cast<const float4*>(take + tok * 32 + 4 * chunk);
+            hv[4 * k] = v.x, hv[4 * k + 1] = v.y, hv[4 * k + 2] = v.z, hv[4 * k + 3] = v.w;
+            amax = fmaxf(fmaxf(amax, fmaxf(fabsf(v.x), fabsf(v.y))), fmaxf(fabsf(v.z), fabsf(v.w)));
           }
+          amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 16));
+          // stage this group's codes (16 features per lane) and scale for the block's write
+          const GroupScale gs = nvfp4_group_scale(amax, S.gnext[t.e]);
+          const int r = cb - c_lo + tok;  // token row within the column block
+          *reinterpret_cast<uint2*>(&S.hstg[sb][kb][r][16 * (q & 1) + 8 * fh]) =
+              make_uint2(nvfp4_word(hv, gs.inv), nvfp4_word(hv + 8, gs.inv));
+          if (fh == 0) S.sstg[sb][kb][r][q & 1] = (uint8_t)gs.sc;
         }
         named_bar_sync(2 + pair, 64);  // the exchange block is free for the next tile
+        // the four warps of this column block hold all 64 features of its 32 tokens:
+        // one TMA store of [32 rows][32 B] codes (rows past the expert's tokens are its
+        // own padding, never read as tokens) and 2-byte scale pairs
+        fence_proxy_async_smem();
+        if (q == 0 && lane == 0) bulk_wait_group_read0();  // the store two tiles back has read its buffer
+        named_bar_sync(10 + kb, 128);
+        if (live) {
+          const int64_t prow0 = (int64_t)S.epad[t.e] + t.nt * BN + c_lo;
+          if (q == 0 && lane == 0) {
+            tma_store_2d(&tmap_y, &S.hstg[sb][kb][0][0], 32 * mt, (int32_t)prow0);
+            bulk_commit_group();
+          }
+          if (q == 1 && lane < t.n_rows - c_lo) {
+            const int64_t prow = prow0 + lane;
+            const int64_t blk = (prow / 128) * (I / 128) + (64 * mt) / 128;
+            *reinterpret_cast<uint16_t*>(p.out_sf + blk * 512 + sf_block_offset((uint32_t)(prow % 128), 2u * (mt & 1))) =
+                *reinterpret_cast<const uint16_t*>(&S.sstg[sb][kb][lane][0]);
+          }
+        }
+        sb ^= 1;
       } else if constexpr (EPI == MOESQ_EPI_BF16) {
         // Stage the bf16 tile as two 64-feature halves [128 token rows][128 B] in
         // the TMA 128-byte swizzle (16-byte chunk j of row r at chunk j ^ (r & 7)),
@@ -587,6 +598,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 
   if constexpr (EPI == MOESQ_EPI_BF16) {
     if (threadIdx.x == 64) bulk_wait_group0();  // the last tile's stores are complete
+  }
+  if constexpr (EPI == MOESQ_EPI_SWIGLU_NVFP4) {
+    if (warp >= 2 && (warp & 3) == 0 && lane == 0) bulk_wait_group0();
   }
   // no CTA of the pair frees TMEM or exits while its peer may still use it
   tc_fence_before();
@@ -738,6 +752,13 @@ extern "C" moesq_status moesq_grouped_gemm(const moesq_linear* W, const uint8_t*
 
   // bf16 output [S rows x out columns]: 64-column x 128-row boxes, 128-byte swizzle
   CUtensorMap ty = ta;
+  if (epilogue == MOESQ_EPI_SWIGLU_NVFP4) {
+    // requantised codes [P_cap rows x I/2 bytes], 32-byte x 32-row boxes, no swizzle
+    const cuuint64_t dims[2] = {(uint64_t)(W->out / 4), (uint64_t)P_cap};
+    const cuuint64_t strides[1] = {(uint64_t)(W->out / 4)};
+    const cuuint32_t box[2] = {32, 32};
+    if (!make_tmap_u8(&ty, out, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE)) return MOESQ_ERR_CUDA;
+  }
   if (epilogue == MOESQ_EPI_BF16) {
     PFN_encodeTiled enc = get_encode_fn();
     const cuuint64_t dims[2] = {(uint64_t)W->out, (uint64_t)S};
