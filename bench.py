@@ -388,6 +388,23 @@ def traffic_record():
     return d if d.get("gemm_sp_sha256") == sha else None
 
 
+def max_over_ranks(ms, world, device):
+    """The slowest rank's time.  Every rank passes its own CUDA-event total; the
+    replicas' whole-job time is the maximum (one all-reduce, outside the timed region)."""
+    if world == 1:
+        return float(ms)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(world, steps, flops_step, max_ms):
+    """Dense-equivalent TFLOP/s of the whole job: every replica does flops_step per step."""
+    return world * steps * flops_step / (max_ms * 1e-3) / 1e12
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -412,16 +429,12 @@ def run_ours(args, rank, world, local_rank):
         if world > 1:
             dist.barrier()
     clocks = clk.summary()
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
     S, H, I = b.S, cfg.H, cfg.I
     fl = step_flops(S, H, I)
     by = step_bytes(S, args.tokens, H, I, b.n_touched)
     flops_step = fl["gate_up"] + fl["down"]
-    value = world * args.steps * flops_step / (total_ms * 1e-3) / 1e12
+    value = whole_job_value(world, args.steps, flops_step, total_ms)
     # roofline of the dominant kernel
     avg = {s: sum(v) / len(v) for s, v in per.items()}
     dom = max(("gemm_gate_up", "gemm_down"), key=lambda s: avg[s])
@@ -473,11 +486,7 @@ def run_ours(args, rank, world, local_rank):
     }
     if not args.no_e2e:
         ms, h2d, d2h = b.e2e(max(3, args.steps // 4), 2)
-        e2e_val = world * flops_step / (ms * 1e-3) / 1e12
-        if world > 1:
-            t = torch.tensor([ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_val = world * flops_step / (float(t.item()) * 1e-3) / 1e12
+        e2e_val = whole_job_value(world, 1, flops_step, max_over_ranks(ms, world, dev))
         out["e2e"] = {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                       "ms_per_step": ms, "api": "moesq_moe_forward_host (pinned host buffers)"}
     if not args.no_sweep and world == 1:

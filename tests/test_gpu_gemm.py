@@ -35,7 +35,7 @@ def bf16_ulp(v):
 class Layer:
     """A small synthetic layer: oracle storage on the host, device copies repacked by the GPU."""
 
-    def __init__(self, cfg, T, g_down_scale=1.0):
+    def __init__(self, cfg, T, g_down_scale=1.0, routing=None):
         self.cfg, self.T = cfg, T
         n_seg = 2 if cfg.split_gate_up_global else 1
         wgu = W.all_expert_weights_bf16(cfg, "gate_up")
@@ -46,8 +46,12 @@ class Layer:
         self.dgu = M.ExpertLinear.from_storage(PU.storage_to_device(self.gu), kind_gu)
         self.ddn = M.ExpertLinear.from_storage(PU.storage_to_device(self.dn), M.KIND_DOWN)
         self.x = W.layer_input_bf16(cfg, T)
-        ids, w = W.routing(cfg, T)
-        self.ids, self.w = ids.numpy(), w.numpy()
+        if routing is None:
+            ids, w = W.routing(cfg, T)
+            self.ids, self.w = ids.numpy(), w.numpy()
+        else:                                   # a given [T, k] routing (ids int, weights f32)
+            self.ids = np.asarray(routing[0], np.int64).reshape(T, cfg.k)
+            self.w = np.asarray(routing[1], np.float32).reshape(T, cfg.k)
         self.perm = R.permute(self.ids, cfg.E)
         self.S = T * cfg.k
         self.P = M.padded_rows(self.S, cfg.E)
