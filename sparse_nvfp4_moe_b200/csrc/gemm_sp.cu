@@ -87,13 +87,12 @@ struct Smem {
   uint32_t tmem_base;
   int abort;
   // per-expert tables, read from global memory once at set-up so that no role
-  // waits on a global load between tiles: first token tile of each expert,
-  // routed-slot offsets, padded-row offsets
-  int tile_start[MAX_E + 1];
-  int eoff[MAX_E + 1];
-  int epad[MAX_E];
-  float alpha[MAX_E];  // g_act[e] * alpha_w[e]: the accumulator's scale
-  float gnext[MAX_E];  // global scale of the requantised output (SwiGLU epilogue)
+  // waits on a global load between tiles.  One 16-byte record per expert, so
+  // that a role finds everything about its next tile in one shared load:
+  // {end of its token tiles (prefix sum), first routed slot, first padded row,
+  // routed-slot count}
+  int4 rec[MAX_E];
+  float2 ag[MAX_E];  // {g_act[e] * alpha_w[e] (the accumulator's scale), global scale of the requantised output}
 };
 
 constexpr size_t SMEM_BYTES = 1024 /*align*/ + (size_t)STAGES * STAGE_BYTES + EPI_BYTES + sizeof(Smem);
@@ -110,23 +109,41 @@ __device__ __forceinline__ uint32_t make_idesc(uint32_t n) {
 
 struct Tile {
   int e, nt, mt, n_rows;
+  int prow;  // first padded row of the token tile
+  int s0;    // first routed slot of the token tile
 };
 
-// Work item `id` -> (expert, token tile, weight tile).  Every role walks its
-// items in increasing order, so the expert is found by stepping `e` forward
-// from the previous item's (tile_start is non-decreasing; empty experts are
-// stepped over).
-__device__ __forceinline__ Tile decode_tile(const Smem& s, int id, int MT, int E, int& e) {
+// Work items run over (token tile q, weight-tile pair m), m fastest; pair `pid`
+// of `npairs` takes items pid, pid + npairs, ...  Every role walks its items in
+// that order, stepping (q, m) by a precomputed (dq, dm) and the expert forward
+// from the previous item's, so no role divides or searches between tiles.
+struct TileWalk {
+  int q, m, dq, dm, e;
+  __device__ __forceinline__ TileWalk(int pid, int npairs, int MT2)
+      : q(pid / MT2), m(pid % MT2), dq(npairs / MT2), dm(npairs % MT2), e(0) {}
+  __device__ __forceinline__ void advance(int MT2) {
+    m += dm;
+    q += dq;
+    if (m >= MT2) {
+      m -= MT2;
+      ++q;
+    }
+  }
+};
+
+// The current item of `w` (empty experts are stepped over: their tiles end
+// where they start).
+__device__ __forceinline__ Tile decode_tile(const Smem& s, TileWalk& w, int E) {
+  int4 r = s.rec[w.e];
+  while (r.x <= w.q && w.e + 1 < E) r = s.rec[++w.e];
   Tile t;
-  const int q = id / MT;
-  t.mt = id % MT;
-  while (e + 1 < E && s.tile_start[e + 1] <= q) ++e;
-  const int lo = e;
-  t.e = lo;
-  t.nt = q - s.tile_start[lo];
-  const int te = s.eoff[lo + 1] - s.eoff[lo];
-  const int r = te - t.nt * BN;
-  t.n_rows = r < BN ? r : BN;
+  t.e = w.e;
+  t.mt = w.m;
+  t.nt = w.q - (r.x - (r.w + BN - 1) / BN);
+  const int rem = r.w - t.nt * BN;
+  t.n_rows = rem < BN ? rem : BN;
+  t.prow = r.z + t.nt * BN;
+  t.s0 = r.y + t.nt * BN;
   return t;
 }
 
@@ -189,37 +206,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   pdl_wait();
   pdl_trigger();
   // per-expert tables: one round of parallel global loads
-  for (int e = threadIdx.x; e <= E; e += blockDim.x) {
-    S.eoff[e] = off[e];
-    if (e < E) {
-      S.epad[e] = p.pad_offsets[e];
-      S.alpha[e] = __fmul_rn(p.g_act[e], p.alpha_w[e]);
-      S.gnext[e] = p.g_next ? p.g_next[e] : 0.0f;
-    }
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int o0 = off[e], o1 = off[e + 1];
+    S.rec[e] = make_int4(0, o0, p.pad_offsets[e], o1 - o0);
+    S.ag[e] = make_float2(__fmul_rn(p.g_act[e], p.alpha_w[e]), p.g_next ? p.g_next[e] : 0.0f);
   }
   __syncthreads();
-  if (warp == 0) {  // tile_start[e] = sum over e' < e of ceil(T_e' / BN)
+  if (warp == 0) {  // end of expert e's token tiles = sum over e' <= e of ceil(T_e' / BN)
     int run = 0;
     for (int e0 = 0; e0 < E; e0 += 32) {
       const int e = e0 + lane;
       int v = 0;
-      if (e < E) v = (S.eoff[e + 1] - S.eoff[e] + BN - 1) / BN;
+      if (e < E) v = (S.rec[e].w + BN - 1) / BN;
       int x = v;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, x, o);
         if (lane >= o) x += y;
       }
-      if (e < E) S.tile_start[e] = run + x - v;
+      if (e < E) S.rec[e].x = run + x;
       run += __shfl_sync(0xffffffffu, x, 31);
     }
-    if (lane == 0) S.tile_start[E] = run;
   }
   tc_fence_before();
   cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem = S.tmem_base;
-  const int total = S.tile_start[E] * MT2;
+  const int total = S.rec[E - 1].x * MT2;
   volatile int* abort = &S.abort;
 
   if (warp == 0) {
@@ -231,15 +244,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       long fills = 0;
-      int e_cur = 0;
+      TileWalk walk(pair_id, npairs, MT2);
       uint32_t full_lead[STAGES];
 #pragma unroll
       for (int i = 0; i < STAGES; ++i) full_lead[i] = cluster_map(&S.full[i], 0);
       const bool b3d = (p.K % 256) == 0;  // both 256-deep token chunks of a stage in one 3-D box
-      for (int id = pair_id; id < total; id += npairs) {
-        const Tile t = decode_tile(S, id, MT2, E, e_cur);
+      for (int id = pair_id; id < total; id += npairs, walk.advance(MT2)) {
+        const Tile t = decode_tile(S, walk, E);
         const int mt = min(2 * t.mt + (int)rank, MT - 1);  // an odd last tile is loaded twice
-        int prow = S.epad[t.e] + t.nt * BN;
+        int prow = t.prow;
         if (prow < 0 || (int64_t)prow + BN > p.P_cap) {  // inconsistent offsets: stay in bounds
           flag(p.d_status, MOESQ_DFLAG_CAPACITY);
           prow = 0;
@@ -315,9 +328,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       const uint64_t dSFA0 = smem_desc(s0 + A_BYTES + B_BYTES + E_BYTES, 16, 128, SWZ_NONE);
       const uint64_t dSFB0 = dSFA0 + (SF_BYTES >> 4);
       const uint32_t tE = tmem + TM_E, tSFA = tmem + TM_SFA, tSFB = tmem + TM_SFB;
-      int e_cur = 0;
-      for (int id = pair_id; id < total; id += npairs) {
-        const Tile t = decode_tile(S, id, MT2, E, e_cur);
+      TileWalk walk(pair_id, npairs, MT2);
+      for (int id = pair_id; id < total; id += npairs, walk.advance(MT2)) {
+        const Tile t = decode_tile(S, walk, E);
         const int n_mma = max(16, (t.n_rows + 15) / 16 * 16);
         const uint32_t idesc = make_idesc((uint32_t)n_mma);
         const uint32_t d_tmem = tmem + TM_ACC + buf * BN;
@@ -395,13 +408,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     // column block; each side hands the other a 16x32 block (column-major, lane-fast).
     const int pair = (q & 1) + 2 * kb;           // 0..7
     float* xch = epi + pair * 2 * 16 * 32;       // [2][16 cols][32 lanes]
-    int e_cur = 0;
+    TileWalk walk(pair_id, npairs, MT2);
     int sb = 0;  // SwiGLU staging buffer of this tile
-    for (int id = pair_id; id < total; id += npairs) {
-      const Tile t = decode_tile(S, id, MT2, E, e_cur);
+    for (int id = pair_id; id < total; id += npairs, walk.advance(MT2)) {
+      const Tile t = decode_tile(S, walk, E);
       const int mt = 2 * t.mt + (int)rank;  // this CTA's weight tile
       const bool own_tile = mt < MT;          // false: the duplicate of an odd last tile
-      const float alpha = S.alpha[t.e];
+      const float2 ag = S.ag[t.e];
+      const float alpha = ag.x;
       mbar_wait_poll(&S.acc_full[buf], acc_phase[buf], abort, p.d_status);
       tc_fence_after();
       const uint32_t tbase = tmem + TM_ACC + buf * BN + ((uint32_t)(32 * q) << 16);
@@ -458,7 +472,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           }
           amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 16));
           // stage this group's codes (16 features per lane) and scale for the block's write
-          const GroupScale gs = nvfp4_group_scale(amax, S.gnext[t.e]);
+          const GroupScale gs = nvfp4_group_scale(amax, ag.y);
           const int r = cb - c_lo + tok;  // token row within the column block
           *reinterpret_cast<uint2*>(&S.hstg[sb][kb][r][16 * (q & 1) + 8 * fh]) =
               make_uint2(nvfp4_word(hv, gs.inv), nvfp4_word(hv + 8, gs.inv));
@@ -472,7 +486,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         if (q == 0 && lane == 0) bulk_wait_group_read0();  // the store two tiles back has read its buffer
         named_bar_sync(10 + kb, 128);
         if (live) {
-          const int64_t prow0 = (int64_t)S.epad[t.e] + t.nt * BN + c_lo;
+          const int64_t prow0 = (int64_t)t.prow + c_lo;
           if (q == 0 && lane == 0) {
             tma_store_2d(&tmap_y, &S.hstg[sb][kb][0][0], 32 * mt, (int32_t)prow0);
             bulk_commit_group();
@@ -494,7 +508,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // features as one word; even lanes take column c, odd lanes column c + 4,
         // whose rows fall on the other half of the banks.
         uint8_t* stg = reinterpret_cast<uint8_t*>(epi);  // 2 x 128 x 128 B
-        const int64_t s0 = (int64_t)S.eoff[t.e] + t.nt * BN;
+        const int64_t s0 = t.s0;
         int nvalid = t.n_rows;
         if (s0 + nvalid > p.S) nvalid = (int)(p.S - s0 > 0 ? p.S - s0 : 0);
         uint32_t acc[32];
@@ -557,7 +571,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         float* tr = epi + ew * 512;
         const int col0 = p.gate_up ? (q < 2 ? 64 * mt + 32 * q : I + 64 * mt + 32 * (q - 2))
                                    : BM * mt + 32 * q;
-        const int64_t s0 = (int64_t)S.eoff[t.e] + t.nt * BN;
+        const int64_t s0 = t.s0;
         int nvalid = t.n_rows;                     // valid columns of the tile
         if (s0 + nvalid > p.S) nvalid = (int)(p.S - s0 > 0 ? p.S - s0 : 0);
         uint32_t acc[32];
