@@ -198,9 +198,12 @@ def fold_up_scales(scale_up, g_gate, g_up) -> np.ndarray:
 # The library lays out whole operands as
 #   meta[e][tile][kb256][128][16]   sfw[e][tile][kb128][512]   sfa[pb][kb128][512]
 # where "tile" is a 128-row block of the weight in tile row order: for down the
-# identity, for fused gate_up tile t rows 0..63 = gate rows 64t..64t+63 and rows
-# 64..127 = up rows I+64t..I+64t+63 (so one accumulator tile holds the gate and
-# up features of the same 64 outputs).
+# identity; for fused gate_up, tile t holds the gate and the up rows of the same
+# 64 outputs 64t..64t+63, interleaved so that the SwiGLU epilogue finds a gate
+# value and its up value, for two adjacent outputs, in one thread: tile row
+# r = 32q + 16h + 8s + j (q < 4, h, s < 2, j < 8) is output f = 64t + 16q + 2j + h
+# of the gate rows (s = 0) or of the up rows (s = 1, source row I + f).  This row
+# order is the library's own layout choice; the pages fix none.
 
 def meta_nibble_from_mask_nibble(n: int) -> int:
     pos = [i for i in range(4) if (n >> i) & 1]
@@ -218,8 +221,9 @@ def tile_rows(out: int, gate_up: bool) -> np.ndarray:
     I = out // 2
     rows = []
     for t in range(out // 128):
-        rows.extend(range(64 * t, 64 * t + 64))
-        rows.extend(range(I + 64 * t, I + 64 * t + 64))
+        for r in range(128):
+            q, h, s, j = r // 32, (r // 16) % 2, (r // 8) % 2, r % 8
+            rows.append(s * I + 64 * t + 16 * q + 2 * j + h)
     return np.array(rows)
 
 

@@ -275,9 +275,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           for (int i = 1; i < STAGES; ++i)
             if (stage == i) bar = full_lead[i];
           if (lead) mbar_arrive_expect_tx(&S.full[stage], 2u * (A_BYTES + nc * b_box + E_BYTES + 2 * SF_BYTES));
-          // weight tile: gate rows 64mt.. and up rows I+64mt.. in one 4-D box,
-          // or 128 consecutive down rows
-          if (p.gate_up) tma_load_4d_pair(st, &tmap_a, kb * 128, 64 * mt, 0, t.e, bar);
+          // weight tile: the interleaved gate and up rows of outputs 64mt..64mt+63 in
+          // one 5-D box (byte, j, gate/up, h, 16-row group), or 128 consecutive down rows
+          if (p.gate_up) tma_load_5d_pair(st, &tmap_a, kb * 128, 0, 0, 0, t.e * (p.M / 16) + 4 * mt, bar);
           else tma_load_2d_pair(st, &tmap_a, kb * 128, t.e * p.M + BM * mt, bar);
           if (b3d && nc > 1 && !small) {  // 64-row chunks: chunk 1 lands at B_CHUNK as the MMA expects
             tma_load_3d_pair(st + A_BYTES, tb3, 0, brow, 2 * kb, bar);
@@ -404,10 +404,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       if (lead) mbar_arrive(&S.acc_empty[b]);
       else mbar_arrive_remote(b ? acc_empty_lead1 : acc_empty_lead0);
     };
-    // SwiGLU exchange: gate quarter q (0,1) pairs with up quarter q+2 on the same
-    // column block; each side hands the other a 16x32 block (column-major, lane-fast).
-    const int pair = (q & 1) + 2 * kb;           // 0..7
-    float* xch = epi + pair * 2 * 16 * 32;       // [2][16 cols][32 lanes]
     TileWalk walk(pair_id, npairs, MT2);
     int sb = 0;  // SwiGLU staging buffer of this tile
     for (int id = pair_id; id < total; id += npairs, walk.advance(MT2)) {
@@ -421,70 +417,78 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       const uint32_t tbase = tmem + TM_ACC + buf * BN + ((uint32_t)(32 * q) << 16);
       const bool live = c_lo < t.n_rows;        // any valid token column in the block
       if constexpr (EPI == MOESQ_EPI_SWIGLU_NVFP4) {
-        const bool is_gate = q < 2;
-        // gate warp finishes columns [c_lo, c_lo+16), up warp [c_lo+16, c_lo+32)
-        uint32_t mine[16], other[16];
+        // Tile rows are interleaved (weight repack): in lane quarter q, lanes 16h + j
+        // hold the gate rows and lanes 16h + 8 + j the up rows of output
+        // o = 16q + 2j + h of this CTA's 64.  A 16x256b load at lane 32q + 16h thus
+        // hands thread t the gate and up values of output 16q + 2(t/4) + h for the
+        // columns c_lo + 8i + 2(t%4) + b (i < 4, b < 2): no exchange between warps.
+        float hv[2][8];  // [h][v]: v = 2i + b
         if (live) {
-          tmem_ld_32x32b_x16(tbase + c_lo + (is_gate ? 16 : 0), other);
-          tmem_ld_32x32b_x16(tbase + c_lo + (is_gate ? 0 : 16), mine);
-          tmem_ld_wait();
+          uint32_t r[16];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            tmem_ld_16x256b_x4(tbase + ((uint32_t)(16 * h) << 16) + c_lo, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              const float gv = __fmul_rn(__uint_as_float(r[4 * (v >> 1) + (v & 1)]), alpha);
+              const float uv = __fmul_rn(__uint_as_float(r[4 * (v >> 1) + 2 + (v & 1)]), alpha);
+              hv[h][v] = __fmul_rn(silu_fast(gv), uv);
+            }
+          }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) release_acc(buf);
-        float* give = xch + (is_gate ? 0 : 1) * 512;
-        float* take = xch + (is_gate ? 1 : 0) * 512;  // read here, then reused for the transpose
         if (live) {
+          // amax of each column over this warp's 16 outputs: per thread over its two,
+          // then over the 8 lanes of equal t%4 (lane bits 2..4) by three halving
+          // exchanges; lane t ends with column v = (t >> 2) & 7 of its own t%4
+          float m[8];
 #pragma unroll
-          for (int c = 0; c < 16; ++c) give[c * 32 + lane] = __fmul_rn(__uint_as_float(other[c]), alpha);
-        }
-        named_bar_sync(2 + pair, 64);
-        const int cb = c_lo + (is_gate ? 0 : 16);   // first tile column finished here
-        if (live && cb < t.n_rows) {
-          // h for feature `lane` x 16 token columns
-          float hv[16];
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const float a = __fmul_rn(__uint_as_float(mine[c]), alpha);
-            const float b = take[c * 32 + lane];
-            const float gv = is_gate ? a : b, uv = is_gate ? b : a;
-            hv[c] = __fmul_rn(silu_fast(gv), uv);
-          }
-          // NVFP4 requant of each token column.  Transpose through the block just
-          // read: column c is one 128-byte row (feature f in 16-byte chunk
-          // (f/4) ^ (c&7), so both the row writes and the chunk reads below spread
-          // over the banks); lane = (column lane&15, feature half lane>>4) then
-          // reads its 16 features with four 16-byte loads.  Each lane of a column
-          // pair computes the scale from the joint amax; codes of adjacent
-          // features pack in-thread.
-          __syncwarp();
-#pragma unroll
-          for (int c = 0; c < 16; ++c) take[c * 32 + ((((lane >> 2) ^ c) & 7) << 2) + (lane & 3)] = hv[c];
-          __syncwarp();
-          const int tok = lane & 15, fh = lane >> 4;
-          float amax = 0.0f;
+          for (int v = 0; v < 8; ++v) m[v] = fmaxf(fabsf(hv[0][v]), fabsf(hv[1][v]));
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const int chunk = (4 * fh + k) ^ (tok & 7);
-            const float4 v = *reinterpret_cast<const float4*>(take + tok * 32 + 4 * chunk);
-            hv[4 * k] = v.x, hv[4 * k + 1] = v.y, hv[4 * k + 2] = v.z, hv[4 * k + 3] = v.w;
-            amax = fmaxf(fmaxf(amax, fmaxf(fabsf(v.x), fabsf(v.y))), fmaxf(fabsf(v.z), fabsf(v.w)));
+            const bool hi = lane & 16;
+            const float x = __shfl_xor_sync(0xffffffffu, hi ? m[k] : m[k + 4], 16);
+            m[k] = fmaxf(hi ? m[k + 4] : m[k], x);
           }
-          amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 16));
-          // stage this group's codes (16 features per lane) and scale for the block's write
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const bool hi = lane & 8;
+            const float x = __shfl_xor_sync(0xffffffffu, hi ? m[k] : m[k + 2], 8);
+            m[k] = fmaxf(hi ? m[k + 2] : m[k], x);
+          }
+          {
+            const bool hi = lane & 4;
+            const float x = __shfl_xor_sync(0xffffffffu, hi ? m[0] : m[1], 4);
+            m[0] = fmaxf(hi ? m[1] : m[0], x);
+          }
+          // the scale group (32 outputs) spans quarters q and q ^ 1, which use the
+          // same lane -> column map: swap the partial amax through shared memory
+          float* xa = epi + (kb * 4 + q) * 32;
+          xa[lane] = m[0];
+          named_bar_sync(2 + (q >> 1) + 2 * kb, 64);
+          const float amax = fmaxf(m[0], epi[(kb * 4 + (q ^ 1)) * 32 + lane]);
           const GroupScale gs = nvfp4_group_scale(amax, ag.y);
-          const int r = cb - c_lo + tok;  // token row within the column block
-          *reinterpret_cast<uint2*>(&S.hstg[sb][kb][r][16 * (q & 1) + 8 * fh]) =
-              make_uint2(nvfp4_word(hv, gs.inv), nvfp4_word(hv + 8, gs.inv));
-          if (fh == 0) S.sstg[sb][kb][r][q & 1] = (uint8_t)gs.sc;
+          const int vc = (lane >> 2) & 7;
+          const int rc = 8 * (vc >> 1) + 2 * (lane & 3) + (vc & 1);  // this lane's column (row of the block)
+          if ((q & 1) == 0) S.sstg[sb][kb][rc][q >> 1] = (uint8_t)gs.sc;
+          // codes: byte 8q + t/4 of each of this thread's 8 token rows (outputs 2(t/4) + {0,1})
+          uint8_t* stg = &S.hstg[sb][kb][0][8 * q + (lane >> 2)];
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            const float inv = __shfl_sync(0xffffffffu, gs.inv, (lane & 3) | (v << 2));
+            const uint32_t byte = inv == 0.0f ? 0u : e2m1x2(__fmul_rn(hv[0][v], inv), __fmul_rn(hv[1][v], inv));
+            stg[(8 * (v >> 1) + 2 * (lane & 3) + (v & 1)) * 32] = (uint8_t)byte;
+          }
         }
-        named_bar_sync(2 + pair, 64);  // the exchange block is free for the next tile
-        // the four warps of this column block hold all 64 features of its 32 tokens:
+        // the four warps of this column block hold all 64 outputs of its 32 tokens:
         // one TMA store of [32 rows][32 B] codes (rows past the expert's tokens are its
         // own padding, never read as tokens) and 2-byte scale pairs
         fence_proxy_async_smem();
         if (q == 0 && lane == 0) bulk_wait_group_read0();  // the store two tiles back has read its buffer
-        named_bar_sync(10 + kb, 128);
+        named_bar_sync(10 + kb, 128);  // also: both amax slots of every pair are read
         if (live) {
           const int64_t prow0 = (int64_t)t.prow + c_lo;
           if (q == 0 && lane == 0) {
@@ -503,10 +507,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // Stage the bf16 tile as two 64-feature halves [128 token rows][128 B] in
         // the TMA 128-byte swizzle (16-byte chunk j of row r at chunk j ^ (r & 7)),
         // then write it with two TMA tensor stores (full tiles) or a row-bounded
-        // copy (a ragged last tile of an expert).  Lane = feature: adjacent lanes
-        // swap one value so that each lane stores a bf16 pair of neighbouring
-        // features as one word; even lanes take column c, odd lanes column c + 4,
-        // whose rows fall on the other half of the banks.
+        // copy (a ragged last tile of an expert).  Lane = feature: the two lanes of
+        // neighbouring features (adjacent lanes for down; lanes 16 apart in the
+        // interleaved gate_up rows) swap one value so that each stores a bf16 pair
+        // as one word; the even feature's lane takes column c, the odd one column
+        // c + 4, whose rows fall on the other half of the banks.
         uint8_t* stg = reinterpret_cast<uint8_t*>(epi);  // 2 x 128 x 128 B
         const int64_t s0 = t.s0;
         int nvalid = t.n_rows;
@@ -522,9 +527,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         if (threadIdx.x == 64) bulk_wait_group_read0();  // the previous tile's stores have read the staging
         named_bar_sync(1, EPI_THREADS);                  // and every copy of it is done
         if (c_lo < nvalid) {
-          const int odd = lane & 1;
-          uint8_t* hb = stg + (q >> 1) * 16384;
-          const int w = 16 * (q & 1) + (lane >> 1);  // feature pair within the 64-feature half
+          const bool gu = p.gate_up;
+          const int odd = gu ? (lane >> 4) & 1 : lane & 1;
+          const int xl = gu ? 16 : 1;                               // the neighbouring feature's lane
+          uint8_t* hb = stg + (gu ? (lane >> 3) & 1 : q >> 1) * 16384;  // gate / up half (or rows 64..127)
+          const int w = gu ? 8 * q + (lane & 7) : 16 * (q & 1) + (lane >> 1);  // feature pair within the half
 #pragma unroll
           for (int c8 = 0; c8 < 32; c8 += 8) {
 #pragma unroll
@@ -532,7 +539,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
               const int c = c8 + c4;
               const float v0 = __fmul_rn(__uint_as_float(acc[c]), alpha);
               const float v1 = __fmul_rn(__uint_as_float(acc[c + 4]), alpha);
-              const float recv = __shfl_xor_sync(0xffffffffu, odd ? v0 : v1, 1);
+              const float recv = __shfl_xor_sync(0xffffffffu, odd ? v0 : v1, xl);
               const float lo = odd ? recv : v0, hi = odd ? v1 : recv;
               const int row = c_lo + c + 4 * odd;
               const __nv_bfloat162 pr = __floats2bfloat162_rn(lo, hi);
@@ -567,10 +574,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       } else {
         // f32: per 16-column half of the block, TMEM (lane = feature) -> swizzled
         // transpose in this warp's shared block -> lanes 0-15 = tokens, one
-        // 128-byte row segment each
+        // 128-byte row segment each (down), or two 64-byte segments, gate and up
+        // outputs 16q..16q+15 of the tile, from the interleaved lanes (gate_up)
         float* tr = epi + ew * 512;
-        const int col0 = p.gate_up ? (q < 2 ? 64 * mt + 32 * q : I + 64 * mt + 32 * (q - 2))
-                                   : BM * mt + 32 * q;
+        const bool gu = p.gate_up;
+        const int col0 = BM * mt + 32 * q;
         const int64_t s0 = t.s0;
         int nvalid = t.n_rows;                     // valid columns of the tile
         if (s0 + nvalid > p.S) nvalid = (int)(p.S - s0 > 0 ? p.S - s0 : 0);
@@ -597,8 +605,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
               for (int u = 0; u < 8; ++u) {
                 float v[4];
 #pragma unroll
-                for (int z = 0; z < 4; ++z) v[z] = __fmul_rn(row[(4 * u + z) ^ lane], alpha);
-                y[u] = make_float4(v[0], v[1], v[2], v[3]);
+                for (int z = 0; z < 4; ++z) {
+                  // output position 4u + z: segment s = pos / 16 at offset o = pos % 16
+                  // comes from lane 16 (o & 1) + 8 s + o / 2 in the interleaved rows
+                  const int pos = 4 * u + z;
+                  const int src = gu ? (((pos & 1) << 4) | ((pos >> 4) << 3) | ((pos & 15) >> 1)) : pos;
+                  v[z] = __fmul_rn(row[src ^ lane], alpha);
+                }
+                if (gu) {
+                  float* yg = (float*)p.out + s * p.M + (u >= 4 ? I : 0) + 64 * mt + 16 * q + 4 * (u & 3);
+                  *reinterpret_cast<float4*>(yg) = make_float4(v[0], v[1], v[2], v[3]);
+                } else {
+                  y[u] = make_float4(v[0], v[1], v[2], v[3]);
+                }
               }
             }
             __syncwarp();
@@ -725,17 +744,21 @@ extern "C" moesq_status moesq_grouped_gemm(const moesq_linear* W, const uint8_t*
   if (sms < 0) return MOESQ_ERR_CUDA;
   if (sms == 0) return MOESQ_ERR_DEVICE;
 
-  // Weight tile: 512 dense K = 128 compressed bytes per row.  gate_up tiles take
-  // 64 gate rows and the 64 up rows of the same features: a 4-D view
-  // (byte, row in half, half, expert) loads both halves with one copy.
+  // Weight tile: 512 dense K = 128 compressed bytes per row.  A gate_up tile holds
+  // the gate and up rows of 64 outputs in the interleaved order of the weight repack
+  // (tile row 32q + 16h + 8s + j = row s*I + 16q + 2j + h of the tile's outputs):
+  // a 5-D view (byte, j [stride 2 rows], s [stride I rows], h [stride 1 row],
+  // 16-row group [stride 16 rows, expert folded in]) loads it with one copy.  Only
+  // coordinates of whole tiles are used, so every byte read lies in the weights.
   CUtensorMap ta, tb, tb16, te, tsfa, tsfb;
   const uint64_t rowA = (uint64_t)(W->K / 4);
   const int64_t MT = W->out / 128, kb128 = W->K / 128, nkb256 = (W->K + 255) / 256;
   if (gate_up) {
-    const cuuint64_t dims[4] = {rowA, (uint64_t)(W->out / 2), 2, (uint64_t)W->E};
-    const cuuint64_t strides[3] = {rowA, rowA * (uint64_t)(W->out / 2), rowA * (uint64_t)W->out};
-    const cuuint32_t box[4] = {128, 64, 2, 1};
-    if (!make_tmap_u8(&ta, W->packed, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+    const uint64_t I = (uint64_t)(W->out / 2);
+    const cuuint64_t dims[5] = {rowA, 8, 2, 2, (uint64_t)(W->E * W->out / 16)};
+    const cuuint64_t strides[4] = {2 * rowA, I * rowA, rowA, 16 * rowA};
+    const cuuint32_t box[5] = {128, 8, 2, 2, 4};
+    if (!make_tmap_u8(&ta, W->packed, 5, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
       return MOESQ_ERR_CUDA;
   } else if (!make_tmap_rows(&ta, W->packed, rowA, (uint64_t)(W->E * W->out), 128, 128,
                              CU_TENSOR_MAP_SWIZZLE_128B)) {

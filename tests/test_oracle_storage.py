@@ -199,6 +199,12 @@ def test_sparse_metadata_golden(golden):
     rows = S.tile_rows(tr["out"], True)
     assert rows[128 * tr["tile"] + tr["tile_row"]] == tr["source_row"]
     assert rows[128 * tr["tile_b"] + tr["tile_row_b"]] == tr["source_row_b"]
+    assert rows[128 * tr["tile_c"] + tr["tile_row_c"]] == tr["source_row_c"]
+    # each tile holds the gate and up rows of the same 64 outputs, once each
+    I = tr["out"] // 2
+    for t in range(tr["out"] // 128):
+        blk = rows[128 * t:128 * t + 128]
+        assert sorted(blk) == list(range(64 * t, 64 * t + 64)) + list(range(I + 64 * t, I + 64 * t + 64))
     sf = g["sf_offset_example"]
     assert S.sf_block_offset(sf["row"], sf["j"]) == sf["offset"]
 
