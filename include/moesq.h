@@ -153,7 +153,8 @@ moesq_status moesq_repack_sizes(int64_t out, int64_t K, size_t* meta_bytes, size
  *   sf     device u8 [E * sf_bytes]: per expert, per tile, per 128 dense K a 512-byte
  *          block, row r scale j at (r%32)*16 + (r/32)*4 + j
  *   alpha_w device f32 [E]: the weight global the GEMM applies (gate global for gate_up)
- * Tile row order: DOWN identity; GATE_UP tile t holds the gate and up rows of outputs
+ * Tile row order: DOWN tile t holds rows 128t..128t+127, tile row 16g + 8p + j being
+ * row 128t + 16g + 2j + p (g < 8; p < 2; j < 8); GATE_UP tile t holds the gate and up rows of outputs
  * 64t..64t+63: tile row r = 32q + 16h + 8s + j (q < 4; h, s < 2; j < 8) is source row
  * s*I + 64t + 16q + 2j + h.  The packed values are used as stored (no repack).
  * out % 128 == 0, K % 128 == 0.  Bad nibbles raise MOESQ_DFLAG_BAD_SPARSITY. */

@@ -197,8 +197,10 @@ def fold_up_scales(scale_up, g_gate, g_up) -> np.ndarray:
 #     row r scale j at (r % 32) * 16 + (r // 32) * 4 + j.
 # The library lays out whole operands as
 #   meta[e][tile][kb256][128][16]   sfw[e][tile][kb128][512]   sfa[pb][kb128][512]
-# where "tile" is a 128-row block of the weight in tile row order: for down the
-# identity; for fused gate_up, tile t holds the gate and the up rows of the same
+# where "tile" is a 128-row block of the weight in tile row order.  For down,
+# tile t holds rows 128t..128t+127 with neighbouring rows 8 apart inside each
+# 16-row group (tile row 16g + 8p + j is row 128t + 16g + 2j + p), so that one TMEM
+# load gives a thread both outputs of a bf16 pair.  For fused gate_up, tile t holds the gate and the up rows of the same
 # 64 outputs 64t..64t+63, interleaved so that the SwiGLU epilogue finds a gate
 # value and its up value, for two adjacent outputs, in one thread: tile row
 # r = 32q + 16h + 8s + j (q < 4, h, s < 2, j < 8) is output f = 64t + 16q + 2j + h
@@ -217,7 +219,8 @@ def tile_rows(out: int, gate_up: bool) -> np.ndarray:
     if out % 128:
         raise ValueError("out must be a multiple of 128")
     if not gate_up:
-        return np.arange(out)
+        r = np.arange(out)
+        return (r // 16) * 16 + 2 * (r % 8) + (r // 8) % 2
     I = out // 2
     rows = []
     for t in range(out // 128):

@@ -275,10 +275,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           for (int i = 1; i < STAGES; ++i)
             if (stage == i) bar = full_lead[i];
           if (lead) mbar_arrive_expect_tx(&S.full[stage], 2u * (A_BYTES + nc * b_box + E_BYTES + 2 * SF_BYTES));
-          // weight tile: the interleaved gate and up rows of outputs 64mt..64mt+63 in
-          // one 5-D box (byte, j, gate/up, h, 16-row group), or 128 consecutive down rows
+          // weight tile in the repack's interleaved row order: gate and up rows of
+          // outputs 64mt..64mt+63 in one 5-D box (byte, j, gate/up, h, 16-row group), or
+          // down rows 128mt.. in one 4-D box (byte, j, p, 16-row group)
           if (p.gate_up) tma_load_5d_pair(st, &tmap_a, kb * 128, 0, 0, 0, t.e * (p.M / 16) + 4 * mt, bar);
-          else tma_load_2d_pair(st, &tmap_a, kb * 128, t.e * p.M + BM * mt, bar);
+          else tma_load_4d_pair(st, &tmap_a, kb * 128, 0, 0, (t.e * p.M + BM * mt) / 16, bar);
           if (b3d && nc > 1 && !small) {  // 64-row chunks: chunk 1 lands at B_CHUNK as the MMA expects
             tma_load_3d_pair(st + A_BYTES, tb3, 0, brow, 2 * kb, bar);
           } else {
@@ -504,78 +505,83 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
         sb ^= 1;
       } else if constexpr (EPI == MOESQ_EPI_BF16) {
-        // Stage the bf16 tile as two 64-feature halves [128 token rows][128 B] in
-        // the TMA 128-byte swizzle (16-byte chunk j of row r at chunk j ^ (r & 7)),
-        // then write it with two TMA tensor stores (full tiles) or a row-bounded
-        // copy (a ragged last tile of an expert).  Lane = feature: the two lanes of
-        // neighbouring features (adjacent lanes for down; lanes 16 apart in the
-        // interleaved gate_up rows) swap one value so that each stores a bf16 pair
-        // as one word; the even feature's lane takes column c, the odd one column
-        // c + 4, whose rows fall on the other half of the banks.
-        uint8_t* stg = reinterpret_cast<uint8_t*>(epi);  // 2 x 128 x 128 B
+        // Per 32-token column block kb, its four warps (one per lane quarter q) stage
+        // [32 tokens][128 outputs] bf16 as two 64-output halves [32 rows][128 B] in the
+        // TMA 128-byte swizzle (16-byte chunk c of row r at c ^ (r & 7)), then one lane
+        // writes them with two TMA stores, or the 128 threads copy the valid rows when
+        // the block reaches past the expert's tokens.  The interleaved weight rows put
+        // both outputs of a bf16 pair in one thread of a 16x256b TMEM load (down:
+        // lanes j and 8 + j of a 16-lane group; gate_up: gate or up of outputs
+        // 16q + 2j + {0,1} from the loads at lane 32q and 32q + 16), so each pair
+        // is one word and no lanes exchange values.  Words of one store land on 8
+        // consecutive pair slots of 4 rows two apart: no bank conflicts.
+        uint8_t* stg = reinterpret_cast<uint8_t*>(epi) + kb * 8192;  // [2 halves][32 rows][128 B]
         const int64_t s0 = t.s0;
         int nvalid = t.n_rows;
         if (s0 + nvalid > p.S) nvalid = (int)(p.S - s0 > 0 ? p.S - s0 : 0);
-        uint32_t acc[32];
-        if (c_lo < nvalid) {
-          tmem_ld_32x32b_x32(tbase + c_lo, acc);
+        const int nblk = min(32, nvalid - c_lo);  // valid rows of this block (<= 0: none)
+        uint32_t r0[16], r1[16];
+        if (nblk > 0) {
+          tmem_ld_16x256b_x4(tbase + c_lo, r0);
+          tmem_ld_16x256b_x4(tbase + (16u << 16) + c_lo, r1);
           tmem_ld_wait();
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) release_acc(buf);
-        if (threadIdx.x == 64) bulk_wait_group_read0();  // the previous tile's stores have read the staging
-        named_bar_sync(1, EPI_THREADS);                  // and every copy of it is done
-        if (c_lo < nvalid) {
-          const bool gu = p.gate_up;
-          const int odd = gu ? (lane >> 4) & 1 : lane & 1;
-          const int xl = gu ? 16 : 1;                               // the neighbouring feature's lane
-          uint8_t* hb = stg + (gu ? (lane >> 3) & 1 : q >> 1) * 16384;  // gate / up half (or rows 64..127)
-          const int w = gu ? 8 * q + (lane & 7) : 16 * (q & 1) + (lane >> 1);  // feature pair within the half
+        const bool issuer = q == 0 && lane == 0;
+        if (issuer) bulk_wait_group_read0();  // this block's previous stores have read the staging
+        named_bar_sync(10 + kb, 128);         // (and its previous row copy is done)
+        const bool gu = p.gate_up;
+        if (nblk > 0) {
+          const int j = lane >> 2;
+          // pair slots and halves of the thread's two words per column
+          const int w0 = gu ? 8 * q + j : 16 * (q & 1) + j;
+          const int w1 = gu ? w0 : w0 + 8;
+          uint8_t* h0 = stg + (gu ? 0 : (q >> 1) * 4096);
+          uint8_t* h1 = stg + (gu ? 4096 : (q >> 1) * 4096);
 #pragma unroll
-          for (int c8 = 0; c8 < 32; c8 += 8) {
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-              const int c = c8 + c4;
-              const float v0 = __fmul_rn(__uint_as_float(acc[c]), alpha);
-              const float v1 = __fmul_rn(__uint_as_float(acc[c + 4]), alpha);
-              const float recv = __shfl_xor_sync(0xffffffffu, odd ? v0 : v1, xl);
-              const float lo = odd ? recv : v0, hi = odd ? v1 : recv;
-              const int row = c_lo + c + 4 * odd;
-              const __nv_bfloat162 pr = __floats2bfloat162_rn(lo, hi);
-              *reinterpret_cast<uint32_t*>(hb + row * 128 + (((w >> 2) ^ (row & 7)) << 4) + ((w & 3) << 2)) =
-                  *reinterpret_cast<const uint32_t*>(&pr);
-            }
+          for (int v = 0; v < 8; ++v) {
+            const int i = v >> 1, b = v & 1;
+            const int row = 8 * i + 2 * (lane & 3) + b;
+            const float a0 = __uint_as_float(r0[4 * i + b]), a1 = __uint_as_float(r0[4 * i + 2 + b]);
+            const float c0 = __uint_as_float(r1[4 * i + b]), c1 = __uint_as_float(r1[4 * i + 2 + b]);
+            // down: (a0, a1) and (c0, c1) are output pairs; gate_up: (a0, c0) gate, (a1, c1) up
+            const __nv_bfloat162 p0 = __floats2bfloat162_rn(__fmul_rn(a0, alpha), __fmul_rn(gu ? c0 : a1, alpha));
+            const __nv_bfloat162 p1 = __floats2bfloat162_rn(__fmul_rn(gu ? a1 : c0, alpha), __fmul_rn(c1, alpha));
+            *reinterpret_cast<__nv_bfloat162*>(h0 + row * 128 + (((w0 >> 2) ^ (row & 7)) << 4) + ((w0 & 3) << 2)) = p0;
+            *reinterpret_cast<__nv_bfloat162*>(h1 + row * 128 + (((w1 >> 2) ^ (row & 7)) << 4) + ((w1 & 3) << 2)) = p1;
           }
         }
         fence_proxy_async_smem();
-        named_bar_sync(1, EPI_THREADS);  // staging tile complete
-        const int x0 = p.gate_up ? 64 * mt : BM * mt;            // first column of half 0
-        const int x1 = p.gate_up ? I + 64 * mt : BM * mt + 64;   // and of half 1
-        if (own_tile && nvalid == BN) {
-          if (threadIdx.x == 64) {
-            tma_store_2d(&tmap_y, stg, x0, (int32_t)s0);
-            tma_store_2d(&tmap_y, stg + 16384, x1, (int32_t)s0);
+        named_bar_sync(10 + kb, 128);  // staging of the block complete
+        const int x0 = gu ? 64 * mt : BM * mt;            // first column of half 0
+        const int x1 = gu ? I + 64 * mt : BM * mt + 64;   // and of half 1
+        if (own_tile && nblk == 32) {
+          if (issuer) {
+            tma_store_2d(&tmap_y, stg, x0, (int32_t)(s0 + c_lo));
+            tma_store_2d(&tmap_y, stg + 4096, x1, (int32_t)(s0 + c_lo));
             bulk_commit_group();
           }
-        } else if (own_tile) {
+        } else if (own_tile && nblk > 0) {
           // 16-byte chunk i: row i >> 4, half (i >> 3) & 1, chunk i & 7 of the half row
-          const int et = threadIdx.x - 64;  // 0..511
+          const int et = 32 * q + lane;  // 0..127 within the block
 #pragma unroll
           for (int i0 = 0; i0 < 4; ++i0) {
-            const int i = et + EPI_THREADS * i0;
-            const int r = i >> 4, half = (i >> 3) & 1, j = i & 7;
-            if (r < nvalid) {
-              const uint4 v = *reinterpret_cast<const uint4*>(stg + half * 16384 + r * 128 + ((j ^ (r & 7)) << 4));
-              *reinterpret_cast<uint4*>((uint16_t*)p.out + (s0 + r) * p.M + (half ? x1 : x0) + 8 * j) = v;
+            const int i = et + 128 * i0;
+            const int r = i >> 4, half = (i >> 3) & 1, jj = i & 7;
+            if (r < nblk) {
+              const uint4 v = *reinterpret_cast<const uint4*>(stg + half * 4096 + r * 128 + ((jj ^ (r & 7)) << 4));
+              *reinterpret_cast<uint4*>((uint16_t*)p.out + (s0 + c_lo + r) * p.M + (half ? x1 : x0) + 8 * jj) = v;
             }
           }
         }
       } else {
         // f32: per 16-column half of the block, TMEM (lane = feature) -> swizzled
         // transpose in this warp's shared block -> lanes 0-15 = tokens, one
-        // 128-byte row segment each (down), or two 64-byte segments, gate and up
-        // outputs 16q..16q+15 of the tile, from the interleaved lanes (gate_up)
+        // 128-byte row segment each (down: output 16h + 2j + p of the quarter from
+        // lane 16h + 8p + j), or two 64-byte segments, gate and up outputs
+        // 16q..16q+15 of the tile, from the interleaved lanes (gate_up)
         float* tr = epi + ew * 512;
         const bool gu = p.gate_up;
         const int col0 = BM * mt + 32 * q;
@@ -609,7 +615,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                   // output position 4u + z: segment s = pos / 16 at offset o = pos % 16
                   // comes from lane 16 (o & 1) + 8 s + o / 2 in the interleaved rows
                   const int pos = 4 * u + z;
-                  const int src = gu ? (((pos & 1) << 4) | ((pos >> 4) << 3) | ((pos & 15) >> 1)) : pos;
+                  const int src = gu ? (((pos & 1) << 4) | ((pos >> 4) << 3) | ((pos & 15) >> 1))
+                                     : ((pos & 16) | ((pos & 1) << 3) | ((pos & 15) >> 1));
                   v[z] = __fmul_rn(row[src ^ lane], alpha);
                 }
                 if (gu) {
@@ -629,11 +636,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     }
   }
 
-  if constexpr (EPI == MOESQ_EPI_BF16) {
-    if (threadIdx.x == 64) bulk_wait_group0();  // the last tile's stores are complete
-  }
-  if constexpr (EPI == MOESQ_EPI_SWIGLU_NVFP4) {
-    if (warp >= 2 && (warp & 3) == 0 && lane == 0) bulk_wait_group0();
+  if constexpr (EPI == MOESQ_EPI_BF16 || EPI == MOESQ_EPI_SWIGLU_NVFP4) {
+    if (warp >= 2 && (warp & 3) == 0 && lane == 0) bulk_wait_group0();  // the last stores are complete
   }
   // no CTA of the pair frees TMEM or exits while its peer may still use it
   tc_fence_before();
@@ -760,9 +764,13 @@ extern "C" moesq_status moesq_grouped_gemm(const moesq_linear* W, const uint8_t*
     const cuuint32_t box[5] = {128, 8, 2, 2, 4};
     if (!make_tmap_u8(&ta, W->packed, 5, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
       return MOESQ_ERR_CUDA;
-  } else if (!make_tmap_rows(&ta, W->packed, rowA, (uint64_t)(W->E * W->out), 128, 128,
-                             CU_TENSOR_MAP_SWIZZLE_128B)) {
-    return MOESQ_ERR_CUDA;
+  } else {
+    // down: tile row 16g + 8p + j = row 16g + 2j + p of the tile: (byte, j [stride 2
+    // rows], p [stride 1 row], 16-row group [stride 16 rows, expert folded in])
+    const cuuint64_t dims[4] = {rowA, 8, 2, (uint64_t)(W->E * W->out / 16)};
+    const cuuint64_t strides[3] = {2 * rowA, rowA, 16 * rowA};
+    const cuuint32_t box[4] = {128, 8, 2, 8};
+    if (!make_tmap_u8(&ta, W->packed, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MOESQ_ERR_CUDA;
   }
   // token codes: a CTA stages 64 (or, for tiles of <= 32 tokens, 16) rows
   if (!make_tmap_rows(&tb, act_codes, (uint64_t)(W->K / 2), (uint64_t)P_cap, 128, 64,
@@ -800,7 +808,7 @@ extern "C" moesq_status moesq_grouped_gemm(const moesq_linear* W, const uint8_t*
     PFN_encodeTiled enc = get_encode_fn();
     const cuuint64_t dims[2] = {(uint64_t)W->out, (uint64_t)S};
     const cuuint64_t strides[1] = {(uint64_t)W->out * 2};
-    const cuuint32_t box[2] = {64, 128}, estr[2] = {1, 1};
+    const cuuint32_t box[2] = {64, 32}, estr[2] = {1, 1};
     if (!enc || enc(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out, dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)

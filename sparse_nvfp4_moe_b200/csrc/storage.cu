@@ -265,11 +265,13 @@ __global__ void k_quant_encode(const uint16_t* __restrict__ w, int64_t E, int64_
 // metadata: thread per (expert, tile, kb256, tile row): 16 mask bytes -> 16 metadata
 // bytes.  The metadata nibble of a chunk is i0 | i1 << 2, its kept pair indices
 // (lowest and highest set bit of the mask nibble).
-// Source row of tile row r.  gate_up: row r = 32q + 16h + 8s + j of tile t is output
-// f = 64t + 16q + 2j + h of the gate (s = 0) or up (s = 1) rows, so that one TMEM
-// load of 16 lanes gives a thread the gate and up values of output f.
+// Source row of tile row r.  down: row r = 16g + 8p + j of tile t is row
+// 128t + 16g + 2j + p, so that one TMEM load of 16 lanes gives a thread two
+// neighbouring outputs.  gate_up: row r = 32q + 16h + 8s + j of tile t is output
+// f = 64t + 16q + 2j + h of the gate (s = 0) or up (s = 1) rows, so that the same
+// load gives a thread the gate and up values of output f.
 __device__ __forceinline__ int64_t tile_src_row(int64_t tile, int64_t r, int64_t out, bool gate_up) {
-  if (!gate_up) return 128 * tile + r;
+  if (!gate_up) return 128 * tile + (r & ~15) + 2 * (r & 7) + ((r >> 3) & 1);
   const int64_t I = out / 2;
   const int64_t q = r >> 5, h = (r >> 4) & 1, s = (r >> 3) & 1, j = r & 7;
   return s * I + 64 * tile + 16 * q + 2 * j + h;
