@@ -316,7 +316,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     if (lead && elect_one()) {
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t acc_phase[2] = {0u, 0u};
+      uint32_t acc_phase = 0u;  // bit b: phase of accumulator buffer b (a register, not an indexed array)
       int buf = 0;
       // Shared-memory descriptors of stage 0 (the same offsets hold the peer's
       // operands); a stage or a K offset only moves the 14-bit start-address
@@ -335,7 +335,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const int n_mma = max(16, (t.n_rows + 15) / 16 * 16);
         const uint32_t idesc = make_idesc((uint32_t)n_mma);
         const uint32_t d_tmem = tmem + TM_ACC + buf * BN;
-        mbar_wait_spin(&S.acc_empty[buf], acc_phase[buf] ^ 1, abort, p.d_status);
+        mbar_wait_spin(&S.acc_empty[buf], ((acc_phase >> buf) & 1u) ^ 1u, abort, p.d_status);
         tc_fence_after();
         for (int kb = 0; kb < nkb; ++kb) {
           mbar_wait_spin(&S.full[stage], phase, abort, p.d_status);
@@ -378,7 +378,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           }
         }
         tc_commit_pair_mc(&S.acc_full[buf], 0x3);
-        acc_phase[buf] ^= 1;
+        acc_phase ^= 1u << buf;
         buf ^= 1;
       }
       // drain: all tensor-core work of the pair complete before TMEM is freed
@@ -395,7 +395,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const int q = warp & 3;             // TMEM lane quarter this warp may access
     const int kb = ew >> 2;             // column block
     const int c_lo = 32 * kb;           // first column of this warp's block
-    uint32_t acc_phase[2] = {0u, 0u};
+    uint32_t acc_phase = 0u;  // bit b: phase of accumulator buffer b
     int buf = 0;
     const int I = p.M / 2;
     // accumulator buffer released to CTA 0's MMA warp: a local arrive in CTA 0,
@@ -413,7 +413,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       const bool own_tile = mt < MT;          // false: the duplicate of an odd last tile
       const float2 ag = S.ag[t.e];
       const float alpha = ag.x;
-      mbar_wait_poll(&S.acc_full[buf], acc_phase[buf], abort, p.d_status);
+      mbar_wait_poll(&S.acc_full[buf], (acc_phase >> buf) & 1u, abort, p.d_status);
       tc_fence_after();
       const uint32_t tbase = tmem + TM_ACC + buf * BN + ((uint32_t)(32 * q) << 16);
       const bool live = c_lo < t.n_rows;        // any valid token column in the block
@@ -631,7 +631,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           }
         }
       }
-      acc_phase[buf] ^= 1;
+      acc_phase ^= 1u << buf;
       buf ^= 1;
     }
   }
