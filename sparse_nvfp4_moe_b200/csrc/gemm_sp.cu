@@ -116,11 +116,18 @@ struct Tile {
 // Work items run over (token tile q, weight-tile pair m), m fastest; pair `pid`
 // of `npairs` takes items pid, pid + npairs, ...  Every role walks its items in
 // that order, stepping (q, m) by a precomputed (dq, dm) and the expert forward
-// from the previous item's, so no role divides or searches between tiles.
+// from the previous item's, so no role divides or searches between tiles.  The
+// current expert's record is kept in registers and the next expert's is loaded
+// as soon as the walk enters an expert, so the shared-memory load is consumed a
+// tile later (its latency is hidden behind the tile's work).
 struct TileWalk {
   int q, m, dq, dm, e;
-  __device__ __forceinline__ TileWalk(int pid, int npairs, int MT2)
-      : q(pid / MT2), m(pid % MT2), dq(npairs / MT2), dm(npairs % MT2), e(0) {}
+  int4 cur, nxt;  // rec[e], rec[e + 1] (rec[e] again past the last expert)
+  __device__ __forceinline__ TileWalk(const Smem& s, int pid, int npairs, int MT2, int E)
+      : q(pid / MT2), m(pid % MT2), dq(npairs / MT2), dm(npairs % MT2), e(0) {
+    cur = s.rec[0];
+    nxt = E > 1 ? s.rec[1] : cur;
+  }
   __device__ __forceinline__ void advance(int MT2) {
     m += dm;
     q += dq;
@@ -134,8 +141,12 @@ struct TileWalk {
 // The current item of `w` (empty experts are stepped over: their tiles end
 // where they start).
 __device__ __forceinline__ Tile decode_tile(const Smem& s, TileWalk& w, int E) {
-  int4 r = s.rec[w.e];
-  while (r.x <= w.q && w.e + 1 < E) r = s.rec[++w.e];
+  while (w.cur.x <= w.q && w.e + 1 < E) {
+    ++w.e;
+    w.cur = w.nxt;
+    w.nxt = w.e + 1 < E ? s.rec[w.e + 1] : w.cur;
+  }
+  const int4 r = w.cur;
   Tile t;
   t.e = w.e;
   t.mt = w.m;
@@ -244,7 +255,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       long fills = 0;
-      TileWalk walk(pair_id, npairs, MT2);
+      TileWalk walk(S, pair_id, npairs, MT2, E);
       uint32_t full_lead[STAGES];
 #pragma unroll
       for (int i = 0; i < STAGES; ++i) full_lead[i] = cluster_map(&S.full[i], 0);
@@ -329,7 +340,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       const uint64_t dSFA0 = smem_desc(s0 + A_BYTES + B_BYTES + E_BYTES, 16, 128, SWZ_NONE);
       const uint64_t dSFB0 = dSFA0 + (SF_BYTES >> 4);
       const uint32_t tE = tmem + TM_E, tSFA = tmem + TM_SFA, tSFB = tmem + TM_SFB;
-      TileWalk walk(pair_id, npairs, MT2);
+      TileWalk walk(S, pair_id, npairs, MT2, E);
       for (int id = pair_id; id < total; id += npairs, walk.advance(MT2)) {
         const Tile t = decode_tile(S, walk, E);
         const int n_mma = max(16, (t.n_rows + 15) / 16 * 16);
@@ -405,7 +416,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       if (lead) mbar_arrive(&S.acc_empty[b]);
       else mbar_arrive_remote(b ? acc_empty_lead1 : acc_empty_lead0);
     };
-    TileWalk walk(pair_id, npairs, MT2);
+    TileWalk walk(S, pair_id, npairs, MT2, E);
     int sb = 0;  // SwiGLU staging buffer of this tile
     for (int id = pair_id; id < total; id += npairs, walk.advance(MT2)) {
       const Tile t = decode_tile(S, walk, E);
