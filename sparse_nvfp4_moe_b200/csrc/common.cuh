@@ -80,6 +80,26 @@ __device__ __forceinline__ float silu_fast(float x) {
   return __fdividef(x, 1.0f + __expf(-x));
 }
 
+// ex2.approx / rcp.approx (PTX ISA), denormal outputs flushed to zero
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// silu of two values with packed (f32x2) multiplies and adds: x / (1 + 2^(-x log2 e)),
+// the exponential and the reciprocal on the MUFU (the same arithmetic as silu_fast).
+// Where 1 + e >= 2^126 the reciprocal flushes to 0 and so does silu.
+__device__ __forceinline__ float2 silu2(float2 x) {
+  const float2 t = __fmul2_rn(x, make_float2(-1.4426950408889634f, -1.4426950408889634f));
+  const float2 d = __fadd2_rn(make_float2(ex2_approx(t.x), ex2_approx(t.y)), make_float2(1.0f, 1.0f));
+  return __fmul2_rn(x, make_float2(rcp_approx(d.x), rcp_approx(d.y)));
+}
+
 // E4M3 (finite, saturating) code of a nonnegative float32, nearest-even.
 __device__ __forceinline__ uint32_t e4m3_code(float s) {
   return (uint32_t)__nv_cvt_float_to_fp8(s, __NV_SATFINITE, __NV_E4M3);

@@ -437,15 +437,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         float hv[2][8];  // [h][v]: v = 2i + b
         if (live) {
           uint32_t r[16];
+          const float2 al2 = make_float2(alpha, alpha);
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             tmem_ld_16x256b_x4(tbase + ((uint32_t)(16 * h) << 16) + c_lo, r);
             tmem_ld_wait();
 #pragma unroll
-            for (int v = 0; v < 8; ++v) {
-              const float gv = __fmul_rn(__uint_as_float(r[4 * (v >> 1) + (v & 1)]), alpha);
-              const float uv = __fmul_rn(__uint_as_float(r[4 * (v >> 1) + 2 + (v & 1)]), alpha);
-              hv[h][v] = __fmul_rn(silu_fast(gv), uv);
+            for (int i = 0; i < 4; ++i) {  // columns b = 0, 1 as one packed pair
+              const float2 g = __fmul2_rn(make_float2(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1])), al2);
+              const float2 u = __fmul2_rn(make_float2(__uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3])), al2);
+              const float2 hh = __fmul2_rn(silu2(g), u);
+              hv[h][2 * i] = hh.x;
+              hv[h][2 * i + 1] = hh.y;
             }
           }
         }
@@ -491,7 +494,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int v = 0; v < 8; ++v) {
             const float inv = __shfl_sync(0xffffffffu, gs.inv, (lane & 3) | (v << 2));
-            const uint32_t byte = inv == 0.0f ? 0u : e2m1x2(__fmul_rn(hv[0][v], inv), __fmul_rn(hv[1][v], inv));
+            const float2 x = __fmul2_rn(make_float2(hv[0][v], hv[1][v]), make_float2(inv, inv));
+            const uint32_t byte = inv == 0.0f ? 0u : e2m1x2(x.x, x.y);
             stg[(8 * (v >> 1) + 2 * (lane & 3) + (v & 1)) * 32] = (uint8_t)byte;
           }
         }
@@ -558,8 +562,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             const float a0 = __uint_as_float(r0[4 * i + b]), a1 = __uint_as_float(r0[4 * i + 2 + b]);
             const float c0 = __uint_as_float(r1[4 * i + b]), c1 = __uint_as_float(r1[4 * i + 2 + b]);
             // down: (a0, a1) and (c0, c1) are output pairs; gate_up: (a0, c0) gate, (a1, c1) up
-            const __nv_bfloat162 p0 = __floats2bfloat162_rn(__fmul_rn(a0, alpha), __fmul_rn(gu ? c0 : a1, alpha));
-            const __nv_bfloat162 p1 = __floats2bfloat162_rn(__fmul_rn(gu ? a1 : c0, alpha), __fmul_rn(c1, alpha));
+            const float2 w0v = __fmul2_rn(make_float2(a0, gu ? c0 : a1), make_float2(alpha, alpha));
+            const float2 w1v = __fmul2_rn(make_float2(gu ? a1 : c0, c1), make_float2(alpha, alpha));
+            const __nv_bfloat162 p0 = __floats2bfloat162_rn(w0v.x, w0v.y);
+            const __nv_bfloat162 p1 = __floats2bfloat162_rn(w1v.x, w1v.y);
             *reinterpret_cast<__nv_bfloat162*>(h0 + row * 128 + (((w0 >> 2) ^ (row & 7)) << 4) + ((w0 & 3) << 2)) = p0;
             *reinterpret_cast<__nv_bfloat162*>(h1 + row * 128 + (((w1 >> 2) ^ (row & 7)) << 4) + ((w1 & 3) << 2)) = p1;
           }
