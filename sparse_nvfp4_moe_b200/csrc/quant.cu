@@ -101,14 +101,22 @@ __global__ void k_quant_act_routed(const uint16_t* __restrict__ x, int64_t T, in
     float amax = 0.0f;
 #pragma unroll
     for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(v[j]));
+    // the codes and scale depend on the slot only through its expert's global: a
+    // slot whose global equals the previous slot's (bit for bit) reuses them
+    float g_prev = 0.0f;
+    GroupScale gs = {0u, 0.0f};
+    uint32_t o[4] = {0u, 0u, 0u, 0u};
     for (int j = 0; j < k; ++j) {
       int e = topk_ids[t * k + j];
       if (e < 0 || e >= E) e = 0;
       const int64_t s = token_slot[t * k + j];
-      const GroupScale gs = nvfp4_group_scale(amax, g_in[e]);
-      uint32_t o[4];
+      const float g = g_in[e];
+      if (j == 0 || __float_as_uint(g) != __float_as_uint(g_prev)) {
+        g_prev = g;
+        gs = nvfp4_group_scale(amax, g);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) o[c] = nvfp4_word(v + 8 * c, gs.inv);
+        for (int c = 0; c < 4; ++c) o[c] = nvfp4_word(v + 8 * c, gs.inv);
+      }
       const int64_t row = (int64_t)pad_offsets[e] + (s - expert_offsets[e]);
       *reinterpret_cast<uint4*>(codes + row * (K / 2) + 16 * grp) = make_uint4(o[0], o[1], o[2], o[3]);
       const int64_t blk = (row / 128) * (K / 128) + grp / 4;

@@ -129,14 +129,19 @@ def test_combine_golden_on_gpu(golden):
 
 @pytest.mark.parametrize("cfg_name,T", [("tiny", 64), ("qwen3_30b_a3b", 512), ("qwen3_5_397b_a17b", 16),
                                         ("kimi_k2", 32)])
-def test_quant_act_routed_bit_exact(cfg_name, T):
-    """Token-major quantisation (x read once per token) equals the per-slot oracle rule."""
+@pytest.mark.parametrize("shared_global", [False, True])
+def test_quant_act_routed_bit_exact(cfg_name, T, shared_global):
+    """Token-major quantisation (x read once per token) equals the per-slot oracle rule,
+    with a global per expert and with one global shared by all experts (the kernel then
+    reuses a group's codes across the token's slots)."""
     cfg = W.CONFIGS[cfg_name]
     x = W.layer_input_bf16(cfg, T)
     ids, _ = W.routing(cfg, T)
     ref = R.permute(ids.numpy(), cfg.E)
     rng = np.random.default_rng(T + 1)
     g_in = (np.float32(W.activation_global_scale_input(x)) * rng.uniform(0.5, 2.0, cfg.E)).astype(np.float32)
+    if shared_global:
+        g_in[:] = g_in[0]
     want_c, want_s = G.quant_act(x.float().numpy(), ref["slot_token"], ref["expert_offsets"], g_in)
     want_packed = (want_c[:, 0::2] | (want_c[:, 1::2] << 4)).astype(np.uint8)
     eo, po, st, ts, _ = gpu_permute(ids.numpy(), cfg.E)
