@@ -138,7 +138,11 @@ moesq_status moesq_quant_weight_workspace_size(int64_t E, int32_t n_seg, size_t*
 typedef enum moesq_linear_kind {
   MOESQ_LINEAR_DOWN = 0,          /* plain linear [out, K] */
   MOESQ_LINEAR_GATE_UP = 1,       /* fused [2I, K], gate rows first, one global (g_w[e]) */
-  MOESQ_LINEAR_GATE_UP_SPLIT = 2  /* fused [2I, K], globals g_w[2e] (gate), g_w[2e+1] (up): folded */
+  MOESQ_LINEAR_GATE_UP_SPLIT = 2, /* fused [2I, K], globals g_w[2e] (gate), g_w[2e+1] (up): the
+                                     up/gate ratio is folded into the up block scales (lossy by at
+                                     most half an E4M3 step, the pages' load-time fold) */
+  MOESQ_LINEAR_GATE_UP_EXACT = 3  /* fused [2I, K], globals g_w[2e] (gate), g_w[2e+1] (up): not
+                                     folded; the GEMM applies each global to its own half */
 } moesq_linear_kind;
 
 /* Bytes of the repacked metadata and block scales of ONE expert linear. */
@@ -146,13 +150,14 @@ moesq_status moesq_repack_sizes(int64_t out, int64_t K, size_t* meta_bytes, size
 
 /* Mask + block scales -> tcgen05 sparse metadata and scale-factor blocks.
  *   mask   device u8 [E, out, K/16];  scale device u8 [E, out, K/32];
- *   g_w    device f32 [E] (DOWN, GATE_UP) or [E, 2] (GATE_UP_SPLIT)
+ *   g_w    device f32 [E] (DOWN, GATE_UP) or [E, 2] (GATE_UP_SPLIT, GATE_UP_EXACT)
  *   meta   device u8 [E * meta_bytes]: per expert, per 128-row tile, per 256 dense
  *          K: 128 rows x 16 bytes, row r at 16r; each chunk's nibble = i0 | i1<<2
  *          (ascending kept byte positions), lower-K chunk in the low nibble
  *   sf     device u8 [E * sf_bytes]: per expert, per tile, per 128 dense K a 512-byte
  *          block, row r scale j at (r%32)*16 + (r/32)*4 + j
- *   alpha_w device f32 [E]: the weight global the GEMM applies (gate global for gate_up)
+ *   alpha_w device f32 [E]: the weight global the GEMM applies (gate global for gate_up);
+ *          [E, 2] (gate, up) for GATE_UP_EXACT
  * Tile row order: DOWN tile t holds rows 128t..128t+127, tile row 16g + 8p + j being
  * row 128t + 16g + 2j + p (g < 8; p < 2; j < 8); GATE_UP tile t holds the gate and up rows of outputs
  * 64t..64t+63: tile row r = 32q + 16h + 8s + j (q < 4; h, s < 2; j < 8) is source row
@@ -262,11 +267,12 @@ typedef struct moesq_linear {
   const uint8_t* packed; /* device u8 [E, out, K/4]  weight_sparse_packed, used as stored */
   const uint8_t* meta;   /* device, moesq_repack_meta output */
   const uint8_t* sf;     /* device, moesq_repack_meta output */
-  const float* alpha_w;  /* device f32 [E] */
+  const float* alpha_w;  /* device f32 [E]; [E, 2] (gate, up) for GATE_UP_EXACT */
   int64_t out;           /* output features (2I for gate_up) */
   int64_t K;             /* dense K */
   int32_t E;             /* experts */
-  int32_t kind;          /* moesq_linear_kind (GATE_UP_SPLIT behaves as GATE_UP here) */
+  int32_t kind;          /* moesq_linear_kind (GATE_UP_SPLIT behaves as GATE_UP here; GATE_UP_EXACT
+                            scales the up half by its own global) */
 } moesq_linear;
 
 typedef enum moesq_epilogue {

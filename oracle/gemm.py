@@ -93,6 +93,39 @@ def grouped_gemm_exact(W_int, g_w, A_int, g_act, expert_offsets):
     return y, bound
 
 
+def gate_up_exact(storage_per_expert, A_int, g_act, expert_offsets, fold=True):
+    """The fused gate_up GEMM over the routed activations, exact.
+
+    ``storage_per_expert``: list of storage dicts (packed, mask, scale, g) of the
+    fused [2I, K] weight, gate rows first.  With one global, or with two and
+    ``fold`` (the pages' load-time fold, "Compression details"/"Known limitations"
+    of the Qwen3.5-397B-A17B-P48NVFP4-MoESQ model card: the up/gate ratio of the
+    globals goes into the up block scales and the gate global serves both halves),
+    one pass with g[0].  With two globals and not ``fold``: the gate rows with g[0]
+    and the up rows with g[1], each with its own unfolded scales.
+    Returns (acc float64 [S, 2I], absbound float64 [S, 2I]).
+    """
+    from .storage import fold_up_scales
+
+    gs = [np.asarray(st["g"], dtype=np.float32).reshape(-1) for st in storage_per_expert]
+    split = any(g.size == 2 for g in gs)
+    if not split or fold:
+        W, gw = [], []
+        for st, g in zip(storage_per_expert, gs):
+            scale = np.array(st["scale"], dtype=np.uint8, copy=True)
+            if g.size == 2:
+                I = scale.shape[0] // 2
+                scale[I:] = fold_up_scales(scale[I:], g[0], g[1])
+            W.append(dequant_int(unpack_codes(decode(st["packed"], st["mask"])), scale))
+            gw.append(g[0])
+        return grouped_gemm_exact(W, gw, A_int, g_act, expert_offsets)
+    Wfull = [weight_int(st) for st in storage_per_expert]
+    I = Wfull[0].shape[0] // 2
+    yg, bg = grouped_gemm_exact([w[:I] for w in Wfull], [g[0] for g in gs], A_int, g_act, expert_offsets)
+    yu, bu = grouped_gemm_exact([w[I:] for w in Wfull], [g[1] for g in gs], A_int, g_act, expert_offsets)
+    return np.concatenate([yg, yu], axis=1), np.concatenate([bg, bu], axis=1)
+
+
 def silu(x):
     x = np.asarray(x, dtype=np.float64)
     return x / (1.0 + np.exp(-x))
@@ -119,33 +152,20 @@ def quant_act(x_bf16, slot_token, expert_offsets, g_in):
     return quantize_groups(x[st], g)
 
 
-def moe_forward(x_bf16, topk_ids, topk_w, gate_up, down, g_in_gu, g_in_down, E):
+def moe_forward(x_bf16, topk_ids, topk_w, gate_up, down, g_in_gu, g_in_down, E, fold=True):
     """The routed-expert MLP of one MoE layer, every step exact or float64.
 
     gate_up / down: lists over experts of storage dicts (packed, mask, scale, g);
-    the gate_up global is g[0] with the up scales folded as the load-time
-    repack does (see storage.repack_linear), or g[0] alone when there is one
-    global.  Returns dict with the intermediate results and ``out`` (float64,
+    gate_up as in gate_up_exact (folded, the default, or each half with its own
+    global).  Returns dict with the intermediate results and ``out`` (float64,
     before the final bf16 rounding) and ``out_bf16``.
     """
-    from .storage import fold_up_scales
-
     perm = permute(topk_ids, E)
     off = perm["expert_offsets"]
     a_codes, a_sf = quant_act(x_bf16, perm["slot_token"], off, g_in_gu)
     A = dequant_int(a_codes, a_sf)
 
-    Wg, gg = [], []
-    for st in gate_up:
-        g = np.asarray(st["g"], dtype=np.float32).reshape(-1)
-        scale = np.array(st["scale"], dtype=np.uint8, copy=True)
-        if g.size == 2:
-            I = scale.shape[0] // 2
-            scale[I:] = fold_up_scales(scale[I:], g[0], g[1])
-        dense = decode(st["packed"], st["mask"])
-        Wg.append(dequant_int(unpack_codes(dense), scale))
-        gg.append(g[0])
-    acc_gu, bound_gu = grouped_gemm_exact(Wg, gg, A, g_in_gu, off)
+    acc_gu, bound_gu = gate_up_exact(gate_up, A, g_in_gu, off, fold=fold)
     h = swiglu(acc_gu)
 
     e_of_slot = np.repeat(np.arange(E), np.diff(off))

@@ -271,25 +271,30 @@ def repack_weight_scales(scale, gate_up: bool) -> np.ndarray:
     return res.reshape(-1)
 
 
-def repack_linear(storage_per_expert, kind: str):
+def repack_linear(storage_per_expert, kind: str, fold: bool = True):
     """Load-time repack of one linear over all experts.
 
     ``storage_per_expert``: list of dicts (packed, mask, scale, g) per expert.
     kind: "gate_up" (fused, g has 1 or 2 entries) or "down".
     Returns dict(meta, sf, alpha) where alpha[e] is the FP32 weight global the
-    kernel applies (the gate global for gate_up).
+    kernel applies (the gate global for gate_up).  With two gate_up globals and
+    ``fold`` False, the up scales are left as stored and alpha holds both
+    globals per expert, [E, 2] flattened (gate, up).
     """
     gate_up = kind == "gate_up"
     metas, sfs, alpha = [], [], []
     for st in storage_per_expert:
         scale = np.array(st["scale"], dtype=np.uint8, copy=True)
         g = np.asarray(st["g"], dtype=np.float32).reshape(-1)
-        if gate_up and g.size == 2:
+        if gate_up and g.size == 2 and fold:
             I = scale.shape[0] // 2
             scale[I:] = fold_up_scales(scale[I:], g[0], g[1])
         metas.append(repack_meta(st["mask"], gate_up))
         sfs.append(repack_weight_scales(scale, gate_up))
-        alpha.append(g[0])
+        if gate_up and g.size == 2 and not fold:
+            alpha.extend([g[0], g[1]])
+        else:
+            alpha.append(g[0])
     return dict(meta=np.concatenate(metas), sf=np.concatenate(sfs),
                 alpha=np.array(alpha, dtype=np.float32))
 

@@ -13,7 +13,7 @@ from ._lib import (Linear, MoeLayer, MoesqError, declared_symbols, lib, moesq_de
                    padded_rows, permute_workspace_size, quant_weight_workspace_size, repack_sizes,
                    status_string)
 from .layer import (EPI_BF16, EPI_F32, EPI_SWIGLU_NVFP4, KIND_DOWN, KIND_GATE_UP,  # noqa: F401
-                    KIND_GATE_UP_SPLIT, SF_KERNEL, SF_LINEAR, ExpertLinear, MoELayer,
+                    KIND_GATE_UP_EXACT, KIND_GATE_UP_SPLIT, SF_KERNEL, SF_LINEAR, ExpertLinear, MoELayer,
                     quantize_expert_weights)
 
 __all__ = [n for n in dir() if not n.startswith("_")]

@@ -74,6 +74,7 @@ struct Params {
   uint8_t* out_sf;
   int32_t* d_status;
   int E, M, K, epi, gate_up;
+  int exact;  // gate_up with its own up global: alpha_w is [E, 2] (gate, up)
   int64_t S, P_cap;
 };
 
@@ -220,7 +221,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     const int o0 = off[e], o1 = off[e + 1];
     S.rec[e] = make_int4(0, o0, p.pad_offsets[e], o1 - o0);
-    S.ag[e] = make_float2(__fmul_rn(p.g_act[e], p.alpha_w[e]), p.g_next ? p.g_next[e] : 0.0f);
+    S.ag[e] = make_float2(__fmul_rn(p.g_act[e], p.alpha_w[p.exact ? 2 * e : e]), p.g_next ? p.g_next[e] : 0.0f);
   }
   __syncthreads();
   if (warp == 0) {  // end of expert e's token tiles = sum over e' <= e of ceil(T_e' / BN)
@@ -423,7 +424,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       const int mt = 2 * t.mt + (int)rank;  // this CTA's weight tile
       const bool own_tile = mt < MT;          // false: the duplicate of an odd last tile
       const float2 ag = S.ag[t.e];
-      const float alpha = ag.x;
+      const float alpha = ag.x;  // the accumulator's scale (gate rows of gate_up)
+      // up rows: the same, or their own global (read before the accumulator wait)
+      const float alpha_u = p.exact ? __fmul_rn(__ldg(p.g_act + t.e), __ldg(p.alpha_w + 2 * t.e + 1)) : alpha;
       mbar_wait_poll(&S.acc_full[buf], (acc_phase >> buf) & 1u, abort, p.d_status);
       tc_fence_after();
       const uint32_t tbase = tmem + TM_ACC + buf * BN + ((uint32_t)(32 * q) << 16);
@@ -437,7 +440,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         float hv[2][8];  // [h][v]: v = 2i + b
         if (live) {
           uint32_t r[16];
-          const float2 al2 = make_float2(alpha, alpha);
+          const float2 al2 = make_float2(alpha, alpha), au2 = make_float2(alpha_u, alpha_u);
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             tmem_ld_16x256b_x4(tbase + ((uint32_t)(16 * h) << 16) + c_lo, r);
@@ -445,7 +448,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {  // columns b = 0, 1 as one packed pair
               const float2 g = __fmul2_rn(make_float2(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1])), al2);
-              const float2 u = __fmul2_rn(make_float2(__uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3])), al2);
+              const float2 u = __fmul2_rn(make_float2(__uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3])), au2);
               const float2 hh = __fmul2_rn(silu2(g), u);
               hv[h][2 * i] = hh.x;
               hv[h][2 * i + 1] = hh.y;
@@ -563,7 +566,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             const float c0 = __uint_as_float(r1[4 * i + b]), c1 = __uint_as_float(r1[4 * i + 2 + b]);
             // down: (a0, a1) and (c0, c1) are output pairs; gate_up: (a0, c0) gate, (a1, c1) up
             const float2 w0v = __fmul2_rn(make_float2(a0, gu ? c0 : a1), make_float2(alpha, alpha));
-            const float2 w1v = __fmul2_rn(make_float2(gu ? a1 : c0, c1), make_float2(alpha, alpha));
+            const float2 w1v = __fmul2_rn(make_float2(gu ? a1 : c0, c1), make_float2(gu ? alpha_u : alpha, gu ? alpha_u : alpha));
             const __nv_bfloat162 p0 = __floats2bfloat162_rn(w0v.x, w0v.y);
             const __nv_bfloat162 p1 = __floats2bfloat162_rn(w1v.x, w1v.y);
             *reinterpret_cast<__nv_bfloat162*>(h0 + row * 128 + (((w0 >> 2) ^ (row & 7)) << 4) + ((w0 & 3) << 2)) = p0;
@@ -634,7 +637,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                   const int pos = 4 * u + z;
                   const int src = gu ? (((pos & 1) << 4) | ((pos >> 4) << 3) | ((pos & 15) >> 1))
                                      : ((pos & 16) | ((pos & 1) << 3) | ((pos & 15) >> 1));
-                  v[z] = __fmul_rn(row[src ^ lane], alpha);
+                  v[z] = __fmul_rn(row[src ^ lane], gu && pos >= 16 ? alpha_u : alpha);
                 }
                 if (gu) {
                   float* yg = (float*)p.out + s * p.M + (u >= 4 ? I : 0) + 64 * mt + 16 * q + 4 * (u & 3);
@@ -749,6 +752,7 @@ extern "C" moesq_status moesq_grouped_gemm(const moesq_linear* W, const uint8_t*
   MOESQ_REQUIRE(W->out * (int64_t)W->E < (1ll << 31) && W->K < (1 << 20), MOESQ_ERR_UNSUPPORTED_SHAPE);
   MOESQ_REQUIRE(P_cap >= moesq_padded_rows(S, W->E) && P_cap < (1ll << 31),
                 MOESQ_ERR_UNSUPPORTED_SHAPE);
+  MOESQ_REQUIRE(W->kind >= MOESQ_LINEAR_DOWN && W->kind <= MOESQ_LINEAR_GATE_UP_EXACT, MOESQ_ERR_INVALID_ARG);
   const bool gate_up = W->kind != MOESQ_LINEAR_DOWN;
   if (epilogue == MOESQ_EPI_SWIGLU_NVFP4) {
     MOESQ_REQUIRE(gate_up && g_next && out_sf, MOESQ_ERR_INVALID_ARG);
@@ -871,6 +875,7 @@ extern "C" moesq_status moesq_grouped_gemm(const moesq_linear* W, const uint8_t*
   prm.K = (int)W->K;
   prm.epi = epilogue;
   prm.gate_up = gate_up ? 1 : 0;
+  prm.exact = W->kind == MOESQ_LINEAR_GATE_UP_EXACT ? 1 : 0;
   prm.S = S;
   prm.P_cap = P_cap;
   cudaStream_t st = (cudaStream_t)stream;

@@ -326,11 +326,19 @@ __global__ void k_repack_sf(const uint8_t* __restrict__ scale, const float* __re
                             int64_t E, int64_t out, int64_t K, int32_t kind,
                             uint8_t* __restrict__ sf, float* __restrict__ alpha_w) {
   const bool gate_up = kind != MOESQ_LINEAR_DOWN;
-  const bool split = kind == MOESQ_LINEAR_GATE_UP_SPLIT;
+  const bool split = kind == MOESQ_LINEAR_GATE_UP_SPLIT;   // fold the up/gate ratio
+  const bool exact = kind == MOESQ_LINEAR_GATE_UP_EXACT;   // keep both globals
   const int64_t tiles = out / 128, nkb = K / 128, sbytes_row = K / 32;
   const int64_t n = E * tiles * nkb * 32;
   const int64_t tid0 = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-  if (tid0 < E) alpha_w[tid0] = split ? g_w[2 * tid0] : g_w[tid0];
+  if (tid0 < E) {
+    if (exact) {
+      alpha_w[2 * tid0] = g_w[2 * tid0];
+      alpha_w[2 * tid0 + 1] = g_w[2 * tid0 + 1];
+    } else {
+      alpha_w[tid0] = split ? g_w[2 * tid0] : g_w[tid0];
+    }
+  }
   for (int64_t i = tid0; i < n; i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t l = i % 32;
     const int64_t kb = (i / 32) % nkb;
@@ -440,7 +448,7 @@ extern "C" moesq_status moesq_repack_meta(const uint8_t* mask, const uint8_t* sc
                                           moesq_stream_t stream) {
   MOESQ_REQUIRE(mask && scale && g_w && meta && sf && alpha_w, MOESQ_ERR_INVALID_ARG);
   MOESQ_REQUIRE(E >= 0 && out >= 0 && K >= 0, MOESQ_ERR_INVALID_ARG);
-  MOESQ_REQUIRE(kind >= MOESQ_LINEAR_DOWN && kind <= MOESQ_LINEAR_GATE_UP_SPLIT,
+  MOESQ_REQUIRE(kind >= MOESQ_LINEAR_DOWN && kind <= MOESQ_LINEAR_GATE_UP_EXACT,
                 MOESQ_ERR_INVALID_ARG);
   MOESQ_REQUIRE(moesq_aligned16(mask) && moesq_aligned16(scale) && moesq_aligned16(meta) &&
                     moesq_aligned16(sf),

@@ -15,7 +15,7 @@ import torch
 
 from . import _lib as L
 
-KIND_DOWN, KIND_GATE_UP, KIND_GATE_UP_SPLIT = 0, 1, 2
+KIND_DOWN, KIND_GATE_UP, KIND_GATE_UP_SPLIT, KIND_GATE_UP_EXACT = 0, 1, 2, 3
 EPI_F32, EPI_BF16, EPI_SWIGLU_NVFP4 = 0, 1, 2
 SF_LINEAR, SF_KERNEL = 0, 1
 
@@ -56,7 +56,7 @@ class ExpertLinear:
         mb, sb = L.repack_sizes(out, K)
         meta = torch.empty(E * mb, dtype=torch.uint8, device=dev)
         sf = torch.empty(E * sb, dtype=torch.uint8, device=dev)
-        alpha = torch.empty(E, dtype=torch.float32, device=dev)
+        alpha = torch.empty(2 * E if kind == KIND_GATE_UP_EXACT else E, dtype=torch.float32, device=dev)
         L.moesq_repack_meta(st["mask"], st["scale"], st["g_w"].contiguous(), E, out, K, kind, meta, sf,
                             alpha, d_status, stream)
         return cls(st["packed"], meta, sf, alpha, E, out, K, kind)

@@ -15,7 +15,7 @@ from oracle import nvfp4 as N
 from oracle import routing as R
 from oracle import storage as S
 
-KIND_DOWN, KIND_GATE_UP, KIND_GATE_UP_SPLIT = 0, 1, 2
+KIND_DOWN, KIND_GATE_UP, KIND_GATE_UP_SPLIT, KIND_GATE_UP_EXACT = 0, 1, 2, 3
 
 
 def cuda(a, dtype=None):

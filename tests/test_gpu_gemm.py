@@ -35,14 +35,15 @@ def bf16_ulp(v):
 class Layer:
     """A small synthetic layer: oracle storage on the host, device copies repacked by the GPU."""
 
-    def __init__(self, cfg, T, g_down_scale=1.0, routing=None):
-        self.cfg, self.T = cfg, T
+    def __init__(self, cfg, T, g_down_scale=1.0, routing=None, exact=False):
+        """exact: gate_up with its own up global (kind GATE_UP_EXACT) instead of the fold."""
+        self.cfg, self.T, self.exact = cfg, T, exact
         n_seg = 2 if cfg.split_gate_up_global else 1
         wgu = W.all_expert_weights_bf16(cfg, "gate_up")
         wdn = W.all_expert_weights_bf16(cfg, "down")
         self.gu = [S.quantize_weight(wgu[e].float().numpy(), n_seg) for e in range(cfg.E)]
         self.dn = [S.quantize_weight(wdn[e].float().numpy(), 1) for e in range(cfg.E)]
-        kind_gu = M.KIND_GATE_UP_SPLIT if n_seg == 2 else M.KIND_GATE_UP
+        kind_gu = (M.KIND_GATE_UP_EXACT if exact else M.KIND_GATE_UP_SPLIT) if n_seg == 2 else M.KIND_GATE_UP
         self.dgu = M.ExpertLinear.from_storage(PU.storage_to_device(self.gu), kind_gu)
         self.ddn = M.ExpertLinear.from_storage(PU.storage_to_device(self.dn), M.KIND_DOWN)
         self.x = W.layer_input_bf16(cfg, T)
@@ -60,17 +61,8 @@ class Layer:
         a_c, a_s = G.quant_act(self.x.float().numpy(), self.perm["slot_token"], self.perm["expert_offsets"],
                                self.g_in_gu)
         self.A = G.dequant_int(a_c, a_s)
-        Wg, gg = [], []
-        for st in self.gu:
-            g = np.asarray(st["g"], np.float32).reshape(-1)
-            sc = st["scale"].copy()
-            if g.size == 2:
-                I = sc.shape[0] // 2
-                sc[I:] = S.fold_up_scales(sc[I:], g[0], g[1])
-            Wg.append(G.dequant_int(N.unpack_codes(S.decode(st["packed"], st["mask"])), sc))
-            gg.append(g[0])
-        self.acc_gu, self.bound_gu = G.grouped_gemm_exact(Wg, gg, self.A, self.g_in_gu,
-                                                          self.perm["expert_offsets"])
+        self.acc_gu, self.bound_gu = G.gate_up_exact(self.gu, self.A, self.g_in_gu, self.perm["expert_offsets"],
+                                                     fold=not exact)
         self.g_in_dn = (PU.calibrate_g_in_down(self.acc_gu, self.perm["expert_offsets"], cfg.E) *
                         np.float32(g_down_scale)).astype(np.float32)
 
@@ -101,13 +93,16 @@ CASES = {
     "mid_ktail": (W.LayerConfig("mid", 42, 16, 4, 384, 256, (300,), "uniform", True), 300),
     # full 512-deep stages (one metadata copy per stage, 3-D token boxes), plus tiles of <= 32 tokens
     "deep_k": (W.LayerConfig("deep", 44, 12, 2, 1024, 512, (150,), "zipf", True), 150),
+    # gate and up each scaled by its own global (no fold into the up block scales)
+    "exact_per_half_alpha": (W.LayerConfig("exact", 45, 8, 2, 512, 256, (200,), "uniform", True), 200,
+                             dict(exact=True)),
 }
 
 
 @pytest.fixture(scope="module", params=sorted(CASES))
 def layer(request):
-    cfg, T = CASES[request.param]
-    return Layer(cfg, T)
+    cfg, T, *opt = CASES[request.param]
+    return Layer(cfg, T, **(opt[0] if opt else {}))
 
 
 def test_gate_up_f32_within_tolerance(layer):
@@ -196,7 +191,7 @@ def test_swiglu_requant_epilogue(layer):
 def test_moe_forward_end_to_end(layer):
     L = layer
     cfg = L.cfg
-    ref = G.moe_forward(L.x.float().numpy(), L.ids, L.w, L.gu, L.dn, L.g_in_gu, L.g_in_dn, cfg.E)
+    ref = G.moe_forward(L.x.float().numpy(), L.ids, L.w, L.gu, L.dn, L.g_in_gu, L.g_in_dn, cfg.E, fold=not L.exact)
     moe = M.MoELayer(cfg.k, L.dgu, L.ddn, cuda(L.g_in_gu), cuda(L.g_in_dn))
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     out = moe.forward(L.x.cuda(), cuda(L.ids.astype(np.int32)), cuda(L.w), d_status=status)

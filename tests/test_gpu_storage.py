@@ -78,7 +78,7 @@ def test_quant_weight_bit_exact(cfg_name, which, n_seg, experts):
 
 
 @pytest.mark.parametrize("kind,out,K", [(0, 128, 256), (0, 256, 384), (1, 256, 256), (2, 512, 384),
-                                        (2, 1536, 2048)])
+                                        (2, 1536, 2048), (3, 512, 384)])
 def test_repack_bit_exact(kind, out, K):
     rng = np.random.default_rng(out + K + kind)
     E = 3
@@ -86,14 +86,15 @@ def test_repack_bit_exact(kind, out, K):
     for e in range(E):
         wv = (rng.standard_normal((out, K)) * 0.02).astype(np.float32)
         sts.append(S.quantize_weight(S.f32(torch.from_numpy(wv).to(torch.bfloat16).float().numpy()),
-                                     2 if kind == 2 else 1))
-    ref = S.repack_linear(sts, "down" if kind == 0 else "gate_up")
+                                     2 if kind >= 2 else 1))
+    # kind 3: both gate_up globals kept (alpha [E, 2]), up scales not folded
+    ref = S.repack_linear(sts, "down" if kind == 0 else "gate_up", fold=kind != 3)
     dev = dict(mask=cuda(np.stack([s["mask"] for s in sts])), scale=cuda(np.stack([s["scale"] for s in sts])),
                g_w=cuda(np.stack([s["g"] for s in sts])))
     mb, sb = M.repack_sizes(out, K)
     meta = torch.empty(E * mb, dtype=torch.uint8, device="cuda")
     sf = torch.empty(E * sb, dtype=torch.uint8, device="cuda")
-    alpha = torch.empty(E, dtype=torch.float32, device="cuda")
+    alpha = torch.empty(2 * E if kind == 3 else E, dtype=torch.float32, device="cuda")
     st = _status()
     M.moesq_repack_meta(dev["mask"], dev["scale"], dev["g_w"], E, out, K, kind, meta, sf, alpha, st)
     assert np.array_equal(meta.cpu().numpy(), ref["meta"])

@@ -149,3 +149,51 @@ def test_moe_forward_composition_tiny_exact():
     ts = perm["token_slot"]
     want = sum(w.numpy()[:, j:j + 1].astype(np.float64) * res["y"][ts[:, j]] for j in range(cfg.k))
     assert np.allclose(res["out"], want, rtol=1e-15, atol=0)
+
+
+def _split_storage(seed=7, I=64, K=256):
+    w = torch.randn((2 * I, K), generator=torch.Generator().manual_seed(seed)) * 0.02
+    return S.quantize_weight(w.to(torch.bfloat16).float().numpy(), 2)
+
+
+def _routed_acts(seed=8, T=24, K=256, E=1):
+    x = torch.randn((T, K), generator=torch.Generator().manual_seed(seed)).to(torch.bfloat16)
+    off = np.array([0, T], np.int64)
+    g_in = np.array([np.float32(x.float().abs().max()) / np.float32(2688)], np.float32)
+    c, s = G.quant_act(x.float().numpy(), np.arange(T), off, g_in)
+    return G.dequant_int(c, s), g_in, off
+
+
+def test_unfolded_gate_up_equals_float64_matmul_of_decoded_halves():
+    """Each half with its own global ("exact per-half alpha"): the exact int64 path
+    against a float64 matmul of the decoded values times scales times globals."""
+    st = _split_storage()
+    A, g_in, off = _routed_acts()
+    acc, _ = G.gate_up_exact([st], A, g_in, off, fold=False)
+    codes = N.unpack_codes(S.decode(st["packed"], st["mask"]))
+    Wd = F.e2m1_decode(codes) * np.repeat(F.e4m3_decode(st["scale"]), 32, axis=1)
+    g = np.asarray(st["g"], np.float64)
+    I = Wd.shape[0] // 2
+    Wd[:I] *= g[0]
+    Wd[I:] *= g[1]
+    ref = (torch.from_numpy(A.astype(np.float64) * 2.0 ** -10) @ torch.from_numpy(Wd).T).numpy() * np.float64(g_in[0])
+    assert np.allclose(acc, ref, rtol=1e-12, atol=1e-300)
+
+
+def test_fold_is_exact_for_a_power_of_two_ratio():
+    """With g_up = g_gate / 2 and every up scale representable at half its value, the
+    pages' fold loses nothing: the folded and the per-half paths agree exactly."""
+    st = dict(_split_storage())
+    g0 = np.float32(st["g"][0])
+    st["g"] = np.array([g0, g0 * np.float32(0.5)], np.float32)
+    sc = np.array(st["scale"], np.uint8, copy=True)
+    I = sc.shape[0] // 2
+    vals = F.e4m3_decode(sc[I:])
+    ok = (vals >= 2.0 ** -5) & (vals <= 448)          # halving stays a normal E4M3 value
+    sc[I:] = np.where(ok, sc[I:], np.uint8(0x38))      # elsewhere 1.0
+    st["scale"] = sc
+    assert (F.e4m3_decode(S.fold_up_scales(sc[I:], st["g"][0], st["g"][1])) == F.e4m3_decode(sc[I:]) / 2).all()
+    A, g_in, off = _routed_acts(seed=9)
+    a, _ = G.gate_up_exact([st], A, g_in, off, fold=True)
+    b, _ = G.gate_up_exact([st], A, g_in, off, fold=False)
+    assert np.array_equal(a, b)
