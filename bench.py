@@ -295,6 +295,79 @@ class Bench:
         per = {s: [evs[i][j][0].elapsed_time(evs[i][j][1]) for i in range(steps)] for j, s in enumerate(self.STAGES)}
         return step_ms, per
 
+    def dense_comparison(self, steps, flush):
+        """The same two GEMMs with the dense comparison kernel on the decoded weights (the
+        pages' --no-sparse-storage form): the seeded weights are exported again (the same
+        bytes as the sparse layer's), decoded, and the scale blocks expanded to 16
+        elements.  Timed like the stages of run(); the 16-element expansion of the
+        activation scales is outside the timed GEMMs."""
+        torch, M, W, cfg = self.torch, self.M, self.W, self.cfg
+        dev = self.dev
+
+        def expand(sf):
+            o = torch.empty(sf.numel() * 2, dtype=torch.uint8, device=dev)
+            M.moesq_sf_expand_block16(sf, o, sf.numel() // 512)
+            return o
+
+        dense = {}
+        for which, ns in (("gate_up", 2 if cfg.split_gate_up_global else 1), ("down", 1)):
+            lin = self.lin[which]
+            w = W.all_expert_weights_bf16(cfg, which, device=dev)
+            st = M.quantize_expert_weights(w, ns)
+            del w
+            codes = torch.empty((lin.E, lin.out, lin.K // 2), dtype=torch.uint8, device=dev)
+            M.moesq_decode(st["packed"], st["mask"], codes, lin.E * lin.out, lin.K, self.status)
+            assert torch.equal(st["packed"], lin.packed), "re-export differs from the sparse layer's weights"
+            del st
+            sf16 = expand(lin.sf)
+            dense[which] = (codes, sf16, M.Linear(codes.data_ptr(), 0, sf16.data_ptr(), lin.alpha_w.data_ptr(),
+                                                  lin.out, lin.K, lin.E, lin.kind))
+        torch.cuda.empty_cache()
+        self.permute()
+        self.quant_act()
+        a_sf16 = expand(self.a_sf)
+        h_codes = torch.empty_like(self.h_codes)
+        h_sf = torch.empty_like(self.h_sf)
+        y = torch.empty_like(self.y)
+        h_sf16 = torch.empty(h_sf.numel() * 2, dtype=torch.uint8, device=dev)
+
+        def gate_up():
+            M.moesq_grouped_gemm_dense(dense["gate_up"][2], self.a_codes, a_sf16, self.g_in_gu, self.eo, self.po,
+                                       self.S, self.P, M.EPI_SWIGLU_NVFP4, self.g_in_dn, h_codes, h_sf,
+                                       d_status=self.status)
+
+        def down():
+            M.moesq_grouped_gemm_dense(dense["down"][2], h_codes, h_sf16, self.g_in_dn, self.eo, self.po, self.S,
+                                       self.P, M.EPI_BF16, None, y.view(torch.uint16), None, d_status=self.status)
+
+        gate_up()
+        M.moesq_sf_expand_block16(h_sf, h_sf16, h_sf.numel() // 512)
+        down()
+        torch.cuda.synchronize()
+        graphs = {}
+        for name, fn in (("gate_up", gate_up), ("down", down)):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fn()
+            graphs[name] = g
+        stream = torch.cuda.current_stream()
+        res = {}
+        for name, g in graphs.items():
+            for _ in range(3):
+                g.replay()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+            for a, b in ev:
+                if flush is not None:
+                    flush.zero_()
+                torch.cuda._sleep(1_000_000)
+                a.record(stream)
+                g.replay()
+                b.record(stream)
+            torch.cuda.synchronize()
+            res[name] = sum(a.elapsed_time(b) for a, b in ev) / steps
+        del graphs
+        return res
+
     def check_against_forward(self):
         """The staged step and the single moesq_moe_forward call give identical bytes."""
         torch = self.torch
@@ -512,6 +585,20 @@ def run_ours(args, rank, world, local_rank):
             del bb
             torch.cuda.empty_cache()
         out["sweep"] = sweep
+    if not args.no_sweep and world == 1:
+        d = b.dense_comparison(10, flush)
+        fl_d = step_flops(b.S, H, I)
+        by_w = {"gate_up": b.n_touched * 2 * I * H, "down": b.n_touched * H * I}
+        out["dense_comparison"] = {
+            "what": "the same gate_up (SwiGLU + requant) and down (bf16) GEMMs on the decoded dense NVFP4 "
+                    "weights (dense tcgen05 MMA, 16-element scale blocks), same workload and inputs",
+            **{f"{k}_ms": d[k] for k in d},
+            **{f"{k}_TFLOPs": fl_d[k] / (d[k] * 1e-3) / 1e12 for k in d},
+            "sparse_speedup": {k: d[k] / avg["gemm_" + k] for k in d},
+            "weight_bytes_per_dense_element": {"sparse": 0.34375, "dense": 0.53125},
+            "weight_bytes_touched_GB": {k: {"sparse": by_w[k] * 0.34375 / 1e9, "dense": by_w[k] * 0.53125 / 1e9}
+                                        for k in by_w},
+        }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = {k: v for k, v in cpu_baseline(cfg, args.tokens, args.cpu_slots).items()
                                if k != "seconds"}

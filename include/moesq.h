@@ -303,6 +303,30 @@ moesq_status moesq_grouped_gemm(const moesq_linear* W, const uint8_t* act_codes,
                                 int32_t* d_status, moesq_stream_t stream);
 moesq_status moesq_grouped_gemm_workspace_size(const moesq_linear* W, int64_t S, size_t* bytes);
 
+/* Dense comparison GEMM: the same grouped GEMM, epilogues and argument meanings on
+ * dense NVFP4 weights, the pages' alternative storage ("--no-sparse-storage writes
+ * dense packed NVFP4 with the pruned elements zeroed", Usage of the MoESQ repository
+ * README), with the dense tensor-core MMA (kind::mxf4nvf4, 64 dense K per MMA).
+ *   W->packed  device u8 [E, out, K/2] dense codes (moesq_decode of the sparse storage),
+ *              same tile row order as the sparse operand; W->meta is not used
+ *   W->sf, act_sf  scale blocks of 16 elements (moesq_sf_expand_block16 of the 32-element
+ *              blocks: [rows/128][K/64][512])
+ * The result equals the sparse GEMM's (same decoded weights and scales) up to the
+ * FP32 accumulation order.  Returns as moesq_grouped_gemm. */
+moesq_status moesq_grouped_gemm_dense(const moesq_linear* W, const uint8_t* act_codes,
+                                      const uint8_t* act_sf, const float* g_act,
+                                      const int32_t* expert_offsets, const int32_t* pad_offsets,
+                                      int64_t S, int64_t P_cap, int32_t epilogue, const float* g_next,
+                                      void* out, uint8_t* out_sf, int32_t* d_status,
+                                      moesq_stream_t stream);
+
+/* 32-element scale blocks -> 16-element scale blocks for the dense MMA: each 512-byte
+ * block b (128 rows x 4 scales, one per 32 K: row r, scale j at (r%32)*16 + (r/32)*4 + j)
+ * becomes blocks 2b and 2b+1 (one scale per 16 K, each 32-element scale written twice).
+ *   sf32 device u8 [nblocks * 512];  sf16 device u8 [2 * nblocks * 512]; 16-byte aligned. */
+moesq_status moesq_sf_expand_block16(const uint8_t* sf32, uint8_t* sf16, int64_t nblocks,
+                                     moesq_stream_t stream);
+
 /* ------------------------------------------------------------------------- *
  * The whole routed-expert MLP of one MoE layer
  * ------------------------------------------------------------------------- */

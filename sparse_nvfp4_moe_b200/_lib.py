@@ -59,6 +59,9 @@ _SIGS = {
                                               c_vp, c_vp, c_vp, c_vp]),
     "moesq_grouped_gemm": (ctypes.c_int, [ctypes.POINTER(Linear), c_vp, c_vp, c_vp, c_vp, c_vp, c_i64,
                                           c_i64, c_i32, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp, c_vp]),
+    "moesq_grouped_gemm_dense": (ctypes.c_int, [ctypes.POINTER(Linear), c_vp, c_vp, c_vp, c_vp, c_vp, c_i64,
+                                                c_i64, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp]),
+    "moesq_sf_expand_block16": (ctypes.c_int, [c_vp, c_vp, c_i64, c_vp]),
     "moesq_grouped_gemm_workspace_size": (ctypes.c_int, [ctypes.POINTER(Linear), c_i64,
                                                          ctypes.POINTER(c_sz)]),
     "moesq_moe_forward": (ctypes.c_int, [ctypes.POINTER(MoeLayer), c_vp, c_vp, c_vp, c_i64, c_vp, c_vp,
@@ -220,6 +223,17 @@ def moesq_grouped_gemm(W: Linear, act_codes, act_sf, g_act, expert_offsets, pad_
         ctypes.byref(W), _p(act_codes), _p(act_sf), _p(g_act), _p(expert_offsets), _p(pad_offsets), S,
         P_cap, epilogue, _p(g_next), _p(out), _p(out_sf), _p(ws), ws_bytes, _p(d_status),
         _stream(stream)))
+
+
+def moesq_grouped_gemm_dense(W: Linear, act_codes, act_sf, g_act, expert_offsets, pad_offsets, S, P_cap,
+                             epilogue, g_next, out, out_sf, d_status=None, stream=None):
+    _check("moesq_grouped_gemm_dense", lib().moesq_grouped_gemm_dense(
+        ctypes.byref(W), _p(act_codes), _p(act_sf), _p(g_act), _p(expert_offsets), _p(pad_offsets), S,
+        P_cap, epilogue, _p(g_next), _p(out), _p(out_sf), _p(d_status), _stream(stream)))
+
+
+def moesq_sf_expand_block16(sf32, sf16, nblocks, stream=None):
+    _check("moesq_sf_expand_block16", lib().moesq_sf_expand_block16(_p(sf32), _p(sf16), nblocks, _stream(stream)))
 
 
 def moesq_moe_forward(layer: MoeLayer, x, topk_ids, topk_w, T, out, ws, ws_bytes, d_status=None,

@@ -516,6 +516,18 @@ __device__ __forceinline__ void tc_mma_pair_sp_nvf4(uint32_t d_tmem, uint64_t a_
       "r"(e_tmem)
       : "memory");
 }
+// dense block-scaled NVFP4 MMA on a CTA pair (M = 256, dense K = 64, one UE4M3 scale
+// per 16 elements of K per operand)
+__device__ __forceinline__ void tc_mma_pair_nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16"
+      " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
 // arrive once on `bar` (same offset) in every CTA of `cta_mask` when all tcgen05
 // work issued so far by this thread is complete
 __device__ __forceinline__ void tc_commit_pair_mc(uint64_t* bar, uint16_t cta_mask) {

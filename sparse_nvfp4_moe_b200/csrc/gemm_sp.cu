@@ -38,18 +38,33 @@ namespace sp {
 
 constexpr int BM = 128;           // weight rows per tile
 constexpr int BN = 128;           // max tokens per tile
-// A pipeline stage covers 512 dense K: four MMAs.  Every copy instruction costs
-// the single issuing thread about the same whatever its size, so a stage is
-// moved by few, large copies: one for the weight tile, two for the token tile,
-// one each for metadata and the two scale blocks.
-constexpr int BK = 512;
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK / 4;       // compressed values: 128 B per row (SW128)
 constexpr int B_CHUNK = (BN / 2) * 128;    // this CTA's half of the tokens, 256 dense K: 128 B per row (SW128)
-constexpr int B_BYTES = 2 * B_CHUNK;
-constexpr int E_BYTES = 2 * BM * 16;       // metadata: 16 B per row per 256 dense K
-constexpr int SF_BYTES = 4 * 512;          // one 512-byte scale block per 128 dense K
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES + E_BYTES + 2 * SF_BYTES;  // 40960
+constexpr int SF_BYTES = 4 * 512;          // one 512-byte scale block per MMA and operand, four MMAs a stage
+constexpr int MAX_STAGES = 5;
+// Stage geometry.  Every copy instruction costs the single issuing thread about the
+// same whatever its size, so a stage is moved by few, large copies: one for the
+// weight tile, one or two for the token tile, one each for metadata and the two
+// scale blocks.
+//   sparse: 512 dense K a stage, four sparse MMAs of 128 dense K (one scale per 32)
+//   dense (the comparison kernel on decoded weights): 256 dense K a stage, four
+//   dense MMAs of 64 dense K (one scale per 16, the 32-group scales duplicated)
+template <bool DENSE> struct Geo;
+template <> struct Geo<false> {
+  static constexpr int BK = 512, KMMA = 128, STAGES = 4;
+  static constexpr int A_BYTES = BM * BK / 4;  // compressed values: 128 B per row (SW128)
+  static constexpr int B_BYTES = 2 * B_CHUNK;  // two 256-deep token chunks
+  static constexpr int E_BYTES = 2 * BM * 16;  // metadata: 16 B per row per 256 dense K
+};
+template <> struct Geo<true> {
+  static constexpr int BK = 256, KMMA = 64, STAGES = 5;
+  static constexpr int A_BYTES = BM * BK / 2;  // dense codes: 128 B per row (SW128)
+  static constexpr int B_BYTES = B_CHUNK;      // one 256-deep token chunk
+  static constexpr int E_BYTES = 0;
+};
+template <bool DENSE>
+__host__ __device__ constexpr int stage_bytes() {
+  return Geo<DENSE>::A_BYTES + Geo<DENSE>::B_BYTES + Geo<DENSE>::E_BYTES + 2 * SF_BYTES;  // 40960 / 28672
+}
 constexpr int EPI_BYTES = 32768;  // epilogue exchange / transpose / staging space
 constexpr int MAX_E = 1024;
 // Sixteen epilogue warps, four per sub-partition: the epilogue is latency-bound
@@ -84,7 +99,7 @@ struct Smem {
   alignas(128) uint8_t hstg[2][4][32][32];
   alignas(16) uint8_t sstg[2][4][32][2];
   // full[s]: stage s landed.  empty[s]: stage s consumed by the tensor core.
-  uint64_t full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], done;
+  uint64_t full[MAX_STAGES], empty[MAX_STAGES], acc_full[2], acc_empty[2], done;
   uint32_t tmem_base;
   int abort;
   // per-expert tables, read from global memory once at set-up so that no role
@@ -96,11 +111,16 @@ struct Smem {
   float2 ag[MAX_E];  // {g_act[e] * alpha_w[e] (the accumulator's scale), global scale of the requantised output}
 };
 
-constexpr size_t SMEM_BYTES = 1024 /*align*/ + (size_t)STAGES * STAGE_BYTES + EPI_BYTES + sizeof(Smem);
-static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+template <bool DENSE>
+constexpr size_t smem_bytes() {
+  return 1024 /*align*/ + (size_t)Geo<DENSE>::STAGES * stage_bytes<DENSE>() + EPI_BYTES + sizeof(Smem);
+}
+static_assert(smem_bytes<false>() <= 227 * 1024 && smem_bytes<true>() <= 227 * 1024, "shared memory budget");
+static_assert(Geo<false>::STAGES <= MAX_STAGES && Geo<true>::STAGES <= MAX_STAGES, "barrier arrays");
 
+template <bool DENSE>
 __device__ __forceinline__ uint32_t make_idesc(uint32_t n) {
-  return (1u << 2)            // sparse
+  return (DENSE ? 0u : 1u << 2)  // sparse
          | (1u << 7)          // A: E2M1
          | (1u << 10)         // B: E2M1
          | ((n >> 3) << 17)   // N
@@ -167,13 +187,16 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-template <int EPI>
+template <int EPI, bool DENSE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     k_grouped_gemm_sp(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                       const __grid_constant__ CUtensorMap tmap_b16, const __grid_constant__ CUtensorMap tmap_e,
                       const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
                       const __grid_constant__ CUtensorMap tmap_y, const __grid_constant__ CUtensorMap tmap_b_3d,
                       const Params p) {
+  using G = Geo<DENSE>;
+  constexpr int STAGES = G::STAGES, STAGE_BYTES = stage_bytes<DENSE>();
+  constexpr int A_BYTES = G::A_BYTES, B_BYTES = G::B_BYTES, E_BYTES = G::E_BYTES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   float* epi = (float*)(smem + STAGES * STAGE_BYTES);
@@ -183,7 +206,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const uint32_t rank = cluster_ctarank();  // 0: issues the pair's MMAs
   const bool lead = rank == 0;
   const int E = p.E, MT = p.M / BM, MT2 = (MT + 1) / 2;
-  const int nkb = (p.K + BK - 1) / BK, kb128 = p.K / 128, nkb256 = (p.K + 255) / 256;
+  // K stages, MMAs over K (= scale blocks per 128 rows), 256-deep metadata chunks
+  const int nkb = (p.K + G::BK - 1) / G::BK, kb128 = p.K / G::KMMA, nkb256 = (p.K + 255) / 256;
   const int32_t* off = p.expert_offsets;
   const int pair_id = blockIdx.x >> 1, npairs = gridDim.x >> 1;
 
@@ -260,7 +284,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       uint32_t full_lead[STAGES];
 #pragma unroll
       for (int i = 0; i < STAGES; ++i) full_lead[i] = cluster_map(&S.full[i], 0);
-      const bool b3d = (p.K % 256) == 0;  // both 256-deep token chunks of a stage in one 3-D box
+      const bool b3d = !DENSE && (p.K % 256) == 0;  // both 256-deep token chunks of a stage in one 3-D box
       for (int id = pair_id; id < total; id += npairs, walk.advance(MT2)) {
         const Tile t = decode_tile(S, walk, E);
         const int mt = min(2 * t.mt + (int)rank, MT - 1);  // an odd last tile is loaded twice
@@ -280,7 +304,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         for (int kb = 0; kb < nkb; ++kb) {
           mbar_wait_spin(&S.empty[stage], phase ^ 1, abort, p.d_status);
           const int nk = min(4, kb128 - 4 * kb);  // 128-deep MMAs in this stage
-          const int nc = (nk + 1) >> 1;           // 256-deep chunks in this stage
+          const int nc = DENSE ? 1 : (nk + 1) >> 1;  // 256-deep token chunks in this stage
           uint8_t* st = smem + stage * STAGE_BYTES;
           uint32_t bar = full_lead[0];
 #pragma unroll
@@ -295,12 +319,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           if (b3d && nc > 1 && !small) {  // 64-row chunks: chunk 1 lands at B_CHUNK as the MMA expects
             tma_load_3d_pair(st + A_BYTES, tb3, 0, brow, 2 * kb, bar);
           } else {
-            tma_load_2d_pair(st + A_BYTES, tb, kb * 256, brow, bar);
+            tma_load_2d_pair(st + A_BYTES, tb, kb * (G::BK / 2), brow, bar);
             if (nc > 1) tma_load_2d_pair(st + A_BYTES + B_CHUNK, tb, kb * 256 + 128, brow, bar);
           }
           // metadata (2 KB per 256 dense K) and scale blocks (512 B per 128 dense K)
           // as 256-byte rows; a stage always moves 4 KB + 2 KB + 2 KB
-          tma_load_2d_pair(st + A_BYTES + B_BYTES, &tmap_e, 0, (wt * nkb256 + 2 * kb) * 8, bar);
+          if constexpr (!DENSE) tma_load_2d_pair(st + A_BYTES + B_BYTES, &tmap_e, 0, (wt * nkb256 + 2 * kb) * 8, bar);
           tma_load_2d_pair(st + A_BYTES + B_BYTES + E_BYTES, &tmap_sfa, 0, (wt * kb128 + 4 * kb) * 2, bar);
           tma_load_2d_pair(st + A_BYTES + B_BYTES + E_BYTES + SF_BYTES, &tmap_sfb, 0,
                            ((prow / 128) * kb128 + 4 * kb) * 2, bar);
@@ -345,7 +369,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       for (int id = pair_id; id < total; id += npairs, walk.advance(MT2)) {
         const Tile t = decode_tile(S, walk, E);
         const int n_mma = max(16, (t.n_rows + 15) / 16 * 16);
-        const uint32_t idesc = make_idesc((uint32_t)n_mma);
+        const uint32_t idesc = make_idesc<DENSE>((uint32_t)n_mma);
         const uint32_t d_tmem = tmem + TM_ACC + buf * BN;
         mbar_wait_spin(&S.acc_empty[buf], ((acc_phase >> buf) & 1u) ^ 1u, abort, p.d_status);
         tc_fence_after();
@@ -354,7 +378,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           tc_fence_after();
           const uint64_t so = (uint64_t)((stage * STAGE_BYTES) >> 4);
           const int nk = min(4, kb128 - 4 * kb);
-          if (nk == 4) {
+          if constexpr (DENSE) {
+            // dense MMAs of 64 dense K: A and B each advance 32 B inside their
+            // 128-byte swizzle rows; one scale block per MMA and operand
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              if (j < nk) {
+                tc_cp_pair_32x128b_warpx4(tSFA + 4 * j, dSFA0 + so + (uint64_t)(j * (512 >> 4)));
+                tc_cp_pair_32x128b_warpx4(tSFB + 4 * j, dSFB0 + so + (uint64_t)(j * (512 >> 4)));
+                tc_mma_pair_nvf4(d_tmem, dA0 + so + (uint64_t)(j * 2), dB0 + so + (uint64_t)(j * 2), idesc,
+                                 tSFA + 4 * j, tSFB + 4 * j, (kb > 0 || j > 0) ? 1u : 0u);
+              }
+            }
+          } else if (nk == 4) {
             // metadata of both 256-deep chunks (2 KB apart) in one copy; MMA j
             // reads columns tE + 2j
             tc_cp_pair_128x256b(tE, dE2 + so);
@@ -730,17 +766,18 @@ extern "C" moesq_status moesq_grouped_gemm_workspace_size(const moesq_linear* W,
   return MOESQ_OK;
 }
 
-extern "C" moesq_status moesq_grouped_gemm(const moesq_linear* W, const uint8_t* act_codes,
-                                           const uint8_t* act_sf, const float* g_act,
-                                           const int32_t* expert_offsets,
-                                           const int32_t* pad_offsets, int64_t S, int64_t P_cap,
-                                           int32_t epilogue, const float* g_next, void* out,
-                                           uint8_t* out_sf, void* ws, size_t ws_bytes,
-                                           int32_t* d_status, moesq_stream_t stream) {
-  (void)ws;
-  (void)ws_bytes;
+// Both grouped GEMMs: DENSE = false is the paired-4:8 sparse kernel (W->packed are
+// the kept bytes, W->meta the sparse metadata); DENSE = true is the comparison
+// kernel on decoded weights (W->packed dense codes [E, out, K/2], no metadata, W->sf
+// and act_sf in the 16-element scale layout of moesq_sf_expand_block16).
+template <bool DENSE>
+static moesq_status grouped_gemm_impl(const moesq_linear* W, const uint8_t* act_codes, const uint8_t* act_sf,
+                                      const float* g_act, const int32_t* expert_offsets,
+                                      const int32_t* pad_offsets, int64_t S, int64_t P_cap, int32_t epilogue,
+                                      const float* g_next, void* out, uint8_t* out_sf, int32_t* d_status,
+                                      moesq_stream_t stream) {
   MOESQ_REQUIRE(W, MOESQ_ERR_INVALID_ARG);
-  MOESQ_REQUIRE(W->packed && W->meta && W->sf && W->alpha_w, MOESQ_ERR_INVALID_ARG);
+  MOESQ_REQUIRE(W->packed && (DENSE || W->meta) && W->sf && W->alpha_w, MOESQ_ERR_INVALID_ARG);
   MOESQ_REQUIRE(act_codes && act_sf && g_act && expert_offsets && pad_offsets && out,
                 MOESQ_ERR_INVALID_ARG);
   MOESQ_REQUIRE(epilogue >= MOESQ_EPI_F32 && epilogue <= MOESQ_EPI_SWIGLU_NVFP4,
@@ -759,7 +796,7 @@ extern "C" moesq_status moesq_grouped_gemm(const moesq_linear* W, const uint8_t*
     MOESQ_REQUIRE(W->out % 256 == 0, MOESQ_ERR_UNSUPPORTED_SHAPE);
   }
   if (gate_up) MOESQ_REQUIRE(W->out % 256 == 0, MOESQ_ERR_UNSUPPORTED_SHAPE);
-  MOESQ_REQUIRE(moesq_aligned16(W->packed) && moesq_aligned16(W->meta) && moesq_aligned16(W->sf) &&
+  MOESQ_REQUIRE(moesq_aligned16(W->packed) && (DENSE || moesq_aligned16(W->meta)) && moesq_aligned16(W->sf) &&
                     moesq_aligned16(act_codes) && moesq_aligned16(act_sf) && moesq_aligned16(out) &&
                     moesq_aligned16(out_sf),
                 MOESQ_ERR_INVALID_ARG);
@@ -769,15 +806,17 @@ extern "C" moesq_status moesq_grouped_gemm(const moesq_linear* W, const uint8_t*
   if (sms < 0) return MOESQ_ERR_CUDA;
   if (sms == 0) return MOESQ_ERR_DEVICE;
 
-  // Weight tile: 512 dense K = 128 compressed bytes per row.  A gate_up tile holds
+  // Weight tile: 128 bytes per row a stage (512 dense K of kept bytes, or 256 dense
+  // K of dense codes).  A gate_up tile holds
   // the gate and up rows of 64 outputs in the interleaved order of the weight repack
   // (tile row 32q + 16h + 8s + j = row s*I + 16q + 2j + h of the tile's outputs):
   // a 5-D view (byte, j [stride 2 rows], s [stride I rows], h [stride 1 row],
   // 16-row group [stride 16 rows, expert folded in]) loads it with one copy.  Only
   // coordinates of whole tiles are used, so every byte read lies in the weights.
   CUtensorMap ta, tb, tb16, te, tsfa, tsfb;
-  const uint64_t rowA = (uint64_t)(W->K / 4);
-  const int64_t MT = W->out / 128, kb128 = W->K / 128, nkb256 = (W->K + 255) / 256;
+  const uint64_t rowA = (uint64_t)(DENSE ? W->K / 2 : W->K / 4);
+  // MMAs over K = scale blocks per 128 rows; 256-deep metadata chunks
+  const int64_t MT = W->out / 128, kb128 = W->K / sp::Geo<DENSE>::KMMA, nkb256 = (W->K + 255) / 256;
   if (gate_up) {
     const uint64_t I = (uint64_t)(W->out / 2);
     const cuuint64_t dims[5] = {rowA, 8, 2, 2, (uint64_t)(W->E * W->out / 16)};
@@ -802,15 +841,16 @@ extern "C" moesq_status moesq_grouped_gemm(const moesq_linear* W, const uint8_t*
   // the same token codes as (128-byte chunk row, row, 256-deep chunk): both 64-row chunks
   // of a 512-deep stage in one box; valid when K % 256 == 0 (else the 2-D boxes are used)
   CUtensorMap tb3 = tb;
-  if (W->K % 256 == 0) {
+  if (!DENSE && W->K % 256 == 0) {
     const cuuint64_t dims[3] = {128, (uint64_t)P_cap, (uint64_t)(W->K / 256)};
     const cuuint64_t strides[2] = {(uint64_t)(W->K / 2), 128};
     const cuuint32_t box64[3] = {128, 64, 2};
     if (!make_tmap_u8(&tb3, act_codes, 3, dims, strides, box64, CU_TENSOR_MAP_SWIZZLE_128B)) return MOESQ_ERR_CUDA;
   }
   // metadata and scale blocks seen as 256-byte rows (no swizzle: contiguous copies)
-  if (!make_tmap_rows(&te, W->meta, 256, (uint64_t)(W->E * MT * nkb256 * 8), 256, 16,
-                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
+  te = ta;  // unused by the dense kernel
+  if ((!DENSE && !make_tmap_rows(&te, W->meta, 256, (uint64_t)(W->E * MT * nkb256 * 8), 256, 16,
+                                 CU_TENSOR_MAP_SWIZZLE_NONE)) ||
       !make_tmap_rows(&tsfa, W->sf, 256, (uint64_t)(W->E * MT * kb128 * 2), 256, 8, CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !make_tmap_rows(&tsfb, act_sf, 256, (uint64_t)(P_cap / 128 * kb128 * 2), 256, 8,
                       CU_TENSOR_MAP_SWIZZLE_NONE))
@@ -837,19 +877,20 @@ extern "C" moesq_status moesq_grouped_gemm(const moesq_linear* W, const uint8_t*
   }
 
   // clusters of 2 CTAs, one CTA per SM: as many pairs as the device can hold at once
+  constexpr size_t smem = sp::smem_bytes<DENSE>();
   static int pairs_cache[64][3] = {{0}};
   const int ei = epilogue - MOESQ_EPI_F32;
   int pairs = dev < 64 ? pairs_cache[dev][ei] : 0;
   if (pairs == 0) {
-    const void* fn = epilogue == MOESQ_EPI_F32 ? (const void*)sp::k_grouped_gemm_sp<MOESQ_EPI_F32>
-                     : epilogue == MOESQ_EPI_BF16 ? (const void*)sp::k_grouped_gemm_sp<MOESQ_EPI_BF16>
-                                                  : (const void*)sp::k_grouped_gemm_sp<MOESQ_EPI_SWIGLU_NVFP4>;
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp::SMEM_BYTES) != cudaSuccess)
+    const void* fn = epilogue == MOESQ_EPI_F32 ? (const void*)sp::k_grouped_gemm_sp<MOESQ_EPI_F32, DENSE>
+                     : epilogue == MOESQ_EPI_BF16 ? (const void*)sp::k_grouped_gemm_sp<MOESQ_EPI_BF16, DENSE>
+                                                  : (const void*)sp::k_grouped_gemm_sp<MOESQ_EPI_SWIGLU_NVFP4, DENSE>;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
       return MOESQ_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(sms & ~1));
     cfg.blockDim = dim3(sp::THREADS);
-    cfg.dynamicSmemBytes = sp::SMEM_BYTES;
+    cfg.dynamicSmemBytes = smem;
     int n = 0;
     if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess || n < 1) {
       (void)cudaGetLastError();
@@ -883,15 +924,15 @@ extern "C" moesq_status moesq_grouped_gemm(const moesq_linear* W, const uint8_t*
   cudaError_t err;
   switch (epilogue) {
     case MOESQ_EPI_F32:
-      err = moesq_launch(sp::k_grouped_gemm_sp<MOESQ_EPI_F32>, grid, dim3(sp::THREADS), sp::SMEM_BYTES, st, ta, tb,
+      err = moesq_launch(sp::k_grouped_gemm_sp<MOESQ_EPI_F32, DENSE>, grid, dim3(sp::THREADS), smem, st, ta, tb,
                          tb16, te, tsfa, tsfb, ty, tb3, prm);
       break;
     case MOESQ_EPI_BF16:
-      err = moesq_launch(sp::k_grouped_gemm_sp<MOESQ_EPI_BF16>, grid, dim3(sp::THREADS), sp::SMEM_BYTES, st, ta, tb,
+      err = moesq_launch(sp::k_grouped_gemm_sp<MOESQ_EPI_BF16, DENSE>, grid, dim3(sp::THREADS), smem, st, ta, tb,
                          tb16, te, tsfa, tsfb, ty, tb3, prm);
       break;
     default:
-      err = moesq_launch(sp::k_grouped_gemm_sp<MOESQ_EPI_SWIGLU_NVFP4>, grid, dim3(sp::THREADS), sp::SMEM_BYTES, st,
+      err = moesq_launch(sp::k_grouped_gemm_sp<MOESQ_EPI_SWIGLU_NVFP4, DENSE>, grid, dim3(sp::THREADS), smem, st,
                          ta, tb, tb16, te, tsfa, tsfb, ty, tb3, prm);
   }
   if (err != cudaSuccess) {
@@ -899,4 +940,27 @@ extern "C" moesq_status moesq_grouped_gemm(const moesq_linear* W, const uint8_t*
     return MOESQ_ERR_CUDA;
   }
   return MOESQ_OK;
+}
+
+extern "C" moesq_status moesq_grouped_gemm(const moesq_linear* W, const uint8_t* act_codes,
+                                           const uint8_t* act_sf, const float* g_act,
+                                           const int32_t* expert_offsets,
+                                           const int32_t* pad_offsets, int64_t S, int64_t P_cap,
+                                           int32_t epilogue, const float* g_next, void* out,
+                                           uint8_t* out_sf, void* ws, size_t ws_bytes,
+                                           int32_t* d_status, moesq_stream_t stream) {
+  (void)ws;
+  (void)ws_bytes;
+  return grouped_gemm_impl<false>(W, act_codes, act_sf, g_act, expert_offsets, pad_offsets, S, P_cap, epilogue,
+                                  g_next, out, out_sf, d_status, stream);
+}
+
+extern "C" moesq_status moesq_grouped_gemm_dense(const moesq_linear* W, const uint8_t* act_codes,
+                                                 const uint8_t* act_sf, const float* g_act,
+                                                 const int32_t* expert_offsets, const int32_t* pad_offsets,
+                                                 int64_t S, int64_t P_cap, int32_t epilogue,
+                                                 const float* g_next, void* out, uint8_t* out_sf,
+                                                 int32_t* d_status, moesq_stream_t stream) {
+  return grouped_gemm_impl<true>(W, act_codes, act_sf, g_act, expert_offsets, pad_offsets, S, P_cap, epilogue,
+                                 g_next, out, out_sf, d_status, stream);
 }

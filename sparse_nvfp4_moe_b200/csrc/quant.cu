@@ -125,9 +125,39 @@ __global__ void k_quant_act_routed(const uint16_t* __restrict__ x, int64_t T, in
   }
 }
 
+// 32-element scale blocks -> 16-element scale blocks: thread per (block, lane l),
+// one 16-byte row of four 4-scale words in, one such row out to each of the two
+// blocks (scales 0,0,1,1 and 2,2,3,3 of every word)
+__global__ void k_sf_expand_block16(const uint4* __restrict__ in, uint4* __restrict__ out, int64_t n) {
+  pdl_wait();
+  pdl_trigger();
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const uint4 v = in[i];
+    const int64_t b = i >> 5, l = i & 31;
+    out[(2 * b) * 32 + l] = make_uint4(__byte_perm(v.x, 0, 0x1100), __byte_perm(v.y, 0, 0x1100),
+                                       __byte_perm(v.z, 0, 0x1100), __byte_perm(v.w, 0, 0x1100));
+    out[(2 * b + 1) * 32 + l] = make_uint4(__byte_perm(v.x, 0, 0x3322), __byte_perm(v.y, 0, 0x3322),
+                                           __byte_perm(v.z, 0, 0x3322), __byte_perm(v.w, 0, 0x3322));
+  }
+}
+
 }  // namespace moesq
 
 using namespace moesq;
+
+extern "C" moesq_status moesq_sf_expand_block16(const uint8_t* sf32, uint8_t* sf16, int64_t nblocks,
+                                                moesq_stream_t stream) {
+  MOESQ_REQUIRE(nblocks >= 0, MOESQ_ERR_INVALID_ARG);
+  if (nblocks == 0) return MOESQ_OK;
+  MOESQ_REQUIRE(sf32 && sf16 && moesq_aligned16(sf32) && moesq_aligned16(sf16), MOESQ_ERR_INVALID_ARG);
+  const int64_t n = nblocks * 32;
+  int64_t g = (n + 255) / 256;
+  if (g > 148 * 16) g = 148 * 16;
+  if (moesq_launch(k_sf_expand_block16, dim3((unsigned)g), dim3(256), 0, (cudaStream_t)stream,
+                   reinterpret_cast<const uint4*>(sf32), reinterpret_cast<uint4*>(sf16), n) != cudaSuccess)
+    return MOESQ_ERR_CUDA;
+  return MOESQ_OK;
+}
 
 extern "C" moesq_status moesq_quant_act_routed(const uint16_t* x, int64_t T, int64_t K,
                                                const int32_t* topk_ids, const int32_t* token_slot,
