@@ -361,6 +361,19 @@ moesq_status moesq_moe_forward_host(const moesq_moe_layer* L, const uint16_t* h_
 moesq_status moesq_moe_forward_host_workspace_size(const moesq_moe_layer* L, int64_t T,
                                                    size_t* bytes);
 
+/* ------------------------------------------------------------------------- *
+ * Self-test of the failure path
+ * ------------------------------------------------------------------------- */
+
+/* Runs the library's three bounded mbarrier waits (the ones every pipeline wait goes
+ * through) on a barrier phase that nothing completes.  Each gives up after limit_ns
+ * (0 < limit_ns <= 1e8; polling checks the clock every few tries, so the kernel runs
+ * a small multiple of limit_ns), ORs MOESQ_DFLAG_TIMEOUT into *d_status and writes 1
+ * to d_gave_up[i] (device i32 [3]: suspending, spinning, polling wait).  The kernel
+ * returns normally: no fault, no trap. */
+moesq_status moesq_selftest_wait_timeout(int32_t* d_status, int64_t limit_ns, int32_t* d_gave_up,
+                                         moesq_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -62,6 +62,7 @@ _SIGS = {
     "moesq_grouped_gemm_dense": (ctypes.c_int, [ctypes.POINTER(Linear), c_vp, c_vp, c_vp, c_vp, c_vp, c_i64,
                                                 c_i64, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp]),
     "moesq_sf_expand_block16": (ctypes.c_int, [c_vp, c_vp, c_i64, c_vp]),
+    "moesq_selftest_wait_timeout": (ctypes.c_int, [c_vp, c_i64, c_vp, c_vp]),
     "moesq_grouped_gemm_workspace_size": (ctypes.c_int, [ctypes.POINTER(Linear), c_i64,
                                                          ctypes.POINTER(c_sz)]),
     "moesq_moe_forward": (ctypes.c_int, [ctypes.POINTER(MoeLayer), c_vp, c_vp, c_vp, c_i64, c_vp, c_vp,
@@ -230,6 +231,11 @@ def moesq_grouped_gemm_dense(W: Linear, act_codes, act_sf, g_act, expert_offsets
     _check("moesq_grouped_gemm_dense", lib().moesq_grouped_gemm_dense(
         ctypes.byref(W), _p(act_codes), _p(act_sf), _p(g_act), _p(expert_offsets), _p(pad_offsets), S,
         P_cap, epilogue, _p(g_next), _p(out), _p(out_sf), _p(d_status), _stream(stream)))
+
+
+def moesq_selftest_wait_timeout(d_status, limit_ns, d_gave_up, stream=None):
+    _check("moesq_selftest_wait_timeout", lib().moesq_selftest_wait_timeout(_p(d_status), limit_ns, _p(d_gave_up),
+                                                                              _stream(stream)))
 
 
 def moesq_sf_expand_block16(sf32, sf16, nblocks, stream=None):

@@ -171,3 +171,37 @@ extern "C" moesq_status moesq_moe_forward_host(const moesq_moe_layer* L, const u
   if (cudaStreamSynchronize(s) != cudaSuccess) return MOESQ_ERR_CUDA;
   return MOESQ_OK;
 }
+
+// ----------------------------------------------------------------- self-test --
+// The bounded-wait failure path, exercised without a fault: thread 0 runs each of
+// the library's three pipeline waits (suspending, spinning, polling) on an mbarrier
+// phase that nothing completes.  Each gives up after limit_ns, ORs
+// MOESQ_DFLAG_TIMEOUT into the status word and reports it; the kernel then
+// returns normally and the context stays usable.
+namespace {
+__global__ void k_wait_timeout_selftest(int32_t* d_status, uint64_t limit_ns, int32_t* gave_up) {
+  __shared__ uint64_t bar[3];
+  __shared__ int abort_flag[3];
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 3; ++i) {
+      moesq::mbar_init(&bar[i], 1);
+      abort_flag[i] = 0;
+    }
+    moesq::fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // phase 0 of a fresh barrier completes on one arrival, which never comes
+    gave_up[0] = moesq::mbar_wait(&bar[0], 0, &abort_flag[0], d_status, limit_ns) ? 0 : 1;
+    gave_up[1] = moesq::mbar_wait_spin(&bar[1], 0, &abort_flag[1], d_status, limit_ns) ? 0 : 1;
+    gave_up[2] = moesq::mbar_wait_poll(&bar[2], 0, &abort_flag[2], d_status, limit_ns) ? 0 : 1;
+  }
+}
+}  // namespace
+
+extern "C" moesq_status moesq_selftest_wait_timeout(int32_t* d_status, int64_t limit_ns, int32_t* d_gave_up,
+                                                    moesq_stream_t stream) {
+  MOESQ_REQUIRE(d_status && d_gave_up && limit_ns > 0 && limit_ns <= 100000000, MOESQ_ERR_INVALID_ARG);
+  k_wait_timeout_selftest<<<1, 32, 0, (cudaStream_t)stream>>>(d_status, (uint64_t)limit_ns, d_gave_up);
+  return cudaGetLastError() == cudaSuccess ? MOESQ_OK : MOESQ_ERR_CUDA;
+}

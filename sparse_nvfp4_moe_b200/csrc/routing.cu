@@ -126,6 +126,108 @@ __global__ void __launch_bounds__(PERM_THREADS) k_perm_scan(int32_t* __restrict_
   }
 }
 
+// pass 2 of moesq_permute, spread over the GPU: a warp per expert scans its row of
+// chunk counts in place (exclusive, within the expert) and writes the expert's
+// total.  Four rows of 32 chunks are in flight per warp at a time.
+__global__ void __launch_bounds__(PERM_THREADS) k_perm_scan_rows(int32_t* __restrict__ counts, int nchunks,
+                                                                 int E, int32_t* __restrict__ totals) {
+  pdl_wait();
+  pdl_trigger();
+  const int lane = threadIdx.x & 31;
+  const int e = blockIdx.x * (PERM_THREADS / 32) + (threadIdx.x >> 5);
+  if (e >= E) return;
+  int32_t* row = counts + (int64_t)e * nchunks;
+  int32_t run = 0;
+  for (int c0 = 0; c0 < nchunks; c0 += 4 * 32) {
+    int32_t v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int c = c0 + 32 * u + lane;
+      v[u] = c < nchunks ? row[c] : 0;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      int32_t x = v[u];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      const int c = c0 + 32 * u + lane;
+      if (c < nchunks) row[c] = run + x - v[u];
+      run += __shfl_sync(0xffffffffu, x, 31);
+    }
+  }
+  if (lane == 0) totals[e] = run;
+}
+
+// pass 3 of moesq_permute: every block scans the expert totals itself (its own
+// slot bases), block 0 also publishes the expert and padded offsets; then the
+// stable scatter of the chunk, warps taking turns in order
+__global__ void __launch_bounds__(PERM_THREADS) k_perm_scatter_scan(
+    const int32_t* __restrict__ ids, int64_t S, int k, int E, const int32_t* __restrict__ chunk_base,
+    const int32_t* __restrict__ totals, int32_t* __restrict__ expert_offsets, int32_t* __restrict__ pad_offsets,
+    int32_t* __restrict__ slot_token, int32_t* __restrict__ token_slot) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ int32_t run[];  // [E] next free slot of each expert for this chunk
+  __shared__ int32_t warp_sums[32];
+  __shared__ int32_t total;
+  const int ept = (E + PERM_THREADS - 1) / PERM_THREADS;
+  const int e0 = threadIdx.x * ept;
+  int32_t la = 0, lb = 0;
+  for (int j = 0; j < ept; ++j)
+    if (e0 + j < E) {
+      const int32_t t = totals[e0 + j];
+      la += t;
+      lb += (t + 127) / 128 * 128;
+    }
+  int32_t ea = block_excl_scan(la, warp_sums, &total);
+  const int32_t ta = total;
+  int32_t eb = block_excl_scan(lb, warp_sums, &total);
+  const int32_t tb = total;
+  for (int j = 0; j < ept; ++j)
+    if (e0 + j < E) {
+      const int e = e0 + j;
+      const int32_t t = totals[e];
+      run[e] = ea + chunk_base[(int64_t)e * gridDim.x + blockIdx.x];
+      if (blockIdx.x == 0) {
+        expert_offsets[e] = ea;
+        pad_offsets[e] = eb;
+      }
+      ea += t;
+      eb += (t + 127) / 128 * 128;
+    }
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    expert_offsets[E] = ta;
+    pad_offsets[E] = tb;
+  }
+  __syncthreads();
+  const int64_t i = (int64_t)blockIdx.x * PERM_CHUNK + threadIdx.x;
+  const bool valid = i < S;
+  int e = 0;
+  if (valid) {
+    e = ids[i];
+    if (e < 0 || e >= E) e = 0;
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const unsigned vmask = __ballot_sync(0xffffffffu, valid);
+  const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : -1);
+  const int rank = __popc(peers & ((1u << lane) - 1u));
+  const int cnt = __popc(peers);
+  const bool leader = valid && (rank == cnt - 1);
+  for (int w = 0; w < PERM_THREADS / 32; ++w) {
+    if (warp == w && valid) {
+      const int pos = run[e] + rank;
+      __syncwarp(vmask);
+      if (leader) run[e] = pos + 1;
+      slot_token[pos] = (int32_t)(i / k);
+      token_slot[i] = pos;
+    }
+    __syncthreads();
+  }
+}
+
 // pass 3: stable scatter; warps of the chunk take turns in order
 __global__ void __launch_bounds__(PERM_THREADS) k_perm_scatter(
     const int32_t* __restrict__ ids, int64_t S, int k, int E, const int32_t* __restrict__ chunk_base,
@@ -211,7 +313,8 @@ extern "C" moesq_status moesq_permute_workspace_size(int64_t T, int32_t k, int32
                 MOESQ_ERR_INVALID_ARG);
   const int64_t S = T * k;
   const int64_t nchunks = (S + PERM_CHUNK - 1) / PERM_CHUNK;
-  *bytes = (size_t)((nchunks > 0 ? nchunks : 1) * E) * sizeof(int32_t);
+  // per-chunk expert counts, then one total per expert
+  *bytes = (size_t)((nchunks > 0 ? nchunks : 1) * E + E) * sizeof(int32_t);
   return MOESQ_OK;
 }
 
@@ -231,19 +334,23 @@ extern "C" moesq_status moesq_permute(const int32_t* topk_ids, int64_t T, int32_
   const int nchunks = (int)((S + PERM_CHUNK - 1) / PERM_CHUNK);
   int32_t* counts = (int32_t*)ws;
   const size_t shm = (size_t)E * sizeof(int32_t);
-  if (nchunks > 0) {
-    if (moesq_launch(k_perm_count, dim3(nchunks), dim3(PERM_THREADS), shm, s, topk_ids, S, E, nchunks, counts,
-                     d_status) != cudaSuccess)
+  if (nchunks == 0) {  // no slots: the offsets are all zero
+    if (moesq_launch(k_perm_scan, dim3(1), dim3(PERM_THREADS), shm, s, counts, nchunks, E, expert_offsets,
+                     pad_offsets) != cudaSuccess)
       return MOESQ_ERR_CUDA;
+    return MOESQ_OK;
   }
-  if (moesq_launch(k_perm_scan, dim3(1), dim3(PERM_THREADS), shm, s, counts, nchunks, E, expert_offsets,
-                   pad_offsets) != cudaSuccess)
+  int32_t* totals = counts + (int64_t)nchunks * E;
+  if (moesq_launch(k_perm_count, dim3(nchunks), dim3(PERM_THREADS), shm, s, topk_ids, S, E, nchunks, counts,
+                   d_status) != cudaSuccess)
     return MOESQ_ERR_CUDA;
-  if (nchunks > 0) {
-    if (moesq_launch(k_perm_scatter, dim3(nchunks), dim3(PERM_THREADS), shm, s, topk_ids, S, k, E,
-                     (const int32_t*)counts, (const int32_t*)expert_offsets, slot_token, token_slot) != cudaSuccess)
-      return MOESQ_ERR_CUDA;
-  }
+  if (moesq_launch(k_perm_scan_rows, dim3((E + PERM_THREADS / 32 - 1) / (PERM_THREADS / 32)), dim3(PERM_THREADS),
+                   0, s, counts, nchunks, E, totals) != cudaSuccess)
+    return MOESQ_ERR_CUDA;
+  if (moesq_launch(k_perm_scatter_scan, dim3(nchunks), dim3(PERM_THREADS), shm, s, topk_ids, S, k, E,
+                   (const int32_t*)counts, (const int32_t*)totals, expert_offsets, pad_offsets, slot_token,
+                   token_slot) != cudaSuccess)
+    return MOESQ_ERR_CUDA;
   return MOESQ_OK;
 }
 

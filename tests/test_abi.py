@@ -65,6 +65,15 @@ def test_argument_validation_is_synchronous(lib):
                                   None, None) == INVALID                       # SwiGLU on down
 
 
+def test_selftest_arguments_checked_before_launch(lib):
+    INVALID = 1
+    buf = ctypes.create_string_buffer(64)
+    p = ctypes.addressof(buf)
+    assert lib.moesq_selftest_wait_timeout(None, 1000, p, None) == INVALID
+    assert lib.moesq_selftest_wait_timeout(p, 0, p, None) == INVALID
+    assert lib.moesq_selftest_wait_timeout(p, 200000000, p, None) == INVALID   # limit above 0.1 s
+
+
 def test_size_queries(lib):
     from sparse_nvfp4_moe_b200 import _lib
     assert _lib.repack_sizes(256, 256) == (2 * 1 * 2048, 2 * 2 * 512)
@@ -72,5 +81,5 @@ def test_size_queries(lib):
     assert _lib.padded_rows(0, 8) == 0
     assert _lib.padded_rows(1, 8) == 128
     assert _lib.padded_rows(300, 2) == ((300 + 2 * 127 + 127) // 128) * 128
-    assert _lib.permute_workspace_size(64, 2, 8) == 8 * 4
+    assert _lib.permute_workspace_size(64, 2, 8) == (1 * 8 + 8) * 4      # chunk counts + expert totals
     assert _lib.quant_weight_workspace_size(8, 2) == 64
