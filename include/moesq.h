@@ -320,6 +320,19 @@ moesq_status moesq_grouped_gemm_dense(const moesq_linear* W, const uint8_t* act_
                                       void* out, uint8_t* out_sf, int32_t* d_status,
                                       moesq_stream_t stream);
 
+/* Routed NVFP4 rows quantised elsewhere (e.g. received from the GPU that holds the
+ * tokens) -> the padded operand layout of moesq_grouped_gemm.
+ *   codes_in device u8 [n, K/2], sf_in device u8 [n, K/32] (linear, MOESQ_SF_LINEAR)
+ *   gather   device i32 [S]: input row of slot s, slots in expert order (moesq_permute's
+ *            slot_token of the received rows)
+ *   expert_offsets, pad_offsets device i32 [E+1] (moesq_permute)
+ *   codes_out device u8 [P, K/2], sf_out device u8 [P/128][K/128][512] (MOESQ_SF_KERNEL)
+ * K % 128 == 0; codes 16-byte aligned.  Bytes are copied unchanged. */
+moesq_status moesq_gather_act(const uint8_t* codes_in, const uint8_t* sf_in, const int32_t* gather,
+                              int64_t S, int64_t K, const int32_t* expert_offsets,
+                              const int32_t* pad_offsets, int32_t E, uint8_t* codes_out, uint8_t* sf_out,
+                              moesq_stream_t stream);
+
 /* 32-element scale blocks -> 16-element scale blocks for the dense MMA: each 512-byte
  * block b (128 rows x 4 scales, one per 32 K: row r, scale j at (r%32)*16 + (r/32)*4 + j)
  * becomes blocks 2b and 2b+1 (one scale per 16 K, each 32-element scale written twice).

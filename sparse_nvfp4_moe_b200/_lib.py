@@ -63,6 +63,7 @@ _SIGS = {
                                                 c_i64, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp]),
     "moesq_sf_expand_block16": (ctypes.c_int, [c_vp, c_vp, c_i64, c_vp]),
     "moesq_selftest_wait_timeout": (ctypes.c_int, [c_vp, c_i64, c_vp, c_vp]),
+    "moesq_gather_act": (ctypes.c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp]),
     "moesq_grouped_gemm_workspace_size": (ctypes.c_int, [ctypes.POINTER(Linear), c_i64,
                                                          ctypes.POINTER(c_sz)]),
     "moesq_moe_forward": (ctypes.c_int, [ctypes.POINTER(MoeLayer), c_vp, c_vp, c_vp, c_i64, c_vp, c_vp,
@@ -231,6 +232,13 @@ def moesq_grouped_gemm_dense(W: Linear, act_codes, act_sf, g_act, expert_offsets
     _check("moesq_grouped_gemm_dense", lib().moesq_grouped_gemm_dense(
         ctypes.byref(W), _p(act_codes), _p(act_sf), _p(g_act), _p(expert_offsets), _p(pad_offsets), S,
         P_cap, epilogue, _p(g_next), _p(out), _p(out_sf), _p(d_status), _stream(stream)))
+
+
+def moesq_gather_act(codes_in, sf_in, gather, S, K, expert_offsets, pad_offsets, E, codes_out, sf_out,
+                     stream=None):
+    _check("moesq_gather_act", lib().moesq_gather_act(_p(codes_in), _p(sf_in), _p(gather), S, K, _p(expert_offsets),
+                                                      _p(pad_offsets), E, _p(codes_out), _p(sf_out),
+                                                      _stream(stream)))
 
 
 def moesq_selftest_wait_timeout(d_status, limit_ns, d_gave_up, stream=None):

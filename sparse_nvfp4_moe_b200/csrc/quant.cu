@@ -125,6 +125,31 @@ __global__ void k_quant_act_routed(const uint16_t* __restrict__ x, int64_t T, in
   }
 }
 
+// Routed NVFP4 rows quantised elsewhere (codes [n, K/2], linear scales [n, K/32], e.g.
+// received from another GPU) into the grouped GEMM's padded operand layout: slot s of
+// the expert-ordered list takes input row gather[s] and lands on padded row
+// pad_offsets[e] + (s - expert_offsets[e]).  Thread per (slot, 32-element group): one
+// 16-byte code chunk and one scale byte.
+__global__ void k_gather_act(const uint8_t* __restrict__ codes_in, const uint8_t* __restrict__ sf_in,
+                             const int32_t* __restrict__ gather, int64_t S, int64_t K,
+                             const int32_t* __restrict__ expert_offsets, const int32_t* __restrict__ pad_offsets,
+                             int E, uint8_t* __restrict__ codes_out, uint8_t* __restrict__ sf_out) {
+  pdl_wait();
+  pdl_trigger();
+  const int64_t G = K / 32;
+  const int64_t n = S * G;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t s = i / G, grp = i % G;
+    const int64_t src = gather[s];
+    const int e = find_expert(expert_offsets, E, s);
+    const int64_t row = (int64_t)pad_offsets[e] + (s - expert_offsets[e]);
+    *reinterpret_cast<uint4*>(codes_out + row * (K / 2) + 16 * grp) =
+        *reinterpret_cast<const uint4*>(codes_in + src * (K / 2) + 16 * grp);
+    const int64_t blk = (row / 128) * (K / 128) + grp / 4;
+    sf_out[blk * 512 + sf_block_offset((uint32_t)(row % 128), (uint32_t)(grp % 4))] = sf_in[src * G + grp];
+  }
+}
+
 // 32-element scale blocks -> 16-element scale blocks: thread per (block, lane l),
 // one 16-byte row of four 4-scale words in, one such row out to each of the two
 // blocks (scales 0,0,1,1 and 2,2,3,3 of every word)
@@ -144,6 +169,26 @@ __global__ void k_sf_expand_block16(const uint4* __restrict__ in, uint4* __restr
 }  // namespace moesq
 
 using namespace moesq;
+
+extern "C" moesq_status moesq_gather_act(const uint8_t* codes_in, const uint8_t* sf_in, const int32_t* gather,
+                                         int64_t S, int64_t K, const int32_t* expert_offsets,
+                                         const int32_t* pad_offsets, int32_t E, uint8_t* codes_out,
+                                         uint8_t* sf_out, moesq_stream_t stream) {
+  MOESQ_REQUIRE(S >= 0 && K >= 0 && E >= 1, MOESQ_ERR_INVALID_ARG);
+  MOESQ_REQUIRE(K % 128 == 0, MOESQ_ERR_UNSUPPORTED_SHAPE);
+  if (S == 0 || K == 0) return MOESQ_OK;
+  MOESQ_REQUIRE(codes_in && sf_in && gather && expert_offsets && pad_offsets && codes_out && sf_out,
+                MOESQ_ERR_INVALID_ARG);
+  MOESQ_REQUIRE(moesq_aligned16(codes_in) && moesq_aligned16(codes_out) && moesq_aligned16(sf_out),
+                MOESQ_ERR_INVALID_ARG);
+  const int64_t n = S * (K / 32);
+  int64_t g = (n + 255) / 256;
+  if (g > 148 * 16) g = 148 * 16;
+  if (moesq_launch(k_gather_act, dim3((unsigned)g), dim3(256), 0, (cudaStream_t)stream, codes_in, sf_in, gather, S, K,
+                   expert_offsets, pad_offsets, (int)E, codes_out, sf_out) != cudaSuccess)
+    return MOESQ_ERR_CUDA;
+  return MOESQ_OK;
+}
 
 extern "C" moesq_status moesq_sf_expand_block16(const uint8_t* sf32, uint8_t* sf16, int64_t nblocks,
                                                 moesq_stream_t stream) {
