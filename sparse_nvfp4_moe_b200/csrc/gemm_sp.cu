@@ -21,11 +21,18 @@
 //     tokens, metadata, block scales) into a 4-stage shared-memory ring of
 //     512-deep K blocks; warp 1 of the first CTA copies metadata and scales
 //     smem->TMEM (tcgen05.cp) and issues the MMAs (dense K = 128 each, four per
-//     stage); warps 2..9 of each CTA drain its double-buffered FP32
+//     stage); warps 2..17 of each CTA drain its double-buffered FP32
 //     accumulators (tcgen05.ld) while the next tile runs;
+//   * reads weight tiles whose rows the repack interleaves, so that one 16x256b
+//     TMEM load gives a thread both operands of an epilogue pair (gate and up of
+//     an output, or two neighbouring outputs) and no lanes exchange values;
 //   * fuses the epilogue: FP32 or bf16 output per slot, or SwiGLU followed by
 //     NVFP4 requantisation written straight into the next GEMM's B operand
 //     layout (codes + 512-byte scale blocks).
+//
+// The same kernel, with a dense stage geometry (256-deep stages of four dense
+// kind::mxf4nvf4 MMAs, no metadata), is the dense comparison GEMM on decoded
+// weights (moesq_grouped_gemm_dense).
 //
 // Every mbarrier wait is bounded (2 s); on expiry the kernel flags
 // MOESQ_DFLAG_TIMEOUT, drains its own copies in flight, frees TMEM and exits.
@@ -65,10 +72,10 @@ template <bool DENSE>
 __host__ __device__ constexpr int stage_bytes() {
   return Geo<DENSE>::A_BYTES + Geo<DENSE>::B_BYTES + Geo<DENSE>::E_BYTES + 2 * SF_BYTES;  // 40960 / 28672
 }
-constexpr int EPI_BYTES = 32768;  // epilogue exchange / transpose / staging space
+constexpr int EPI_BYTES = 32768;  // epilogue space: bf16 staging, f32 transposes, SwiGLU amax swaps
 constexpr int MAX_E = 1024;
-// Sixteen epilogue warps, four per sub-partition: the epilogue is latency-bound
-// (TMEM loads, shared-memory transposes, MUFU-heavy SiLU), so it wants warps;
+// Sixteen epilogue warps, four per sub-partition: the epilogue is bound by issue
+// and latency (TMEM loads, MUFU-heavy SiLU, lane exchanges), so it wants warps;
 // 18 warps leave 112 registers a thread.
 constexpr int EPI_WARPS = 16;
 constexpr int EPI_THREADS = 32 * EPI_WARPS;
