@@ -72,6 +72,7 @@ __global__ void k_quant_act(const uint16_t* __restrict__ x, int64_t K, const int
 // Token-major variant for the MoE forward: thread per (token, 32-group); x is
 // read once per token and written once per routed slot (k times), each with the
 // global of the slot's expert, into the padded operand layout.
+template <bool BATCHED>
 __global__ void k_quant_act_routed(const uint16_t* __restrict__ x, int64_t T, int64_t K,
                                    const int32_t* __restrict__ topk_ids,
                                    const int32_t* __restrict__ token_slot, int k,
@@ -106,21 +107,61 @@ __global__ void k_quant_act_routed(const uint16_t* __restrict__ x, int64_t T, in
     float g_prev = 0.0f;
     GroupScale gs = {0u, 0.0f};
     uint32_t o[4] = {0u, 0u, 0u, 0u};
-    for (int j = 0; j < k; ++j) {
-      int e = topk_ids[t * k + j];
-      if (e < 0 || e >= E) e = 0;
-      const int64_t s = token_slot[t * k + j];
-      const float g = g_in[e];
-      if (j == 0 || __float_as_uint(g) != __float_as_uint(g_prev)) {
-        g_prev = g;
-        gs = nvfp4_group_scale(amax, g);
+    if constexpr (!BATCHED) {
+      // large batches: one slot at a time (fewer registers, more warps to hide latency)
+      for (int j = 0; j < k; ++j) {
+        int e = topk_ids[t * k + j];
+        if (e < 0 || e >= E) e = 0;
+        const int64_t s = token_slot[t * k + j];
+        const float g = g_in[e];
+        if (j == 0 || __float_as_uint(g) != __float_as_uint(g_prev)) {
+          g_prev = g;
+          gs = nvfp4_group_scale(amax, g);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) o[c] = nvfp4_word(v + 8 * c, gs.inv);
+          for (int c = 0; c < 4; ++c) o[c] = nvfp4_word(v + 8 * c, gs.inv);
+        }
+        const int64_t row = (int64_t)pad_offsets[e] + (s - expert_offsets[e]);
+        *reinterpret_cast<uint4*>(codes + row * (K / 2) + 16 * grp) = make_uint4(o[0], o[1], o[2], o[3]);
+        const int64_t blk = (row / 128) * (K / 128) + grp / 4;
+        sf[blk * 512 + sf_block_offset((uint32_t)(row % 128), (uint32_t)(grp % 4))] = (uint8_t)gs.sc;
       }
-      const int64_t row = (int64_t)pad_offsets[e] + (s - expert_offsets[e]);
-      *reinterpret_cast<uint4*>(codes + row * (K / 2) + 16 * grp) = make_uint4(o[0], o[1], o[2], o[3]);
-      const int64_t blk = (row / 128) * (K / 128) + grp / 4;
-      sf[blk * 512 + sf_block_offset((uint32_t)(row % 128), (uint32_t)(grp % 4))] = (uint8_t)gs.sc;
+    } else {
+      // slots in chunks of 8: all index and table loads of a chunk are issued before any
+      // is used, so a small batch waits for two load round trips per chunk, not per slot
+      for (int j0 = 0; j0 < k; j0 += 8) {
+        int ev[8];
+        int64_t rowv[8];
+        float gv[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int j = j0 + u;
+          int e = j < k ? topk_ids[t * k + j] : 0;
+          ev[u] = (e < 0 || e >= E) ? 0 : e;
+          rowv[u] = j < k ? (int64_t)token_slot[t * k + j] : 0;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          gv[u] = g_in[ev[u]];
+          rowv[u] += (int64_t)pad_offsets[ev[u]] - expert_offsets[ev[u]];
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int j = j0 + u;
+          if (j < k) {
+            const float g = gv[u];
+            if (j == 0 || __float_as_uint(g) != __float_as_uint(g_prev)) {
+              g_prev = g;
+              gs = nvfp4_group_scale(amax, g);
+#pragma unroll
+              for (int c = 0; c < 4; ++c) o[c] = nvfp4_word(v + 8 * c, gs.inv);
+            }
+            const int64_t row = rowv[u];
+            *reinterpret_cast<uint4*>(codes + row * (K / 2) + 16 * grp) = make_uint4(o[0], o[1], o[2], o[3]);
+            const int64_t blk = (row / 128) * (K / 128) + grp / 4;
+            sf[blk * 512 + sf_block_offset((uint32_t)(row % 128), (uint32_t)(grp % 4))] = (uint8_t)gs.sc;
+          }
+        }
+      }
     }
   }
 }
@@ -220,9 +261,13 @@ extern "C" moesq_status moesq_quant_act_routed(const uint16_t* x, int64_t T, int
   const int64_t n = T * (K / 32);
   int64_t g = (n + 127) / 128;
   if (g > 148 * 32) g = 148 * 32;
-  if (moesq_launch(k_quant_act_routed, dim3((unsigned)g), dim3(128), 0, (cudaStream_t)stream, x, T, K, topk_ids,
-                   token_slot, k, expert_offsets, pad_offsets, E, g_in, codes, sf) != cudaSuccess)
-    return MOESQ_ERR_CUDA;
+  // small batches (decode): every slot's index loads in flight at once; large: more warps
+  const cudaError_t err =
+      T <= 512 ? moesq_launch(k_quant_act_routed<true>, dim3((unsigned)g), dim3(128), 0, (cudaStream_t)stream, x, T, K,
+                              topk_ids, token_slot, k, expert_offsets, pad_offsets, E, g_in, codes, sf)
+               : moesq_launch(k_quant_act_routed<false>, dim3((unsigned)g), dim3(128), 0, (cudaStream_t)stream, x, T, K,
+                              topk_ids, token_slot, k, expert_offsets, pad_offsets, E, g_in, codes, sf);
+  if (err != cudaSuccess) return MOESQ_ERR_CUDA;
   return MOESQ_OK;
 }
 

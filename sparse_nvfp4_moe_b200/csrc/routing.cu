@@ -228,6 +228,74 @@ __global__ void __launch_bounds__(PERM_THREADS) k_perm_scatter_scan(
   }
 }
 
+// moesq_permute for a batch of at most one chunk (decode-sized): count, expert and
+// padded offsets, and the stable scatter in one block and one launch
+__global__ void __launch_bounds__(PERM_THREADS) k_perm_small(const int32_t* __restrict__ ids, int64_t S, int k,
+                                                             int E, int32_t* __restrict__ expert_offsets,
+                                                             int32_t* __restrict__ pad_offsets,
+                                                             int32_t* __restrict__ slot_token,
+                                                             int32_t* __restrict__ token_slot, int32_t* d_status) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ int32_t sm_small[];
+  int32_t* hist = sm_small;      // [E] counts, then the next free slot of each expert
+  __shared__ int32_t warp_sums[32];
+  __shared__ int32_t total;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int64_t i = threadIdx.x;
+  const bool valid = i < S;
+  int e = 0;
+  if (valid) {
+    e = clamp_expert(ids[i], E, d_status);
+    atomicAdd(&hist[e], 1);
+  }
+  __syncthreads();
+  const int ept = (E + PERM_THREADS - 1) / PERM_THREADS;
+  const int e0 = threadIdx.x * ept;
+  int32_t la = 0, lb = 0;
+  for (int j = 0; j < ept; ++j)
+    if (e0 + j < E) {
+      la += hist[e0 + j];
+      lb += (hist[e0 + j] + 127) / 128 * 128;
+    }
+  int32_t ea = block_excl_scan(la, warp_sums, &total);
+  const int32_t ta = total;
+  int32_t eb = block_excl_scan(lb, warp_sums, &total);
+  const int32_t tb = total;
+  for (int j = 0; j < ept; ++j)
+    if (e0 + j < E) {
+      const int32_t c = hist[e0 + j];
+      expert_offsets[e0 + j] = ea;
+      pad_offsets[e0 + j] = eb;
+      hist[e0 + j] = ea;  // each thread rewrites only its own experts
+      ea += c;
+      eb += (c + 127) / 128 * 128;
+    }
+  if (threadIdx.x == 0) {
+    expert_offsets[E] = ta;
+    pad_offsets[E] = tb;
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const unsigned vmask = __ballot_sync(0xffffffffu, valid);
+  const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : -1);
+  const int rank = __popc(peers & ((1u << lane) - 1u));
+  const int cnt = __popc(peers);
+  const bool leader = valid && (rank == cnt - 1);
+  const int nwarps = (int)((S + 31) / 32);
+  for (int w = 0; w < nwarps; ++w) {
+    if (warp == w && valid) {
+      const int pos = hist[e] + rank;
+      __syncwarp(vmask);
+      if (leader) hist[e] = pos + 1;
+      slot_token[pos] = (int32_t)(i / k);
+      token_slot[i] = pos;
+    }
+    __syncthreads();
+  }
+}
+
 // pass 3: stable scatter; warps of the chunk take turns in order
 __global__ void __launch_bounds__(PERM_THREADS) k_perm_scatter(
     const int32_t* __restrict__ ids, int64_t S, int k, int E, const int32_t* __restrict__ chunk_base,
@@ -265,6 +333,7 @@ __global__ void __launch_bounds__(PERM_THREADS) k_perm_scatter(
 }
 
 // combine: thread per (token, 8 features); float32 in j order, no fused multiply-add
+template <bool BATCHED>
 __global__ void k_unpermute(const uint16_t* __restrict__ y, const int32_t* __restrict__ token_slot,
                             const float* __restrict__ topk_w, int64_t T, int k, int64_t H,
                             uint16_t* __restrict__ out) {
@@ -278,15 +347,47 @@ __global__ void k_unpermute(const uint16_t* __restrict__ y, const int32_t* __res
     float acc[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
-    for (int j = 0; j < k; ++j) {
-      const int64_t s = token_slot[t * k + j];
-      const float w = topk_w[t * k + j];
-      const uint4 u = *reinterpret_cast<const uint4*>(y + s * H + 8 * c);
-      const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
+    if constexpr (!BATCHED) {
+      // large batches: one slot at a time (fewer registers, more warps to hide latency)
+      for (int j = 0; j < k; ++j) {
+        const int64_t s = token_slot[t * k + j];
+        const float w = topk_w[t * k + j];
+        const uint4 u = *reinterpret_cast<const uint4*>(y + s * H + 8 * c);
+        const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        acc[2 * q] = __fadd_rn(acc[2 * q], __fmul_rn(w, bf16_bits_to_float(wd[q] & 0xFFFF)));
-        acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], __fmul_rn(w, bf16_bits_to_float(wd[q] >> 16)));
+        for (int q = 0; q < 4; ++q) {
+          acc[2 * q] = __fadd_rn(acc[2 * q], __fmul_rn(w, bf16_bits_to_float(wd[q] & 0xFFFF)));
+          acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], __fmul_rn(w, bf16_bits_to_float(wd[q] >> 16)));
+        }
+      }
+    } else {
+      // slots in chunks of 8: the slot indices, weights and rows of a chunk are loaded
+      // before the sums, which still run in j order
+      for (int j0 = 0; j0 < k; j0 += 8) {
+        int64_t sv[8];
+        float wv[8];
+        uint4 uv[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int j = j0 + u;
+          sv[u] = j < k ? (int64_t)token_slot[t * k + j] : -1;
+          wv[u] = j < k ? topk_w[t * k + j] : 0.0f;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          uv[u] = sv[u] >= 0 ? *reinterpret_cast<const uint4*>(y + sv[u] * H + 8 * c) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (j0 + u < k) {
+            const float w = wv[u];
+            const uint32_t wd[4] = {uv[u].x, uv[u].y, uv[u].z, uv[u].w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              acc[2 * q] = __fadd_rn(acc[2 * q], __fmul_rn(w, bf16_bits_to_float(wd[q] & 0xFFFF)));
+              acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], __fmul_rn(w, bf16_bits_to_float(wd[q] >> 16)));
+            }
+          }
+        }
       }
     }
     uint32_t o[4];
@@ -340,6 +441,12 @@ extern "C" moesq_status moesq_permute(const int32_t* topk_ids, int64_t T, int32_
       return MOESQ_ERR_CUDA;
     return MOESQ_OK;
   }
+  if (nchunks == 1) {  // one chunk: everything in one block and one launch
+    if (moesq_launch(k_perm_small, dim3(1), dim3(PERM_THREADS), shm, s, topk_ids, S, k, E, expert_offsets, pad_offsets,
+                     slot_token, token_slot, d_status) != cudaSuccess)
+      return MOESQ_ERR_CUDA;
+    return MOESQ_OK;
+  }
   int32_t* totals = counts + (int64_t)nchunks * E;
   if (moesq_launch(k_perm_count, dim3(nchunks), dim3(PERM_THREADS), shm, s, topk_ids, S, E, nchunks, counts,
                    d_status) != cudaSuccess)
@@ -365,9 +472,13 @@ extern "C" moesq_status moesq_unpermute(const uint16_t* y, const int32_t* token_
   const int64_t n = T * (H / 8);
   int64_t g = (n + 255) / 256;
   if (g > 148 * 16) g = 148 * 16;
-  if (moesq_launch(k_unpermute, dim3((unsigned)g), dim3(256), 0, (cudaStream_t)stream, y, token_slot, topk_w, T, k,
-                   H, out) != cudaSuccess)
-    return MOESQ_ERR_CUDA;
+  // small batches (decode): every slot's loads in flight at once; large: more warps
+  const cudaError_t err =
+      T <= 512 ? moesq_launch(k_unpermute<true>, dim3((unsigned)g), dim3(256), 0, (cudaStream_t)stream, y, token_slot,
+                              topk_w, T, k, H, out)
+               : moesq_launch(k_unpermute<false>, dim3((unsigned)g), dim3(256), 0, (cudaStream_t)stream, y, token_slot,
+                              topk_w, T, k, H, out);
+  if (err != cudaSuccess) return MOESQ_ERR_CUDA;
   return MOESQ_OK;
 }
 
