@@ -462,8 +462,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     };
     TileWalk walk(S, pair_id, npairs, MT2, E);
     int sb = 0;  // SwiGLU staging buffer of this tile
-    for (int id = pair_id; id < total; id += npairs, walk.advance(MT2)) {
-      const Tile t = decode_tile(S, walk, E);
+    // the next tile is decoded while this one drains (a chain of shared-memory
+    // loads that would otherwise stand alone between tiles)
+    Tile tn = pair_id < total ? decode_tile(S, walk, E) : Tile{};
+    for (int id = pair_id; id < total; id += npairs) {
+      const Tile t = tn;
+      auto decode_next = [&]() {
+        if (id + npairs < total) {
+          walk.advance(MT2);
+          tn = decode_tile(S, walk, E);
+        }
+      };
       const int mt = 2 * t.mt + (int)rank;  // this CTA's weight tile
       const bool own_tile = mt < MT;          // false: the duplicate of an odd last tile
       const float2 ag = S.ag[t.e];
@@ -501,6 +510,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) release_acc(buf);
+        decode_next();
         if (live) {
           // amax of each column over this warp's 16 outputs: per thread over its two,
           // then over the 8 lanes of equal t%4 (lane bits 2..4) by three halving
@@ -549,15 +559,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // one TMA store of [32 rows][32 B] codes (rows past the expert's tokens are its
         // own padding, never read as tokens) and 2-byte scale pairs
         fence_proxy_async_smem();
-        if (q == 0 && lane == 0) bulk_wait_group_read0();  // the store two tiles back has read its buffer
+        if (q == 2 && lane == 0) bulk_wait_group_read0();  // the store two tiles back has read its buffer
         named_bar_sync(10 + kb, 128);  // also: both amax slots of every pair are read
         if (live) {
           const int64_t prow0 = (int64_t)t.prow + c_lo;
-          if (q == 0 && lane == 0) {
+          if (q == 2 && lane == 0) {
             tma_store_2d(&tmap_y, &S.hstg[sb][kb][0][0], 32 * mt, (int32_t)prow0);
             bulk_commit_group();
           }
-          if (q == 1 && lane < t.n_rows - c_lo) {
+          if (q == 3 && lane < t.n_rows - c_lo) {
             const int64_t prow = prow0 + lane;
             const int64_t blk = (prow / 128) * (I / 128) + (64 * mt) / 128;
             *reinterpret_cast<uint16_t*>(p.out_sf + blk * 512 + sf_block_offset((uint32_t)(prow % 128), 2u * (mt & 1))) =
@@ -590,7 +600,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) release_acc(buf);
-        const bool issuer = q == 0 && lane == 0;
+        decode_next();
+        const bool issuer = q == 2 && lane == 0;
         if (issuer) bulk_wait_group_read0();  // this block's previous stores have read the staging
         named_bar_sync(10 + kb, 128);         // (and its previous row copy is done)
         const bool gu = p.gate_up;
@@ -659,6 +670,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) release_acc(buf);
+        decode_next();
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
           const int cb = c_lo + 16 * h2;
@@ -700,7 +712,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   }
 
   if constexpr (EPI == MOESQ_EPI_BF16 || EPI == MOESQ_EPI_SWIGLU_NVFP4) {
-    if (warp >= 2 && (warp & 3) == 0 && lane == 0) bulk_wait_group0();  // the last stores are complete
+    if (warp >= 2 && (warp & 3) == 2 && lane == 0) bulk_wait_group0();  // the last stores are complete
   }
   // no CTA of the pair frees TMEM or exits while its peer may still use it
   tc_fence_before();
