@@ -3,10 +3,13 @@
 // The grouped GEMM of the pages runs over the tokens the router sends to each
 // expert (kernel line of the Qwen3.5-397B-A17B-P48NVFP4-MoESQ model card).  The
 // slot order is (expert, token, j): a stable counting sort of the flattened
-// top-k ids in three passes -- per-chunk histograms, one block scanning them,
-// and a stable scatter in which warps of a chunk take turns (match_any gives
-// the rank inside a warp).  Each expert's group also gets a 128-row aligned
-// place in the padded GEMM operand buffers (pad_offsets).
+// top-k ids.  Batches of more than 1024 slots take three passes -- per-chunk
+// histograms, a scan of them, and a stable scatter per 1024-slot chunk; smaller
+// ones take one block and one launch.  Within a chunk match_any gives a slot's rank among
+// its warp's slots of the same expert, and a [warp][expert] table of counts (up to
+// 512 experts; above that the warps take turns) its place after the chunk's
+// earlier warps.  Each expert's group also gets a 128-row aligned place in the
+// padded GEMM operand buffers (pad_offsets).
 #include "common.cuh"
 
 #include <mutex>
@@ -161,6 +164,60 @@ __global__ void __launch_bounds__(PERM_THREADS) k_perm_scan_rows(int32_t* __rest
   if (lane == 0) totals[e] = run;
 }
 
+// Largest expert count for which a block keeps a [32 warps][E] table of per-warp
+// counts in shared memory (64 KB + the run array); above it the warps take turns.
+constexpr int PERM_TABLE_MAX_E = 512;
+// Largest batch (flattened slots) that moesq_permute sorts in a single block: one
+// chunk.  Past it three launches win, since a block loops over its 1024-slot
+// sub-chunks at about 2.4 us each, while the three passes take about 8 us up to
+// 16K slots.
+constexpr int64_t PERM_BLOCK_MAX_S = PERM_CHUNK;
+
+// Stable scatter of the slots [base, base + 1024) by the whole block.  run[e] is the
+// next free position of expert e and is advanced past this sub-chunk's slots.  Each
+// warp ranks its lanes among equal experts (match_any) and its last lane of each
+// expert writes the warp's count into wcnt[warp][e]; one thread per expert then turns
+// its column of counts into exclusive prefixes over the warps, which places every
+// slot after all slots of lower index with the same expert.
+// e: expert of this thread's slot base + threadIdx.x (any value when past S).
+__device__ __forceinline__ void block_stable_scatter(int e, int64_t base, int64_t S, int k, int E, int32_t* run,
+                                                     int32_t* wcnt, int32_t* __restrict__ slot_token,
+                                                     int32_t* __restrict__ token_slot) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t i = base + threadIdx.x;
+  const bool valid = i < S;
+  if (!valid || e < 0 || e >= E) e = 0;
+  for (int x = threadIdx.x; x < 32 * E; x += blockDim.x) wcnt[x] = 0;
+  const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : -1);
+  const int rank = __popc(peers & ((1u << lane) - 1u));
+  const int cnt = __popc(peers);
+  __syncthreads();
+  if (valid && rank == cnt - 1) wcnt[warp * E + e] = cnt;
+  __syncthreads();
+  for (int x = threadIdx.x; x < E; x += blockDim.x) {
+    int32_t r = run[x];
+#pragma unroll
+    for (int w0 = 0; w0 < 32; w0 += 16) {  // 16 loads in flight (the block's 64-register limit)
+      int32_t c[16];
+#pragma unroll
+      for (int w = 0; w < 16; ++w) c[w] = wcnt[(w0 + w) * E + x];
+#pragma unroll
+      for (int w = 0; w < 16; ++w) {
+        wcnt[(w0 + w) * E + x] = r;
+        r += c[w];
+      }
+    }
+    run[x] = r;
+  }
+  __syncthreads();
+  if (valid) {
+    const int pos = wcnt[warp * E + e] + rank;
+    slot_token[pos] = (int32_t)(i / k);
+    token_slot[i] = pos;
+  }
+  __syncthreads();  // wcnt and run are reused by the next sub-chunk
+}
+
 // pass 3 of moesq_permute: every block scans the expert totals itself (its own
 // slot bases), block 0 also publishes the expert and padded offsets; then the
 // stable scatter of the chunk, warps taking turns in order
@@ -203,6 +260,12 @@ __global__ void __launch_bounds__(PERM_THREADS) k_perm_scatter_scan(
     pad_offsets[E] = tb;
   }
   __syncthreads();
+  if (E <= PERM_TABLE_MAX_E) {  // table of per-warp counts after run[E] (the launch sizes it)
+    const int64_t i0 = (int64_t)blockIdx.x * PERM_CHUNK + threadIdx.x;
+    block_stable_scatter(i0 < S ? ids[i0] : 0, (int64_t)blockIdx.x * PERM_CHUNK, S, k, E, run, run + E, slot_token,
+                         token_slot);
+    return;
+  }
   const int64_t i = (int64_t)blockIdx.x * PERM_CHUNK + threadIdx.x;
   const bool valid = i < S;
   int e = 0;
@@ -228,28 +291,33 @@ __global__ void __launch_bounds__(PERM_THREADS) k_perm_scatter_scan(
   }
 }
 
-// moesq_permute for a batch of at most one chunk (decode-sized): count, expert and
-// padded offsets, and the stable scatter in one block and one launch
-__global__ void __launch_bounds__(PERM_THREADS) k_perm_small(const int32_t* __restrict__ ids, int64_t S, int k,
+// moesq_permute for a batch of at most PERM_BLOCK_MAX_S slots (decode-sized): count,
+// expert and padded offsets, and the stable scatter in one block and one launch
+// (per-warp count table up to PERM_TABLE_MAX_E experts, else the warps take turns)
+__global__ void __launch_bounds__(PERM_THREADS) k_perm_block(const int32_t* __restrict__ ids, int64_t S, int k,
                                                              int E, int32_t* __restrict__ expert_offsets,
                                                              int32_t* __restrict__ pad_offsets,
                                                              int32_t* __restrict__ slot_token,
                                                              int32_t* __restrict__ token_slot, int32_t* d_status) {
   pdl_wait();
   pdl_trigger();
-  extern __shared__ int32_t sm_small[];
-  int32_t* hist = sm_small;      // [E] counts, then the next free slot of each expert
+  extern __shared__ int32_t sm_block[];
+  int32_t* hist = sm_block;      // [E] counts, then the next free slot of each expert
+  int32_t* wcnt = sm_block + E;  // [32][E] per-warp counts of a sub-chunk (table form only)
   __shared__ int32_t warp_sums[32];
   __shared__ int32_t total;
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
-  const int64_t i = threadIdx.x;
-  const bool valid = i < S;
-  int e = 0;
-  if (valid) {
-    e = clamp_expert(ids[i], E, d_status);
-    atomicAdd(&hist[e], 1);
+  // every thread keeps the experts of its slots (threadIdx.x + 1024 j) for the scatter
+  int ev[PERM_BLOCK_MAX_S / PERM_THREADS];
+#pragma unroll
+  for (int j = 0; j < PERM_BLOCK_MAX_S / PERM_THREADS; ++j) {
+    const int64_t i = threadIdx.x + (int64_t)PERM_THREADS * j;
+    ev[j] = i < S ? clamp_expert(ids[i], E, d_status) : 0;
   }
+#pragma unroll
+  for (int j = 0; j < PERM_BLOCK_MAX_S / PERM_THREADS; ++j)
+    if (threadIdx.x + (int64_t)PERM_THREADS * j < S) atomicAdd(&hist[ev[j]], 1);
   __syncthreads();
   const int ept = (E + PERM_THREADS - 1) / PERM_THREADS;
   const int e0 = threadIdx.x * ept;
@@ -277,14 +345,24 @@ __global__ void __launch_bounds__(PERM_THREADS) k_perm_small(const int32_t* __re
     pad_offsets[E] = tb;
   }
   __syncthreads();
+  if (E <= PERM_TABLE_MAX_E) {
+#pragma unroll
+    for (int j = 0; j < PERM_BLOCK_MAX_S / PERM_THREADS; ++j)
+      if ((int64_t)PERM_THREADS * j < S)
+        block_stable_scatter(ev[j], (int64_t)PERM_THREADS * j, S, k, E, hist, wcnt, slot_token, token_slot);
+    return;
+  }
+  static_assert(PERM_BLOCK_MAX_S == PERM_THREADS, "the turns form scatters one chunk");
+  const int64_t i = threadIdx.x;
+  const bool valid = i < S;
+  const int e = ev[0];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const unsigned vmask = __ballot_sync(0xffffffffu, valid);
   const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : -1);
   const int rank = __popc(peers & ((1u << lane) - 1u));
   const int cnt = __popc(peers);
   const bool leader = valid && (rank == cnt - 1);
-  const int nwarps = (int)((S + 31) / 32);
-  for (int w = 0; w < nwarps; ++w) {
+  for (int w = 0; w < PERM_THREADS / 32; ++w) {
     if (warp == w && valid) {
       const int pos = hist[e] + rank;
       __syncwarp(vmask);
@@ -402,6 +480,13 @@ __global__ void k_unpermute(const uint16_t* __restrict__ y, const int32_t* __res
 
 using namespace moesq;
 
+// dynamic shared memory above the 48 KB default needs the kernel's opt-in
+template <typename Kernel>
+static cudaError_t allow_dynamic_smem(Kernel kernel, size_t bytes) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  return cudaFuncSetAttribute((const void*)kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
 extern "C" int64_t moesq_padded_rows(int64_t S, int32_t E) {
   if (S < 0 || E <= 0) return 0;
   const int64_t extra = 127 * (int64_t)(S < E ? S : E);  // only nonempty groups pad
@@ -441,9 +526,13 @@ extern "C" moesq_status moesq_permute(const int32_t* topk_ids, int64_t T, int32_
       return MOESQ_ERR_CUDA;
     return MOESQ_OK;
   }
-  if (nchunks == 1) {  // one chunk: everything in one block and one launch
-    if (moesq_launch(k_perm_small, dim3(1), dim3(PERM_THREADS), shm, s, topk_ids, S, k, E, expert_offsets, pad_offsets,
-                     slot_token, token_slot, d_status) != cudaSuccess)
+  const bool table = E <= PERM_TABLE_MAX_E;
+  const size_t shm_table = (size_t)33 * E * sizeof(int32_t);  // run[E] + per-warp counts [32][E]
+  if (S <= PERM_BLOCK_MAX_S) {  // decode-sized: everything in one block and one launch
+    const size_t shm_block = table ? shm_table : shm;
+    if (allow_dynamic_smem(k_perm_block, shm_block) != cudaSuccess) return MOESQ_ERR_CUDA;
+    if (moesq_launch(k_perm_block, dim3(1), dim3(PERM_THREADS), shm_block, s, topk_ids, S, k, E, expert_offsets,
+                     pad_offsets, slot_token, token_slot, d_status) != cudaSuccess)
       return MOESQ_ERR_CUDA;
     return MOESQ_OK;
   }
@@ -454,7 +543,9 @@ extern "C" moesq_status moesq_permute(const int32_t* topk_ids, int64_t T, int32_
   if (moesq_launch(k_perm_scan_rows, dim3((E + PERM_THREADS / 32 - 1) / (PERM_THREADS / 32)), dim3(PERM_THREADS),
                    0, s, counts, nchunks, E, totals) != cudaSuccess)
     return MOESQ_ERR_CUDA;
-  if (moesq_launch(k_perm_scatter_scan, dim3(nchunks), dim3(PERM_THREADS), shm, s, topk_ids, S, k, E,
+  const size_t shm_scatter = table ? shm_table : shm;
+  if (allow_dynamic_smem(k_perm_scatter_scan, shm_scatter) != cudaSuccess) return MOESQ_ERR_CUDA;
+  if (moesq_launch(k_perm_scatter_scan, dim3(nchunks), dim3(PERM_THREADS), shm_scatter, s, topk_ids, S, k, E,
                    (const int32_t*)counts, (const int32_t*)totals, expert_offsets, pad_offsets, slot_token,
                    token_slot) != cudaSuccess)
     return MOESQ_ERR_CUDA;

@@ -46,6 +46,35 @@ def test_permute_bit_exact(cfg_name, T):
     assert int(status.item()) == 0
 
 
+@pytest.mark.parametrize("T,k,E,dist", [
+    (128, 8, 128, "uniform"),    # one block at its largest batch (1024 slots)
+    (128, 8, 512, "uniform"),    # one block, largest table (above the 48 KB default shared memory)
+    (129, 8, 512, "uniform"),    # just past one chunk: three passes, largest table
+    (200, 4, 1024, "uniform"),   # one block, more experts than the table holds: warps take turns
+    (600, 4, 1024, "uniform"),   # three passes, warps take turns
+    (512, 8, 128, "uniform"),    # three passes, table
+    (1024, 8, 384, "uniform"),   # three passes, table above 48 KB
+    (3000, 8, 16, "skew"),       # most slots on one expert: long runs inside every warp
+    (100, 8, 16, "skew"),        # the same in one block
+    (1, 1, 1, "uniform"),
+    (5000, 2, 2, "uniform"),
+])
+def test_permute_bit_exact_sizes(T, k, E, dist):
+    """Stable expert-major order against the oracle's counting sort at the sizes where
+    the kernel changes form (one block or three passes; table or turns)."""
+    rng = np.random.default_rng(T * 1000 + k * 10 + E)
+    ids = rng.integers(0, E, size=(T, k)).astype(np.int32)
+    if dist == "skew":
+        ids[rng.random((T, k)) < 0.9] = 3
+    ref = R.permute(ids, E)
+    eo, po, st, ts, status = gpu_permute(ids, E)
+    assert np.array_equal(eo.cpu().numpy(), ref["expert_offsets"])
+    assert np.array_equal(po.cpu().numpy(), ref["pad_offsets"])
+    assert np.array_equal(st.cpu().numpy()[:T * k], ref["slot_token"])
+    assert np.array_equal(ts.cpu().numpy()[:T * k].reshape(T, k), ref["token_slot"])
+    assert int(status.item()) == 0
+
+
 def test_permute_flags_bad_expert():
     ids = np.array([[0, 1], [2, 9]], np.int32)
     *_, status = gpu_permute(ids, 4)
