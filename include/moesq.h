@@ -18,7 +18,7 @@
  * Conventions common to every call
  *  - Pointers named d_* or documented as "device" are CUDA device pointers; the
  *    caller owns every buffer.  No call allocates, frees or synchronises, except
- *    moesq_moe_forward_host (host buffers, documented there).
+ *    moesq_moe_forward_host (host buffers, internal copy streams; documented there).
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream);
  *    work is enqueued asynchronously on it.
  *  - Row-major, K innermost.  A packed NVFP4 byte holds element 2i in its low
@@ -363,10 +363,19 @@ moesq_status moesq_moe_forward(const moesq_moe_layer* L, const uint16_t* x,
 moesq_status moesq_moe_forward_workspace_size(const moesq_moe_layer* L, int64_t T,
                                               size_t* bytes);
 
-/* Same as moesq_moe_forward with HOST inputs and output: copies x/topk_ids/topk_w
- * host->device into `ws` (which must also hold the forward workspace; see
- * moesq_moe_forward_host_workspace_size), runs the layer, copies out back to the
- * host buffer and synchronises `stream`.  Host buffers should be pinned for speed. */
+/* Same as moesq_moe_forward with HOST inputs and output.  The batch is cut into
+ * token chunks (at least 2048 tokens, at most 8 chunks); for each, x/topk_ids/topk_w
+ * are copied host->device into `ws`, the layer runs on `stream`, and out is copied
+ * back to the host buffer.  The uploads and downloads run on two internal streams of
+ * the current device (created on the first call and kept for the process), ordered
+ * against `stream` by events, so the copies of one chunk overlap the forward of
+ * another.  The copies start after the work already queued on `stream`; the call
+ * returns after everything it queued has completed (it synchronises all three
+ * streams, also on error).  The output equals moesq_moe_forward's bit for bit: a
+ * token's result depends only on its own row and routing.  `ws` holds the forward
+ * workspace of one chunk and one input/output buffer set per chunk, so no upload
+ * waits for an earlier chunk's download (see moesq_moe_forward_host_workspace_size).  Host buffers should be pinned: pageable
+ * ones are copied correctly but without overlap. */
 moesq_status moesq_moe_forward_host(const moesq_moe_layer* L, const uint16_t* h_x,
                                     const int32_t* h_topk_ids, const float* h_topk_w,
                                     int64_t T, uint16_t* h_out, void* ws, size_t ws_bytes,

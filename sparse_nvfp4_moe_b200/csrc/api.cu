@@ -9,6 +9,8 @@
 // MoESQ model card).
 #include "common.cuh"
 
+#include <mutex>
+
 namespace {
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -126,14 +128,70 @@ extern "C" moesq_status moesq_moe_forward(const moesq_moe_layer* L, const uint16
   return moesq_unpermute(y, token_slot, topk_w, T, L->k, L->H, out, stream);
 }
 
+// ------------------------------------------------------------- host forward --
+// The batch is cut into token chunks whose host->device copies, forward and
+// device->host copies overlap: uploads run on one internal stream, the forward on
+// the caller's stream, downloads on a second internal stream, ordered by events.
+// Each token's result depends only on its own row and routing, so the chunked
+// forward equals the whole-batch one bit for bit.
+namespace {
+
+constexpr int64_t HOST_MIN_CHUNK = 2048;   // tokens: smaller chunks cost GEMM efficiency
+constexpr int64_t HOST_MAX_CHUNKS = 8;     // each chunk has its own device buffers
+
+int64_t host_chunk_tokens(int64_t T) {
+  int64_t c = (T + HOST_MAX_CHUNKS - 1) / HOST_MAX_CHUNKS;
+  if (c < HOST_MIN_CHUNK) c = HOST_MIN_CHUNK;
+  return c < T ? c : T;
+}
+
+struct HostBufs {
+  size_t x_bytes, idw_bytes, set_bytes, fw;
+};
+
+moesq_status host_layout(const moesq_moe_layer* L, int64_t T, HostBufs* h) {
+  const int64_t tc = host_chunk_tokens(T);
+  size_t fw = 0;
+  moesq_status st = moesq_moe_forward_workspace_size(L, tc, &fw);
+  if (st != MOESQ_OK) return st;
+  h->fw = align256(fw);
+  h->x_bytes = align256((size_t)tc * L->H * 2);
+  h->idw_bytes = align256((size_t)tc * L->k * 4);
+  h->set_bytes = 2 * h->x_bytes + 2 * h->idw_bytes;  // x, out, ids, weights
+  return MOESQ_OK;
+}
+
+// the two copy streams of each device, created on first use and kept for the process
+std::mutex g_copy_mu;
+cudaStream_t g_copy_streams[64][2] = {};
+
+cudaError_t copy_streams(cudaStream_t* up, cudaStream_t* down) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_copy_mu);
+  for (int i = 0; i < 2; ++i)
+    if (!g_copy_streams[dev][i]) {
+      e = cudaStreamCreateWithFlags(&g_copy_streams[dev][i], cudaStreamNonBlocking);
+      if (e != cudaSuccess) return e;
+    }
+  *up = g_copy_streams[dev][0];
+  *down = g_copy_streams[dev][1];
+  return cudaSuccess;
+}
+
+}  // namespace
+
 extern "C" moesq_status moesq_moe_forward_host_workspace_size(const moesq_moe_layer* L,
                                                               int64_t T, size_t* bytes) {
-  if (!bytes || !L) return MOESQ_ERR_INVALID_ARG;
-  size_t fw = 0;
-  moesq_status st = moesq_moe_forward_workspace_size(L, T, &fw);
+  if (!bytes || !L || T < 0) return MOESQ_ERR_INVALID_ARG;
+  HostBufs h;
+  moesq_status st = host_layout(L, T > 0 ? T : 1, &h);
   if (st != MOESQ_OK) return st;
-  const size_t io = align256((size_t)T * L->H * 2) * 2 + align256((size_t)T * L->k * 4) * 2;
-  *bytes = align256(fw) + io;
+  const int64_t tc = host_chunk_tokens(T > 0 ? T : 1);
+  const int64_t nsets = T > 0 ? (T + tc - 1) / tc : 1;
+  *bytes = h.fw + (size_t)nsets * h.set_bytes;
   return MOESQ_OK;
 }
 
@@ -142,34 +200,70 @@ extern "C" moesq_status moesq_moe_forward_host(const moesq_moe_layer* L, const u
                                                int64_t T, uint16_t* h_out, void* ws,
                                                size_t ws_bytes, int32_t* d_status,
                                                moesq_stream_t stream) {
-  size_t need = 0, fw = 0;
+  size_t need = 0;
   moesq_status st = moesq_moe_forward_host_workspace_size(L, T, &need);
   if (st != MOESQ_OK) return st;
-  moesq_moe_forward_workspace_size(L, T, &fw);
   if (T == 0) return MOESQ_OK;
   MOESQ_REQUIRE(h_x && h_topk_ids && h_topk_w && h_out, MOESQ_ERR_INVALID_ARG);
   MOESQ_REQUIRE(ws && ws_bytes >= need && moesq_aligned16(ws), MOESQ_ERR_WORKSPACE);
-  cudaStream_t s = (cudaStream_t)stream;
+  HostBufs hb;
+  host_layout(L, T, &hb);
+  const int64_t tc = host_chunk_tokens(T);
+  const int64_t nchunks = (T + tc - 1) / tc;  // <= HOST_MAX_CHUNKS, one buffer set each
+  cudaStream_t s = (cudaStream_t)stream, up = nullptr, down = nullptr;
+  if (copy_streams(&up, &down) != cudaSuccess) return MOESQ_ERR_CUDA;
   uint8_t* w = (uint8_t*)ws;
-  size_t o = align256(fw);
-  uint16_t* dx = (uint16_t*)(w + o);
-  o += align256((size_t)T * L->H * 2);
-  uint16_t* dout = (uint16_t*)(w + o);
-  o += align256((size_t)T * L->H * 2);
-  int32_t* dids = (int32_t*)(w + o);
-  o += align256((size_t)T * L->k * 4);
-  float* dw = (float*)(w + o);
-  if (cudaMemcpyAsync(dx, h_x, (size_t)T * L->H * 2, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(dids, h_topk_ids, (size_t)T * L->k * 4, cudaMemcpyHostToDevice, s) !=
-          cudaSuccess ||
-      cudaMemcpyAsync(dw, h_topk_w, (size_t)T * L->k * 4, cudaMemcpyHostToDevice, s) != cudaSuccess)
-    return MOESQ_ERR_CUDA;
-  st = moesq_moe_forward(L, dx, dids, dw, T, dout, ws, fw, d_status, stream);
-  if (st != MOESQ_OK) return st;
-  if (cudaMemcpyAsync(h_out, dout, (size_t)T * L->H * 2, cudaMemcpyDeviceToHost, s) != cudaSuccess)
-    return MOESQ_ERR_CUDA;
-  if (cudaStreamSynchronize(s) != cudaSuccess) return MOESQ_ERR_CUDA;
-  return MOESQ_OK;
+  void* fws = w;
+  // events: [chunk][0] uploaded, [chunk][1] computed; plus the entry point
+  cudaEvent_t ev[HOST_MAX_CHUNKS][2] = {}, start = nullptr;
+  moesq_status ret = MOESQ_OK;
+  auto fail = [&](moesq_status code) {
+    if (ret == MOESQ_OK) ret = code;
+  };
+  if (cudaEventCreateWithFlags(&start, cudaEventDisableTiming) != cudaSuccess) return MOESQ_ERR_CUDA;
+  for (int64_t c = 0; c < nchunks && ret == MOESQ_OK; ++c)
+    for (int j = 0; j < 2; ++j)
+      if (cudaEventCreateWithFlags(&ev[c][j], cudaEventDisableTiming) != cudaSuccess) fail(MOESQ_ERR_CUDA);
+  // the copies start after the work already queued on the caller's stream
+  if (ret == MOESQ_OK && (cudaEventRecord(start, s) != cudaSuccess || cudaStreamWaitEvent(up, start, 0) != cudaSuccess))
+    fail(MOESQ_ERR_CUDA);
+  for (int64_t c = 0; c < nchunks && ret == MOESQ_OK; ++c) {
+    const int64_t t0 = c * tc, n = (T - t0) < tc ? (T - t0) : tc;
+    uint8_t* set = w + hb.fw + (size_t)c * hb.set_bytes;
+    uint16_t* dx = (uint16_t*)set;
+    uint16_t* dout = (uint16_t*)(set + hb.x_bytes);
+    int32_t* dids = (int32_t*)(set + 2 * hb.x_bytes);
+    float* dw = (float*)(set + 2 * hb.x_bytes + hb.idw_bytes);
+    if (cudaMemcpyAsync(dx, h_x + t0 * L->H, (size_t)n * L->H * 2, cudaMemcpyHostToDevice, up) != cudaSuccess ||
+        cudaMemcpyAsync(dids, h_topk_ids + t0 * L->k, (size_t)n * L->k * 4, cudaMemcpyHostToDevice, up) !=
+            cudaSuccess ||
+        cudaMemcpyAsync(dw, h_topk_w + t0 * L->k, (size_t)n * L->k * 4, cudaMemcpyHostToDevice, up) !=
+            cudaSuccess ||
+        cudaEventRecord(ev[c][0], up) != cudaSuccess || cudaStreamWaitEvent(s, ev[c][0], 0) != cudaSuccess) {
+      fail(MOESQ_ERR_CUDA);
+      break;
+    }
+    st = moesq_moe_forward(L, dx, dids, dw, n, dout, fws, hb.fw, d_status, stream);
+    if (st != MOESQ_OK) {
+      fail(st);
+      break;
+    }
+    if (cudaEventRecord(ev[c][1], s) != cudaSuccess || cudaStreamWaitEvent(down, ev[c][1], 0) != cudaSuccess ||
+        cudaMemcpyAsync(h_out + t0 * L->H, dout, (size_t)n * L->H * 2, cudaMemcpyDeviceToHost, down) !=
+            cudaSuccess) {
+      fail(MOESQ_ERR_CUDA);
+      break;
+    }
+  }
+  // whatever was queued completes before the caller's buffers are handed back
+  if (cudaStreamSynchronize(up) != cudaSuccess) fail(MOESQ_ERR_CUDA);
+  if (cudaStreamSynchronize(s) != cudaSuccess) fail(MOESQ_ERR_CUDA);
+  if (cudaStreamSynchronize(down) != cudaSuccess) fail(MOESQ_ERR_CUDA);
+  for (int c = 0; c < HOST_MAX_CHUNKS; ++c)
+    for (int j = 0; j < 2; ++j)
+      if (ev[c][j]) cudaEventDestroy(ev[c][j]);
+  if (start) cudaEventDestroy(start);
+  return ret;
 }
 
 // ----------------------------------------------------------------- self-test --
