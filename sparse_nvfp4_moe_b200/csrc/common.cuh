@@ -91,13 +91,14 @@ __device__ __forceinline__ float rcp_approx(float x) {
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-// silu of two values with packed (f32x2) multiplies and adds: x / (1 + 2^(-x log2 e)),
-// the exponential and the reciprocal on the MUFU (the same arithmetic as silu_fast).
-// Where 1 + e >= 2^126 the reciprocal flushes to 0 and so does silu.
-__device__ __forceinline__ float2 silu2(float2 x) {
-  const float2 t = __fmul2_rn(x, make_float2(-1.4426950408889634f, -1.4426950408889634f));
+// g / (1 + 2^(g * ce)) for two values, with packed (f32x2) multiplies and adds:
+// silu(a g) / a with ce = -a log2 e.  The exponential and the reciprocal run on the
+// MUFU (the same arithmetic as silu_fast); where 1 + 2^(g ce) >= 2^126 the
+// reciprocal flushes to 0 and so does the result.
+__device__ __forceinline__ float2 sigmoid_scaled2(float2 g, float ce) {
+  const float2 t = __fmul2_rn(g, make_float2(ce, ce));
   const float2 d = __fadd2_rn(make_float2(ex2_approx(t.x), ex2_approx(t.y)), make_float2(1.0f, 1.0f));
-  return __fmul2_rn(x, make_float2(rcp_approx(d.x), rcp_approx(d.y)));
+  return __fmul2_rn(g, make_float2(rcp_approx(d.x), rcp_approx(d.y)));
 }
 
 // E4M3 (finite, saturating) code of a nonnegative float32, nearest-even.

@@ -489,19 +489,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // o = 16q + 2j + h of this CTA's 64.  A 16x256b load at lane 32q + 16h thus
         // hands thread t the gate and up values of output 16q + 2(t/4) + h for the
         // columns c_lo + 8i + 2(t%4) + b (i < 4, b < 2): no exchange between warps.
+        // hv holds h / (alpha * alpha_u) for the raw accumulators g and u: silu(alpha g)
+        // = alpha g / (1 + 2^(g * (-alpha log2 e))), so alpha enters the exponent's
+        // multiplier and the product alpha * alpha_u enters the amax and the code
+        // multiplier below (a few ulp of reassociation, no multiply per element)
         float hv[2][8];  // [h][v]: v = 2i + b
+        const float ch = __fmul_rn(alpha, alpha_u);
         if (live) {
           uint32_t r[16];
-          const float2 al2 = make_float2(alpha, alpha), au2 = make_float2(alpha_u, alpha_u);
+          const float ce = __fmul_rn(alpha, -1.4426950408889634f);
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             tmem_ld_16x256b_x4(tbase + ((uint32_t)(16 * h) << 16) + c_lo, r);
             tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 4; ++i) {  // columns b = 0, 1 as one packed pair
-              const float2 g = __fmul2_rn(make_float2(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1])), al2);
-              const float2 u = __fmul2_rn(make_float2(__uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3])), au2);
-              const float2 hh = __fmul2_rn(silu2(g), u);
+              const float2 g = make_float2(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]));
+              const float2 u = make_float2(__uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+              const float2 hh = __fmul2_rn(sigmoid_scaled2(g, ce), u);
               hv[h][2 * i] = hh.x;
               hv[h][2 * i + 1] = hh.y;
             }
@@ -540,8 +545,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           float* xa = epi + (kb * 4 + q) * 32;
           xa[lane] = m[0];
           named_bar_sync(2 + (q >> 1) + 2 * kb, 64);
-          const float amax = fmaxf(m[0], epi[(kb * 4 + (q ^ 1)) * 32 + lane]);
+          const float amax = __fmul_rn(fmaxf(m[0], epi[(kb * 4 + (q ^ 1)) * 32 + lane]), fabsf(ch));
           const GroupScale gs = nvfp4_group_scale(amax, ag.y);
+          // code multiplier of column (lane >> 2) & 7 for the scaled hv, transposed through
+          // shared memory so that each thread reads its 8 columns with two vector loads
+          float* xi = epi + 512 + ew * 32;
+          xi[(lane & 3) * 8 + ((lane >> 2) & 7)] = __fmul_rn(gs.inv, ch);
+          __syncwarp();
+          const float4 iv0 = *reinterpret_cast<const float4*>(xi + (lane & 3) * 8);
+          const float4 iv1 = *reinterpret_cast<const float4*>(xi + (lane & 3) * 8 + 4);
+          const float ivs[8] = {iv0.x, iv0.y, iv0.z, iv0.w, iv1.x, iv1.y, iv1.z, iv1.w};
           const int vc = (lane >> 2) & 7;
           const int rc = 8 * (vc >> 1) + 2 * (lane & 3) + (vc & 1);  // this lane's column (row of the block)
           if ((q & 1) == 0) S.sstg[sb][kb][rc][q >> 1] = (uint8_t)gs.sc;
@@ -549,7 +562,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           uint8_t* stg = &S.hstg[sb][kb][0][8 * q + (lane >> 2)];
 #pragma unroll
           for (int v = 0; v < 8; ++v) {
-            const float inv = __shfl_sync(0xffffffffu, gs.inv, (lane & 3) | (v << 2));
+            const float inv = ivs[v];
             const float2 x = __fmul2_rn(make_float2(hv[0][v], hv[1][v]), make_float2(inv, inv));
             const uint32_t byte = inv == 0.0f ? 0u : e2m1x2(x.x, x.y);
             stg[(8 * (v >> 1) + 2 * (lane & 3) + (v & 1)) * 32] = (uint8_t)byte;
