@@ -74,12 +74,6 @@ __device__ __forceinline__ uint32_t nvfp4_word(const float* v, float inv) {
                 __fmul_rn(v[6], inv), __fmul_rn(v[7], inv));
 }
 
-// silu(x) = x / (1 + exp(-x)) with the fast exponential and division (relative
-// error a few ulp; the denominator exceeds 2^126 only where silu rounds to 0)
-__device__ __forceinline__ float silu_fast(float x) {
-  return __fdividef(x, 1.0f + __expf(-x));
-}
-
 // ex2.approx / rcp.approx (PTX ISA), denormal outputs flushed to zero
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
@@ -93,8 +87,8 @@ __device__ __forceinline__ float rcp_approx(float x) {
 }
 // g / (1 + 2^(g * ce)) for two values, with packed (f32x2) multiplies and adds:
 // silu(a g) / a with ce = -a log2 e.  The exponential and the reciprocal run on the
-// MUFU (the same arithmetic as silu_fast); where 1 + 2^(g ce) >= 2^126 the
-// reciprocal flushes to 0 and so does the result.
+// MUFU (relative error a few ulp); where 1 + 2^(g ce) >= 2^126 the reciprocal
+// flushes to 0 and so does the result.
 __device__ __forceinline__ float2 sigmoid_scaled2(float2 g, float ce) {
   const float2 t = __fmul2_rn(g, make_float2(ce, ce));
   const float2 d = __fadd2_rn(make_float2(ex2_approx(t.x), ex2_approx(t.y)), make_float2(1.0f, 1.0f));

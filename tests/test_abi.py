@@ -83,3 +83,30 @@ def test_size_queries(lib):
     assert _lib.padded_rows(300, 2) == ((300 + 2 * 127 + 127) // 128) * 128
     assert _lib.permute_workspace_size(64, 2, 8) == (1 * 8 + 8) * 4      # chunk counts + expert totals
     assert _lib.quant_weight_workspace_size(8, 2) == 64
+
+
+def test_host_forward_workspace_layout(lib):
+    """The host-buffer forward holds the forward workspace of one token chunk and one
+    input/output buffer set per chunk: chunks of max(2048, ceil(T / 8)) tokens, at most
+    8 of them (host logic only; no GPU needed)."""
+    from sparse_nvfp4_moe_b200 import _lib
+    layer = _lib.MoeLayer()
+    layer.E, layer.k, layer.H, layer.I = 128, 8, 2048, 768
+
+    def a256(x):
+        return (x + 255) // 256 * 256
+
+    def expected(T):
+        tc = min(max(2048, -(-T // 8)), T)
+        n = -(-T // tc)
+        fw = _lib.moe_forward_workspace_size(layer, tc)
+        per_set = 2 * a256(tc * layer.H * 2) + 2 * a256(tc * layer.k * 4)
+        return a256(fw) + n * per_set, n
+
+    for T, chunks in [(1, 1), (2048, 1), (2049, 2), (5000, 3), (16384, 8), (100000, 8)]:
+        want, n = expected(T)
+        assert n == chunks
+        assert _lib.moe_forward_host_workspace_size(layer, T) == want
+    # the forward workspace never shrinks with more tokens (a chunk's is enough for a shorter one)
+    sizes = [_lib.moe_forward_workspace_size(layer, t) for t in (1, 100, 904, 2047, 2048)]
+    assert sizes == sorted(sizes)
