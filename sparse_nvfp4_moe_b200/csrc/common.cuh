@@ -66,12 +66,14 @@ __device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
   return out;
 }
 
-// codes of v[0..7] under a group multiplier (inv == 0: the group is all zeros)
+// codes of v[0..7] under a group multiplier (inv == 0: the group is all zeros); the
+// products in packed f32x2 multiplies, each rounded to nearest like __fmul_rn
 __device__ __forceinline__ uint32_t nvfp4_word(const float* v, float inv) {
   if (inv == 0.0f) return 0u;
-  return e2m1x8(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv), __fmul_rn(v[2], inv),
-                __fmul_rn(v[3], inv), __fmul_rn(v[4], inv), __fmul_rn(v[5], inv),
-                __fmul_rn(v[6], inv), __fmul_rn(v[7], inv));
+  const float2 m = make_float2(inv, inv);
+  const float2 a = __fmul2_rn(make_float2(v[0], v[1]), m), b = __fmul2_rn(make_float2(v[2], v[3]), m);
+  const float2 c = __fmul2_rn(make_float2(v[4], v[5]), m), d = __fmul2_rn(make_float2(v[6], v[7]), m);
+  return e2m1x8(a.x, a.y, b.x, b.y, c.x, c.y, d.x, d.y);
 }
 
 // ex2.approx / rcp.approx (PTX ISA), denormal outputs flushed to zero
