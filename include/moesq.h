@@ -280,7 +280,13 @@ typedef enum moesq_epilogue {
   MOESQ_EPI_BF16 = 1,        /* out bf16 [S, W.out] */
   MOESQ_EPI_SWIGLU_NVFP4 = 2 /* gate_up only: h = silu(gate)*up requantised with g_next[e]:
                                 out u8 codes [P, I/2] (padded rows), out_sf blocks
-                                [P/128][I/128][512] -- the next GEMM's B operand */
+                                [P/128][I/128][512] -- the next GEMM's B operand.
+                                h is fp32 (exponential and reciprocal of the SiLU on
+                                the MUFU, a few ulp); the NVFP4 rule runs on h with
+                                the accumulator scales folded into its amax and code
+                                multiplier, so it matches the rule on the exact h
+                                except where h lies within that error of a rounding
+                                boundary */
 } moesq_epilogue;
 
 /* y[s, m] = g_act[e] * alpha_w[e] * sum_k W_e[m, k] * A[s, k] for every slot s of expert e.
