@@ -65,6 +65,33 @@ def weight_int(storage) -> np.ndarray:
     return dequant_int(unpack_codes(dense), storage["scale"])
 
 
+def int_matmul_exact(a, w) -> np.ndarray:
+    """a @ w.T for int64 a [n, K] and w [m, K], exactly, by float64 matrix products.
+
+    The quantised operands are integers below 2**22 in magnitude (units of 2**-10:
+    at most 12 halves times 448 * 512).  Writing a = hi * 2**11 + lo with
+    0 <= lo < 2**11 makes both |hi| and |lo| at most 2**11, so every product with
+    w is an integer below 2**33 and every partial sum over K < 2**19 terms an
+    integer below 2**52: float64 represents all of them, and the float64 products
+    are exact whatever order the library sums in.  The operand ranges are
+    checked; outside them the plain int64 product is used.
+    """
+    a = np.asarray(a, dtype=np.int64)
+    w = np.asarray(w, dtype=np.int64)
+    K = a.shape[1]
+    if a.size == 0 or w.size == 0:
+        return np.zeros((a.shape[0], w.shape[0]), dtype=np.int64)
+    wmax = int(np.abs(w).max())
+    if int(np.abs(a).max()) >= 2 ** 22 or wmax * (2 ** 11) * K >= 2 ** 52:
+        return a @ w.T
+    hi = a >> 11
+    lo = a - (hi << 11)
+    wf = w.astype(np.float64).T
+    r_hi = hi.astype(np.float64) @ wf
+    r_lo = lo.astype(np.float64) @ wf
+    return (r_hi.astype(np.int64) << 11) + r_lo.astype(np.int64)
+
+
 def grouped_gemm_exact(W_int, g_w, A_int, g_act, expert_offsets):
     """Exact grouped GEMM.
 
@@ -85,8 +112,8 @@ def grouped_gemm_exact(W_int, g_w, A_int, g_act, expert_offsets):
             continue
         a = A_int[s0:s1]
         w = W_int[e]
-        acc = a @ w.T                                   # int64, exact
-        aab = np.abs(a) @ np.abs(w).T
+        acc = int_matmul_exact(a, w)                    # exact
+        aab = int_matmul_exact(np.abs(a), np.abs(w))
         scale = float(np.float64(g_act[e]) * np.float64(g_w[e])) * 2.0 ** -20
         y[s0:s1] = acc.astype(np.float64) * scale
         bound[s0:s1] = aab.astype(np.float64) * abs(scale)

@@ -197,3 +197,20 @@ def test_fold_is_exact_for_a_power_of_two_ratio():
     a, _ = G.gate_up_exact([st], A, g_in, off, fold=True)
     b, _ = G.gate_up_exact([st], A, g_in, off, fold=False)
     assert np.array_equal(a, b)
+
+
+def test_int_matmul_exact_equals_int64_product():
+    """The float64 route of the exact GEMM equals the int64 product (its definition),
+    including operands at the largest quantised magnitude (12 * 448 * 512) and the
+    deepest K of the layer shapes, where every term has the same sign."""
+    rng = np.random.default_rng(31)
+    top = 12 * 448 * 512
+    for n, m, K in ((7, 5, 64), (33, 17, 7168), (3, 4, 4096)):
+        a = rng.integers(-top, top + 1, (n, K), dtype=np.int64)
+        w = rng.integers(-top, top + 1, (m, K), dtype=np.int64)
+        assert np.array_equal(G.int_matmul_exact(a, w), a @ w.T)
+    a = np.full((2, 7168), top, np.int64)
+    w = np.full((3, 7168), -top, np.int64)
+    w[1] = top
+    assert np.array_equal(G.int_matmul_exact(a, w), a @ w.T)
+    assert G.int_matmul_exact(np.zeros((0, 8), np.int64), np.ones((2, 8), np.int64)).shape == (0, 2)
