@@ -27,6 +27,24 @@ def test_nvfp4_groups_golden(golden):
         assert codes[0].tolist() == grp["codes"], grp["name"]
 
 
+def test_reciprocal_multiply_reading_differs_from_division(golden):
+    """The rule multiplies by fp32(1/sdq) (reading R4 of the rounding rule); the golden
+    group 'reciprocal_multiply_not_division' is worked by hand so that dividing by sdq
+    instead gives other codes.  Recompute its key elements with exact rationals."""
+    from fractions import Fraction
+    grp = next(g for g in golden("nvfp4_groups.json")["groups"] if g["name"] == "reciprocal_multiply_not_division")
+    assert grp["codes"] != grp["codes_if_division"]
+    sdq = Fraction(15, 4)                                        # E4M3 0x47 = 2 * 1.875
+    assert F.e4m3_decode(np.uint8(grp["scale"])) == float(sdq)
+    inv = Fraction(float(np.float32(1) / np.float32(3.75)))
+    assert inv == Fraction(8947849, 2 ** 25)                     # 1/3.75 rounded up to fp32
+    for xv, c_mul, c_div in zip(grp["x"], grp["codes"], grp["codes_if_division"]):
+        q = Fraction(xv) / sdq                                   # exact quotient
+        p_ = float(np.float32(float(Fraction(xv) * inv)))        # fp32 product, one rounding
+        assert int(F.e2m1_quantize(np.array([p_], np.float32))[0]) == c_mul
+        assert int(F.e2m1_quantize(np.array([float(q)], np.float32))[0]) == c_div
+
+
 def test_nvfp4_dequant_error_bound():
     """Unsaturated groups: every element lands within half an E2M1 step of x."""
     rng = np.random.default_rng(5)
