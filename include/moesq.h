@@ -309,6 +309,21 @@ moesq_status moesq_grouped_gemm(const moesq_linear* W, const uint8_t* act_codes,
                                 int32_t* d_status, moesq_stream_t stream);
 moesq_status moesq_grouped_gemm_workspace_size(const moesq_linear* W, int64_t S, size_t* bytes);
 
+/* Launch shape of the grouped GEMMs (the pages have no counterpart; these calls
+ * exist so that tests can make every CTA pair run several work items).  A
+ * grouped GEMM launches one persistent CTA pair per two SMs that the device
+ * holds at once, and each pair walks the (expert, token tile, weight-tile pair)
+ * work items pid, pid + npairs, ...
+ *   moesq_set_gemm_pair_limit: caps npairs for every later launch in the process
+ *     (0 = no cap, the default).  The result of a GEMM does not depend on npairs.
+ *     Launches already queued keep the npairs they were launched with;
+ *     max_pairs >= 0.
+ *   moesq_gemm_launch_pairs: npairs that a launch on the current device would use
+ *     now (cap applied), for the sparse (dense = 0) or the dense comparison kernel
+ *     with the given epilogue. */
+moesq_status moesq_set_gemm_pair_limit(int32_t max_pairs);
+moesq_status moesq_gemm_launch_pairs(int32_t dense, int32_t epilogue, int32_t* pairs);
+
 /* Dense comparison GEMM: the same grouped GEMM, epilogues and argument meanings on
  * dense NVFP4 weights, the pages' alternative storage ("--no-sparse-storage writes
  * dense packed NVFP4 with the pruned elements zeroed", Usage of the MoESQ repository

@@ -62,6 +62,8 @@ _SIGS = {
     "moesq_grouped_gemm_dense": (ctypes.c_int, [ctypes.POINTER(Linear), c_vp, c_vp, c_vp, c_vp, c_vp, c_i64,
                                                 c_i64, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp]),
     "moesq_sf_expand_block16": (ctypes.c_int, [c_vp, c_vp, c_i64, c_vp]),
+    "moesq_set_gemm_pair_limit": (ctypes.c_int, [c_i32]),
+    "moesq_gemm_launch_pairs": (ctypes.c_int, [c_i32, c_i32, ctypes.POINTER(c_i32)]),
     "moesq_selftest_wait_timeout": (ctypes.c_int, [c_vp, c_i64, c_vp, c_vp]),
     "moesq_gather_act": (ctypes.c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp]),
     "moesq_grouped_gemm_workspace_size": (ctypes.c_int, [ctypes.POINTER(Linear), c_i64,
@@ -262,3 +264,14 @@ def moesq_moe_forward_host(layer: MoeLayer, h_x, h_topk_ids, h_topk_w, T, h_out,
     _check("moesq_moe_forward_host", lib().moesq_moe_forward_host(
         ctypes.byref(layer), _p(h_x), _p(h_topk_ids), _p(h_topk_w), T, _p(h_out), _p(ws), ws_bytes,
         _p(d_status), _stream(stream)))
+
+
+def moesq_set_gemm_pair_limit(max_pairs):
+    _check("moesq_set_gemm_pair_limit", lib().moesq_set_gemm_pair_limit(max_pairs))
+
+
+def moesq_gemm_launch_pairs(dense, epilogue):
+    """CTA pairs the next grouped-GEMM launch on the current device would use."""
+    n = c_i32(0)
+    _check("moesq_gemm_launch_pairs", lib().moesq_gemm_launch_pairs(dense, epilogue, ctypes.byref(n)))
+    return n.value

@@ -38,6 +38,7 @@
 // MOESQ_DFLAG_TIMEOUT, drains its own copies in flight, frees TMEM and exits.
 #include "common.cuh"
 
+#include <atomic>
 #include <mutex>
 
 namespace moesq {
@@ -798,6 +799,41 @@ extern "C" moesq_status moesq_grouped_gemm_workspace_size(const moesq_linear* W,
   return MOESQ_OK;
 }
 
+// Upper bound on the CTA pairs a grouped GEMM launches (0: none), process-wide.
+static std::atomic<int> g_pair_limit{0};
+
+// CTA pairs of a launch: clusters of 2 CTAs, one CTA per SM, as many pairs as the
+// device can hold at once (cached per device and epilogue), capped by g_pair_limit.
+template <bool DENSE>
+static moesq_status launch_pairs(int dev, int sms, int32_t epilogue, int* pairs_out) {
+  constexpr size_t smem = sp::smem_bytes<DENSE>();
+  static int pairs_cache[64][3] = {{0}};
+  const int ei = epilogue - MOESQ_EPI_F32;
+  int pairs = dev < 64 ? pairs_cache[dev][ei] : 0;
+  if (pairs == 0) {
+    const void* fn = epilogue == MOESQ_EPI_F32 ? (const void*)sp::k_grouped_gemm_sp<MOESQ_EPI_F32, DENSE>
+                     : epilogue == MOESQ_EPI_BF16 ? (const void*)sp::k_grouped_gemm_sp<MOESQ_EPI_BF16, DENSE>
+                                                  : (const void*)sp::k_grouped_gemm_sp<MOESQ_EPI_SWIGLU_NVFP4, DENSE>;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return MOESQ_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(sms & ~1));
+    cfg.blockDim = dim3(sp::THREADS);
+    cfg.dynamicSmemBytes = smem;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess || n < 1) {
+      (void)cudaGetLastError();
+      return MOESQ_ERR_CUDA;
+    }
+    pairs = n < sms / 2 ? n : sms / 2;
+    if (dev < 64) pairs_cache[dev][ei] = pairs;
+  }
+  const int lim = g_pair_limit.load(std::memory_order_relaxed);
+  if (lim > 0 && lim < pairs) pairs = lim;
+  *pairs_out = pairs;
+  return MOESQ_OK;
+}
+
 // Both grouped GEMMs: DENSE = false is the paired-4:8 sparse kernel (W->packed are
 // the kept bytes, W->meta the sparse metadata); DENSE = true is the comparison
 // kernel on decoded weights (W->packed dense codes [E, out, K/2], no metadata, W->sf
@@ -908,29 +944,10 @@ static moesq_status grouped_gemm_impl(const moesq_linear* W, const uint8_t* act_
       return MOESQ_ERR_CUDA;
   }
 
-  // clusters of 2 CTAs, one CTA per SM: as many pairs as the device can hold at once
   constexpr size_t smem = sp::smem_bytes<DENSE>();
-  static int pairs_cache[64][3] = {{0}};
-  const int ei = epilogue - MOESQ_EPI_F32;
-  int pairs = dev < 64 ? pairs_cache[dev][ei] : 0;
-  if (pairs == 0) {
-    const void* fn = epilogue == MOESQ_EPI_F32 ? (const void*)sp::k_grouped_gemm_sp<MOESQ_EPI_F32, DENSE>
-                     : epilogue == MOESQ_EPI_BF16 ? (const void*)sp::k_grouped_gemm_sp<MOESQ_EPI_BF16, DENSE>
-                                                  : (const void*)sp::k_grouped_gemm_sp<MOESQ_EPI_SWIGLU_NVFP4, DENSE>;
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return MOESQ_ERR_CUDA;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(sms & ~1));
-    cfg.blockDim = dim3(sp::THREADS);
-    cfg.dynamicSmemBytes = smem;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess || n < 1) {
-      (void)cudaGetLastError();
-      return MOESQ_ERR_CUDA;
-    }
-    pairs = n < sms / 2 ? n : sms / 2;
-    if (dev < 64) pairs_cache[dev][ei] = pairs;
-  }
+  int pairs = 0;
+  const moesq_status pst = launch_pairs<DENSE>(dev, sms, epilogue, &pairs);
+  if (pst != MOESQ_OK) return pst;
   sp::Params prm;
   prm.meta = W->meta;
   prm.sfw = W->sf;
@@ -995,4 +1012,23 @@ extern "C" moesq_status moesq_grouped_gemm_dense(const moesq_linear* W, const ui
                                                  int32_t* d_status, moesq_stream_t stream) {
   return grouped_gemm_impl<true>(W, act_codes, act_sf, g_act, expert_offsets, pad_offsets, S, P_cap, epilogue,
                                  g_next, out, out_sf, d_status, stream);
+}
+
+extern "C" moesq_status moesq_set_gemm_pair_limit(int32_t max_pairs) {
+  MOESQ_REQUIRE(max_pairs >= 0, MOESQ_ERR_INVALID_ARG);
+  g_pair_limit.store(max_pairs, std::memory_order_relaxed);
+  return MOESQ_OK;
+}
+
+extern "C" moesq_status moesq_gemm_launch_pairs(int32_t dense, int32_t epilogue, int32_t* pairs) {
+  MOESQ_REQUIRE(pairs && epilogue >= MOESQ_EPI_F32 && epilogue <= MOESQ_EPI_SWIGLU_NVFP4, MOESQ_ERR_INVALID_ARG);
+  int dev = 0;
+  const int sms = device_sms(&dev);
+  if (sms < 0) return MOESQ_ERR_CUDA;
+  if (sms == 0) return MOESQ_ERR_DEVICE;
+  int n = 0;
+  const moesq_status st =
+      dense ? launch_pairs<true>(dev, sms, epilogue, &n) : launch_pairs<false>(dev, sms, epilogue, &n);
+  if (st == MOESQ_OK) *pairs = n;
+  return st;
 }

@@ -1,0 +1,152 @@
+"""GPU parity of the grouped GEMMs when every CTA pair runs several work items.
+
+The grouped GEMM is persistent: pair pid of npairs walks the (expert, token tile,
+weight-tile pair) items pid, pid + npairs, ... and alternates two TMEM accumulator
+buffers, so from its second item on a pair uses the second buffer, the accumulator
+phase flips, the expert record it loaded a tile ahead and the (tile, pair) stride
+walk.  The other GEMM tests have fewer items than the device has pairs, so here:
+
+* the layers of tests/test_gpu_gemm.py run with the launch capped at 1, 2 and 3 pairs
+  (moesq_set_gemm_pair_limit), so one pair runs every item or the stride walk wraps
+  over weight-tile pairs with a remainder; every output element is compared with the
+  oracle (FP32 and bf16 gate_up, SwiGLU + requant, bf16 down, the dense comparison
+  kernel);
+* a layer whose item list is many times the device's own pair count (32 experts,
+  top-4, H = 512, I = 256, 8192 tokens: 512 items per GEMM) runs at the uncapped
+  launch, and the whole layer is compared element by element.
+
+Tolerances are those of tests/test_gpu_gemm.py (1e-5 * sum|a w| in FP32, one bf16 ulp
+beyond it; requantised codes bit-exact where the NVFP4 rule fixes them).  The grouped
+GEMM is the kernel line of the Qwen3.5-397B-A17B-P48NVFP4-MoESQ model card.
+"""
+import numpy as np
+import pytest
+import torch
+
+import sparse_nvfp4_moe_b200 as M
+import workloads as W
+from tests import test_gpu_dense as TD
+from tests import test_gpu_gemm as TG
+
+pytestmark = pytest.mark.gpu
+
+LIMITS = (1, 2, 3)
+CAPPED = ("tiny", "ragged_multi_tile", "sparse_routing", "mid_ktail", "deep_k", "exact_per_half_alpha")
+MANY = W.LayerConfig("many_items", 46, 32, 4, 512, 256, (8192,), "uniform", True)
+
+
+def items(layer, out_rows):
+    """Work items of one grouped GEMM: token tiles of 128 times weight-tile pairs."""
+    counts = np.diff(layer.perm["expert_offsets"])
+    mt = out_rows // 128
+    return int(((counts + 127) // 128).sum()) * ((mt + 1) // 2)
+
+
+class PairLimit:
+    def __init__(self, n):
+        self.n = n
+
+    def __enter__(self):
+        M.moesq_set_gemm_pair_limit(self.n)
+        return self
+
+    def __exit__(self, *a):
+        M.moesq_set_gemm_pair_limit(0)
+
+
+@pytest.fixture(scope="module", params=CAPPED)
+def capped_layer(request):
+    cfg, T, *opt = TG.CASES[request.param]
+    return TG.Layer(cfg, T, **(opt[0] if opt else {}))
+
+
+@pytest.mark.parametrize("limit", LIMITS)
+def test_capped_pairs_gate_up_f32(capped_layer, limit):
+    with PairLimit(limit):
+        assert M.moesq_gemm_launch_pairs(0, M.EPI_F32) == limit
+        TG.test_gate_up_f32_within_tolerance(capped_layer)
+
+
+@pytest.mark.parametrize("limit", LIMITS)
+def test_capped_pairs_gate_up_bf16(capped_layer, limit):
+    with PairLimit(limit):
+        TG.test_gate_up_bf16_within_tolerance(capped_layer)
+
+
+@pytest.mark.parametrize("limit", LIMITS)
+def test_capped_pairs_swiglu_requant(capped_layer, limit):
+    with PairLimit(limit):
+        TG.test_swiglu_requant_epilogue(capped_layer)
+
+
+@pytest.mark.parametrize("limit", LIMITS)
+def test_capped_pairs_down_bf16(capped_layer, limit):
+    with PairLimit(limit):
+        TG.test_down_bf16_within_tolerance(capped_layer)
+
+
+@pytest.mark.parametrize("limit", (1, 3))
+def test_capped_pairs_forward(capped_layer, limit):
+    with PairLimit(limit):
+        TG.test_moe_forward_end_to_end(capped_layer)
+
+
+@pytest.fixture(scope="module")
+def dense_layer():
+    cfg, T, *opt = TG.CASES["ragged_multi_tile"]
+    L = TG.Layer(cfg, T, **(opt[0] if opt else {}))
+    L.dense_gu = TD.DenseLinear(L.gu, L.dgu)
+    L.dense_dn = TD.DenseLinear(L.dn, L.ddn)
+    return L
+
+
+@pytest.mark.parametrize("limit", (1, 3))
+def test_capped_pairs_dense_comparison(dense_layer, limit):
+    """The dense comparison kernel on one and on three pairs, against the same oracle."""
+    with PairLimit(limit):
+        assert M.moesq_gemm_launch_pairs(1, M.EPI_F32) == limit
+        TD.test_dense_gate_up_f32_within_tolerance(dense_layer)
+        TD.test_dense_swiglu_requant_epilogue(dense_layer)
+        TD.test_dense_down_bf16_within_tolerance(dense_layer)
+
+
+@pytest.fixture(scope="module")
+def many_layer():
+    M.moesq_set_gemm_pair_limit(0)
+    L = TG.Layer(MANY, 8192)
+    pairs = max(M.moesq_gemm_launch_pairs(0, e) for e in (M.EPI_F32, M.EPI_BF16, M.EPI_SWIGLU_NVFP4))
+    n_gu, n_dn = items(L, 2 * MANY.I), items(L, MANY.H)
+    # every pair of the uncapped launch runs at least two items of each GEMM
+    assert n_gu >= 2 * pairs and n_dn >= 2 * pairs, (n_gu, n_dn, pairs)
+    return L
+
+
+def test_many_items_gate_up_f32(many_layer):
+    TG.test_gate_up_f32_within_tolerance(many_layer)
+
+
+def test_many_items_gate_up_bf16(many_layer):
+    TG.test_gate_up_bf16_within_tolerance(many_layer)
+
+
+def test_many_items_swiglu_requant(many_layer):
+    TG.test_swiglu_requant_epilogue(many_layer)
+
+
+def test_many_items_down_bf16(many_layer):
+    TG.test_down_bf16_within_tolerance(many_layer)
+
+
+def test_many_items_forward(many_layer):
+    TG.test_moe_forward_end_to_end(many_layer)
+    TG.test_forward_is_deterministic(many_layer)
+
+
+def test_pair_limit_arguments():
+    with pytest.raises(M.MoesqError):
+        M.moesq_set_gemm_pair_limit(-1)
+    full = M.moesq_gemm_launch_pairs(0, M.EPI_BF16)
+    assert full >= 1
+    with PairLimit(full + 100):
+        assert M.moesq_gemm_launch_pairs(0, M.EPI_BF16) == full
+    torch.cuda.synchronize()
