@@ -12,8 +12,23 @@ and the quantization config carries "paired48_sparse": {"layout": "pair-bitmask"
 "version": 1}.  The card gives no tensor names beyond these suffixes, so the caller
 names each linear with a template (default: Hugging Face MoE names,
 "{prefix}.experts.{e}.{proj}"), and it does not say whether a stored global is the
-multiplier the dequantisation applies or its reciprocal, so the caller says which
-(``global_convention``).
+multiplier the dequantisation applies or its reciprocal.  The card does say the
+checkpoints are in the compressed-tensors NVFP4 ("nvfp4-pack-quantized") form,
+whose published convention stores the reciprocal, 6 * 448 / amax; the library works
+with the multiplier, amax / (6 * 448).  The reader therefore decides from the
+stored numbers (``global_convention="auto"``, the default) and refuses a reading
+that the numbers contradict:
+
+    read as a multiplier g, a block scale s dequantises to at most 6 * s * g, so the
+    largest weight the stored tensor can hold is A_m = 6 * s_max * g; read as a
+    reciprocal it is A_r = 6 * s_max / g.  A_m * A_r = (6 * s_max)**2, so exactly one
+    of them is below 6 * s_max (2688 when a block reaches the E4M3 maximum 448) unless
+    g == 1: a weight tensor whose largest element is thousands of times its own
+    quantisation range does not exist, so that one is the reading.
+
+An explicit ``global_convention`` ("multiplier" or "reciprocal") is checked the same
+way and raises CheckpointError when the stored numbers say otherwise.  The input
+global of a linear follows the convention of its weight global.
 
 The safetensors container is parsed here directly (8-byte little-endian header
 length, JSON header of name -> dtype, shape, data offsets; raw data after it); a
@@ -132,12 +147,29 @@ def _scalar(a: np.ndarray, name: str) -> np.float32:
     return a[0]
 
 
-def read_linear(ckpt: Checkpoint, name: str, global_convention: str = "multiplier") -> dict:
+CONVENTIONS = ("auto", "multiplier", "reciprocal")
+
+
+def stored_convention(g: np.float32, scale_codes: np.ndarray):
+    """'multiplier' or 'reciprocal': the reading of a stored weight global under which
+    the largest weight the tensor can hold (6 * largest block scale * multiplier) stays
+    below 6 * largest block scale; None when the numbers cannot tell (g == 1, no
+    nonzero block scale, or a global that is not finite and positive)."""
+    s_max = float(torch.from_numpy(np.ascontiguousarray(scale_codes)).view(torch.float8_e4m3fn).float()
+                  .nan_to_num(0.0).abs().max()) if scale_codes.size else 0.0
+    g = float(g)
+    if not (np.isfinite(g) and g > 0) or s_max == 0.0 or g == 1.0:
+        return None
+    a_mult, a_recip = 6.0 * s_max * g, 6.0 * s_max / g
+    return "multiplier" if a_mult < a_recip else "reciprocal"
+
+
+def read_linear(ckpt: Checkpoint, name: str, global_convention: str = "auto") -> dict:
     """One expert linear -> dict(packed [out,K/4] u8, mask [out,K/16] u8, scale [out,K/32]
     u8 (E4M3 codes), g (weight global multiplier, float32), g_in (activation global
-    multiplier, float32))."""
-    if global_convention not in ("multiplier", "reciprocal"):
-        raise ValueError("global_convention is 'multiplier' or 'reciprocal'")
+    multiplier, float32), convention (how the file stored them))."""
+    if global_convention not in CONVENTIONS:
+        raise ValueError(f"global_convention is one of {CONVENTIONS}")
     packed = ckpt.get(f"{name}.weight_sparse_packed")
     mask = ckpt.get(f"{name}.weight_sparse_mask")
     scale = ckpt.get(f"{name}.weight_scale")
@@ -150,13 +182,27 @@ def read_linear(ckpt: Checkpoint, name: str, global_convention: str = "multiplie
                               f"do not describe one [out, K] paired-4:8 NVFP4 weight")
     g = _scalar(ckpt.get(f"{name}.weight_global_scale"), f"{name}.weight_global_scale")
     g_in = _scalar(ckpt.get(f"{name}.input_global_scale"), f"{name}.input_global_scale")
-    if global_convention == "reciprocal":
+    seen = stored_convention(g, scale)
+    conv = global_convention
+    if conv == "auto":
+        if seen is None:
+            fmt = str(ckpt.config.get("quantization_config", {}).get("format", ""))
+            if fmt != "nvfp4-pack-quantized":
+                raise CheckpointError(f"{name}: cannot tell whether the stored global {float(g)!r} is a multiplier "
+                                      f"or its reciprocal; pass global_convention")
+            seen = "reciprocal"        # the compressed-tensors NVFP4 convention
+        conv = seen
+    elif seen is not None and seen != conv:
+        raise CheckpointError(f"{name}: the stored global {float(g)!r} with block scales up to the stored maximum "
+                              f"is a {seen}, not a {conv}")
+    if conv == "reciprocal":
         g, g_in = np.float32(1) / g, np.float32(1) / g_in
-    return dict(packed=packed, mask=mask, scale=scale, g=np.float32(g), g_in=np.float32(g_in), out=out, K=K)
+    return dict(packed=packed, mask=mask, scale=scale, g=np.float32(g), g_in=np.float32(g_in), out=out, K=K,
+                convention=conv)
 
 
 def read_moe_experts(ckpt: Checkpoint, prefix: str, E: int, template: str = "{prefix}.experts.{e}.{proj}",
-                     projs=("gate_proj", "up_proj", "down_proj"), global_convention: str = "multiplier",
+                     projs=("gate_proj", "up_proj", "down_proj"), global_convention: str = "auto",
                      check_marker: bool = True) -> dict:
     """All routed experts of one MoE layer, in the library's storage form.
 
@@ -165,13 +211,14 @@ def read_moe_experts(ckpt: Checkpoint, prefix: str, E: int, template: str = "{pr
                  g_in_gate_up [E], g_in_down [E]) as host tensors; the fused gate_up
     stacks the gate rows above the up rows.  The activation global of gate_up is the
     one stored with gate_proj, and up_proj's must equal it (both quantise the same
-    input)."""
+    input).  Every linear of the layer must have stored its globals the same way."""
     if check_marker:
         ckpt.check_marker()
     gate, up, down = projs
     gu_p, gu_m, gu_s, gu_g, g_in_gu = [], [], [], [], []
     dn_p, dn_m, dn_s, dn_g, g_in_dn = [], [], [], [], []
     shapes = None
+    first_conv = None
     for e in range(E):
         lg = read_linear(ckpt, template.format(prefix=prefix, e=e, proj=gate), global_convention)
         lu = read_linear(ckpt, template.format(prefix=prefix, e=e, proj=up), global_convention)
@@ -184,6 +231,10 @@ def read_moe_experts(ckpt: Checkpoint, prefix: str, E: int, template: str = "{pr
             shapes = sh
         elif sh != shapes:
             raise CheckpointError(f"expert {e}: shape {sh} differs from expert 0's {shapes}")
+        convs = {lg["convention"], lu["convention"], ld["convention"]}
+        if len(convs) > 1 or (e > 0 and convs != {first_conv}):
+            raise CheckpointError(f"expert {e}: globals stored in mixed conventions {sorted(convs)}")
+        first_conv = lg["convention"]
         if lg["g_in"] != lu["g_in"]:
             raise CheckpointError(f"expert {e}: gate and up input globals differ ({lg['g_in']} vs {lu['g_in']})")
         gu_p.append(np.concatenate([lg["packed"], lu["packed"]]))

@@ -39,7 +39,9 @@ def _linear_tensors(name, packed, mask, scale, g, g_in, reciprocal):
             f"{name}.input_global_scale": torch.tensor([gi])}
 
 
-def write_checkpoint(d, reciprocal=False, marker=None):
+def write_checkpoint(d, reciprocal=True, marker=None, fmt="nvfp4-pack-quantized"):
+    """One MoE layer in paired48 storage.  By default the globals are stored the way the
+    compressed-tensors NVFP4 format stores them, as reciprocals (6 * 448 / amax)."""
     st_gu, st_dn, g_in, g_in_dn = _experts()
     I = CFG.I
     shards = [{}, {}]
@@ -61,14 +63,15 @@ def write_checkpoint(d, reciprocal=False, marker=None):
         save_file(sh, os.path.join(d, fn), metadata={"format": "pt"})
         wm.update({n: fn for n in sh})
     json.dump({"metadata": {}, "weight_map": wm}, open(os.path.join(d, "model.safetensors.index.json"), "w"))
-    qc = {"format": "nvfp4-pack-quantized",
+    qc = {"format": fmt,
           "paired48_sparse": marker if marker is not None else {"layout": "pair-bitmask", "version": 1}}
     json.dump({"quantization_config": qc}, open(os.path.join(d, "config.json"), "w"))
     return st_gu, st_dn, g_in, g_in_dn
 
 
 def test_read_back_bit_exact(tmp_path):
-    st_gu, st_dn, g_in, g_in_dn = write_checkpoint(str(tmp_path))
+    """Globals stored as multipliers (the library's own convention) read back bit for bit."""
+    st_gu, st_dn, g_in, g_in_dn = write_checkpoint(str(tmp_path), reciprocal=False, fmt="")
     r = C.read_moe_experts(C.Checkpoint(str(tmp_path)), PREFIX, CFG.E)
     gu, dn = r["gate_up"], r["down"]
     assert (gu["E"], gu["out"], gu["K"]) == (CFG.E, 2 * CFG.I, CFG.H)
@@ -85,11 +88,46 @@ def test_read_back_bit_exact(tmp_path):
 
 def test_reciprocal_convention(tmp_path):
     st_gu, _, g_in, _ = write_checkpoint(str(tmp_path), reciprocal=True)
-    r = C.read_moe_experts(C.Checkpoint(str(tmp_path)), PREFIX, CFG.E, global_convention="reciprocal")
+    for conv in ("auto", "reciprocal"):
+        r = C.read_moe_experts(C.Checkpoint(str(tmp_path)), PREFIX, CFG.E, global_convention=conv)
+        for e in range(CFG.E):
+            stored = np.float32(1) / np.float32(st_gu[e]["g"][0])
+            assert r["gate_up"]["g_w"][e, 0].item() == np.float32(np.float32(1) / stored)
+        assert r["g_in_gate_up"][0].item() == np.float32(np.float32(1) / (np.float32(1) / g_in[0]))
+
+
+def test_compressed_tensors_globals_decode_to_the_weights(tmp_path):
+    """A tensor written as compressed-tensors writes it (global = 6 * 448 / amax, the
+    reciprocal) decodes, under the default reading, to the same weights as the
+    multiplier-form storage it came from: E2M1 x E4M3 x multiplier, elementwise."""
+    from oracle import formats as F
+    from oracle import nvfp4 as N
+    st_gu, st_dn, _, _ = write_checkpoint(str(tmp_path), reciprocal=True)
+    r = C.read_moe_experts(C.Checkpoint(str(tmp_path)), PREFIX, CFG.E)
     for e in range(CFG.E):
-        stored = np.float32(1) / np.float32(st_gu[e]["g"][0])
-        assert r["gate_up"]["g_w"][e, 0].item() == np.float32(np.float32(1) / stored)
-    assert r["g_in_gate_up"][0].item() == np.float32(np.float32(1) / (np.float32(1) / g_in[0]))
+        st = st_dn[e]
+        want = F.e2m1_decode(N.unpack_codes(S.decode(st["packed"], st["mask"])))
+        want = want * np.repeat(F.e4m3_decode(st["scale"]), 32, axis=1) * np.float64(np.float32(st["g"][0]))
+        d = r["down"]
+        got = F.e2m1_decode(N.unpack_codes(S.decode(d["packed"][e].numpy(), d["mask"][e].numpy())))
+        got = got * np.repeat(F.e4m3_decode(d["scale"][e].numpy()), 32, axis=1) * np.float64(d["g_w"][e, 0].item())
+        assert np.allclose(got, want, rtol=2 ** -22, atol=0)
+        assert np.abs(want).max() < 1.0                    # weights of N(0, 0.02), not amax**2 / 2688**2 off
+
+
+def test_a_contradicted_convention_is_refused(tmp_path):
+    """Reading reciprocal globals as multipliers (or the reverse) would scale every weight
+    by about (2688 / amax)**2: the reader refuses instead of guessing."""
+    write_checkpoint(str(tmp_path), reciprocal=True)
+    with pytest.raises(C.CheckpointError):
+        C.read_moe_experts(C.Checkpoint(str(tmp_path)), PREFIX, CFG.E, global_convention="multiplier")
+    d2 = tmp_path / "mult"
+    d2.mkdir()
+    write_checkpoint(str(d2), reciprocal=False, fmt="")
+    with pytest.raises(C.CheckpointError):
+        C.read_moe_experts(C.Checkpoint(str(d2)), PREFIX, CFG.E, global_convention="reciprocal")
+    r = C.read_moe_experts(C.Checkpoint(str(d2)), PREFIX, CFG.E)          # auto: multipliers
+    assert r["down"]["g_w"][0, 0].item() < 1e-3
 
 
 @pytest.mark.parametrize("marker", [{}, {"layout": "pair-bitmask", "version": 2}, {"layout": "dense", "version": 1}])
@@ -139,7 +177,7 @@ def test_loaded_layer_equals_layer_from_storage(tmp_path):
     same storages directly (the reader adds nothing and loses nothing)."""
     import sparse_nvfp4_moe_b200 as M
     from tests import parity_util as PU
-    st_gu, st_dn, g_in, g_in_dn = write_checkpoint(str(tmp_path))
+    st_gu, st_dn, g_in, g_in_dn = write_checkpoint(str(tmp_path), reciprocal=False, fmt="")
     T = 96
     x = W.layer_input_bf16(CFG, T).cuda()
     ids, w = W.routing(CFG, T)
