@@ -133,3 +133,32 @@ def swiglu_error_bound(acc_gu, bound_gu, rel=1e-5):
     sg = G.silu(gte)
     # |silu'| <= 1.1 everywhere; plus the float32 evaluation of silu and the product
     return 1.1 * (np.abs(up) + eu) * eg + np.abs(sg) * eu + 1e-5 * np.abs(sg * up) + 1e-30
+
+
+def forward_error_limit(ref, down_storages, g_in_dn, topk_w, tol=1e-5):
+    """Per-element bound on |out_gpu - out_exact| of the whole expert MLP.
+
+    ref: the oracle's G.moe_forward result.  The bound adds, per slot, the down GEMM
+    tolerance, the largest effect of a legitimate requantisation flip of h (propagated
+    through |W_down|), the bf16 rounding of y, then combines with |w| in j order and
+    adds the final bf16 rounding.
+    """
+    off = ref["perm"]["expert_offsets"]
+    e_of = R.slot_expert(off)
+    an = requant_analysis(ref["h"], swiglu_error_bound(ref["acc_gu"], ref["bound_gu"], tol),
+                          np.asarray(g_in_dn, np.float32)[e_of])
+    flip = np.zeros_like(ref["y"])
+    for e, st in enumerate(down_storages):
+        if off[e + 1] > off[e]:
+            wabs = np.abs(G.weight_int(st)).astype(np.float64) * 2.0 ** -10 * np.float64(st["g"][0])
+            flip[off[e]:off[e + 1]] = an["max_dev"][off[e]:off[e + 1]] @ wabs.T
+    y_lim = tol * ref["bound_d"] + flip + bf16_ulp(ref["y"]) + bf16_ulp(ref["y"] + flip)
+    ts = ref["perm"]["token_slot"]
+    w = np.asarray(topk_w)
+    lim = sum(np.abs(w[:, j:j + 1]).astype(np.float64) * y_lim[ts[:, j]] for j in range(ts.shape[1]))
+    return lim + bf16_ulp(np.abs(ref["out"]) + lim) + 1e-30
+
+
+def bf16_ulp(v):
+    a = np.maximum(np.abs(v), 2.0 ** -126)
+    return 2.0 ** (np.floor(np.log2(a)) - 7)

@@ -198,18 +198,7 @@ def test_moe_forward_end_to_end(layer):
     got = out.float().cpu().numpy().astype(np.float64)
     assert int(status.item()) == 0
     # bound: down tolerance + bf16 rounding of y + requant flips of h + the final bf16 rounding
-    e_of = R.slot_expert(L.perm["expert_offsets"])
-    an = PU.requant_analysis(ref["h"], PU.swiglu_error_bound(L.acc_gu, L.bound_gu, TOL), L.g_in_dn[e_of])
-    Wabs = [np.abs(G.weight_int(s)).astype(np.float64) * 2.0 ** -10 * np.float64(s["g"][0]) for s in L.dn]
-    flip = np.zeros_like(ref["y"])
-    off = L.perm["expert_offsets"]
-    for e in range(cfg.E):
-        if off[e + 1] > off[e]:
-            flip[off[e]:off[e + 1]] = an["max_dev"][off[e]:off[e + 1]] @ Wabs[e].T
-    y_lim = TOL * ref["bound_d"] + flip + bf16_ulp(ref["y"]) + bf16_ulp(ref["y"] + flip)
-    ts = L.perm["token_slot"]
-    lim = sum(np.abs(L.w[:, j:j + 1]).astype(np.float64) * y_lim[ts[:, j]] for j in range(cfg.k))
-    lim = lim + bf16_ulp(np.abs(ref["out"]) + lim) + 1e-30
+    lim = PU.forward_error_limit(ref, L.dn, L.g_in_dn, L.w, TOL)
     err = np.abs(got - ref["out"])
     assert (err <= lim).all(), f"max err/lim {np.max(err / lim):.3g}"
     # and the typical agreement is tight
