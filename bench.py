@@ -2,7 +2,9 @@
 """Benchmark of the paired-4:8 sparse NVFP4 MoE expert layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--config qwen3_30b_a3b] [--tokens T] [--no-sweep]
+                    [--config qwen3_235b_a22b] [--tokens 65536] [--no-shapes] [--no-storage]
+    python bench.py --storage [--config kimi_k2]          # the storage benchmark alone
+    python bench.py --traffic-csv ncu.csv --traffic-cmd "..."   # ncu DRAM bytes -> profiles/
 
 A step is one pass of the whole routed-expert path over one synthetic batch:
 permute -> NVFP4 activation quantisation -> gate_up sparse grouped GEMM with the
@@ -12,12 +14,20 @@ pair-bitmask storage by the library's own kernels, then repacked.  Inputs sit
 in HBM before timing; L2 is flushed (a 256 MiB write) between timed steps and
 every stage is timed with CUDA events on the launch stream.
 
+The headline line runs the largest layer shape that fits one GPU, Qwen3-235B-A22B
+at 65536 tokens, as the full path.  Its `shapes` key holds the GEMM and step rows
+of every layer shape and token count (Qwen3-30B-A3B, Qwen3.5-397B-A17B,
+Qwen3-235B-A22B, Kimi-K2), with each GEMM also timed back to back over rotated
+weight and activation copies (so that every launch streams its operands from HBM,
+not L2); its `storage` key holds the Kimi-K2 storage benchmark.
+
 Metric: dense-equivalent TFLOP/s (2*S*2I*H + 2*S*H*I per step, S = tokens*k),
 whole job over all ranks.  Multi-GPU runs are replicas (weak scaling): every
 rank runs the same layer on its own batch, no collective on the data path.
 
---impl reference times the CPU oracle (numpy, float64/int64) on a bounded sample
-of the same workload on the host cores; it is a deliberately slow program.
+--impl reference times the CPU oracle (numpy, exact integer products through
+float64) on a bounded sample of the same workload on the host cores; it is a
+deliberately slow program.
 """
 from __future__ import annotations
 
@@ -39,6 +49,9 @@ UNIT = "TFLOP/s"
 B_W, B_A = 0.34375, 0.53125     # bytes per dense element: sparse weight storage, NVFP4-32 activation
 FP4_SPARSE_OVER_BF16 = 8.0      # nominal dense-equivalent sparse FP4 (18 PF) / dense bf16 (2.25 PF)
 KERNELS_PER_STEP = 7            # permute x3, routed quant, gate_up GEMM, down GEMM, combine
+L2_BYTES = 126 * 1024 * 1024    # B200 L2
+DEFAULT_CONFIG, DEFAULT_TOKENS = "qwen3_235b_a22b", 65536
+SHAPE_CONFIGS = ("qwen3_30b_a3b", "qwen3_5_397b_a17b", "qwen3_235b_a22b", "kimi_k2")
 
 
 def parse_args():
@@ -47,16 +60,26 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", default="qwen3_30b_a3b")
-    ap.add_argument("--tokens", type=int, default=16384)
-    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--config", default=None, help=f"layer shape (default {DEFAULT_CONFIG})")
+    ap.add_argument("--tokens", type=int, default=DEFAULT_TOKENS)
+    ap.add_argument("--no-shapes", action="store_true", help="skip the rows of every layer shape and token count")
+    ap.add_argument("--shape-configs", default=",".join(SHAPE_CONFIGS))
+    ap.add_argument("--no-storage", action="store_true", help="skip the Kimi-K2 storage benchmark key")
+    ap.add_argument("--no-dense", action="store_true", help="skip the dense comparison GEMMs")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-slots", type=int, default=2048, help="slots in the CPU-baseline sample")
+    ap.add_argument("--cpu-slots", type=int, default=256, help="slots in the CPU-baseline sample")
     ap.add_argument("--storage", action="store_true",
                     help="storage benchmark instead: decode / re-encode / repack every expert's "
                          "pair-bitmask tensors of --config (default kimi_k2 with this flag)")
-    return ap.parse_args()
+    ap.add_argument("--traffic-csv", default=None,
+                    help="write profiles/traffic.json from this ncu CSV (dram__bytes_read.sum and "
+                         "dram__bytes_write.sum of the GEMM launches) and exit")
+    ap.add_argument("--traffic-cmd", default="", help="the command the ncu CSV came from (recorded)")
+    a = ap.parse_args()
+    if a.config is None:
+        a.config = "kimi_k2" if a.storage else DEFAULT_CONFIG
+    return a
 
 
 def load_peaks():
@@ -67,6 +90,24 @@ def load_peaks():
                     bf16_tflops_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
                     source="measured")
     return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def fp4_peaks(peaks):
+    """Dense-equivalent sparse FP4 tensor peaks: 8 x the measured bf16 GEMM rate (the
+    nominal sparse-FP4 / bf16 ratio, 18 / 2.25 PFLOP/s), burst and sustained."""
+    return FP4_SPARSE_OVER_BF16 * peaks["bf16_tflops"], FP4_SPARSE_OVER_BF16 * peaks["bf16_tflops_sustained"]
+
+
+def classify(flops, nbytes, weight_bytes, peaks):
+    """Roofline of one GEMM launch: (bound, roofline time s, class, target).  A row is
+    decode-sized when HBM binds it and weights are at least half its bytes (target: 70%
+    of HBM), else prefill-sized (target: 60% of its roofline)."""
+    p_burst, _ = fp4_peaks(peaks)
+    t_fl = flops / (p_burst * 1e12)
+    t_by = nbytes / (peaks["hbm_gbs"] * 1e9)
+    bound = "tensor" if t_fl > t_by else "hbm"
+    decode = bound == "hbm" and weight_bytes >= 0.5 * nbytes
+    return bound, max(t_fl, t_by), ("decode-sized" if decode else "prefill-sized"), (0.70 if decode else 0.60)
 
 
 def step_flops(S, H, I):
@@ -295,6 +336,83 @@ class Bench:
         per = {s: [evs[i][j][0].elapsed_time(evs[i][j][1]) for i in range(steps)] for j, s in enumerate(self.STAGES)}
         return step_ms, per
 
+    def rotated_gemm_ms(self, which, launches=40, replays=3):
+        """Per-launch time of one grouped GEMM launched back to back inside a CUDA graph,
+        cycling through R rotation slots so that consecutive launches read operands L2
+        does not hold.  Slot i runs on weight copy i % C and on the routing relabelled by
+        a seeded permutation of the experts (the same group sizes on other experts), with
+        its own activations; R * (weight bytes one launch touches) and C * (all the
+        layer's weight bytes) both reach 3 x L2.  Returns (ms per launch, R, C)."""
+        torch, M, cfg = self.torch, self.M, self.cfg
+        lin = self.lin[which]
+        per_elem = lin.out * lin.K * B_W
+        touched, whole = self.n_touched * per_elem, cfg.E * per_elem
+        C = int(min(8, max(1, -(-3 * L2_BYTES // int(whole)))))
+        R = int(min(64, max(C, -(-3 * L2_BYTES // max(1, int(touched))))))
+        lins = [lin] + [M.ExpertLinear(lin.packed.clone(), lin.meta.clone(), lin.sf.clone(), lin.alpha_w.clone(),
+                                       lin.E, lin.out, lin.K, lin.kind) for _ in range(C - 1)]
+        slots = []
+        gen = torch.Generator(device="cpu")
+        for i in range(R):
+            if i == 0:
+                sl = dict(eo=self.eo, po=self.po, a_codes=self.a_codes, a_sf=self.a_sf, h_codes=self.h_codes,
+                          h_sf=self.h_sf)
+            else:
+                gen.manual_seed(1000 + i)
+                perm = torch.randperm(cfg.E, generator=gen).to(self.dev)
+                ids = perm[self.ids.long()].to(torch.int32).contiguous()
+                i32 = dict(dtype=torch.int32, device=self.dev)
+                sl = dict(eo=torch.empty(cfg.E + 1, **i32), po=torch.empty(cfg.E + 1, **i32),
+                          a_codes=torch.empty_like(self.a_codes), a_sf=torch.empty_like(self.a_sf),
+                          h_codes=torch.empty_like(self.h_codes), h_sf=torch.empty_like(self.h_sf))
+                st, ts = torch.empty_like(self.slot_token), torch.empty_like(self.token_slot)
+                M.moesq_permute(ids, self.T, cfg.k, cfg.E, sl["eo"], sl["po"], st, ts, self.perm_ws, self.perm_ws_n,
+                                self.status)
+                M.moesq_quant_act_routed(self.x.view(torch.uint16), self.T, cfg.H, ids, ts, cfg.k, sl["eo"], sl["po"],
+                                         cfg.E, self.g_in_gu, sl["a_codes"], sl["a_sf"])
+                if which == "down":
+                    M.moesq_grouped_gemm(self.lin["gate_up"].struct, sl["a_codes"], sl["a_sf"], self.g_in_gu,
+                                         sl["eo"], sl["po"], self.S, self.P, M.EPI_SWIGLU_NVFP4, self.g_in_dn,
+                                         sl["h_codes"], sl["h_sf"], d_status=self.status)
+                    del sl["a_codes"], sl["a_sf"]
+            slots.append(sl)
+        out_h = (torch.empty_like(self.h_codes), torch.empty_like(self.h_sf))
+        out_y = torch.empty_like(self.y)
+
+        def launch(i):
+            sl, ln = slots[i], lins[i % C]
+            if which == "gate_up":
+                M.moesq_grouped_gemm(ln.struct, sl["a_codes"], sl["a_sf"], self.g_in_gu, sl["eo"], sl["po"], self.S,
+                                     self.P, M.EPI_SWIGLU_NVFP4, self.g_in_dn, out_h[0], out_h[1],
+                                     d_status=self.status)
+            else:
+                M.moesq_grouped_gemm(ln.struct, sl["h_codes"], sl["h_sf"], self.g_in_dn, sl["eo"], sl["po"], self.S,
+                                     self.P, M.EPI_BF16, None, out_y.view(torch.uint16), None, d_status=self.status)
+
+        reps = max(1, -(-launches // R))
+        for i in range(R):
+            launch(i)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(reps):
+                for i in range(R):
+                    launch(i)
+        stream = torch.cuda.current_stream()
+        g.replay()
+        torch.cuda.synchronize()
+        ms = []
+        for _ in range(replays):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+            b.synchronize()
+            ms.append(a.elapsed_time(b) / (reps * R))
+        del g, slots, lins
+        torch.cuda.empty_cache()
+        return statistics.median(ms), R, C
+
     def dense_comparison(self, steps, flush):
         """The same two GEMMs with the dense comparison kernel on the decoded weights (the
         pages' --no-sparse-storage form): the seeded weights are exported again (the same
@@ -401,64 +519,140 @@ class Bench:
         return sum(times) / len(times), h2d, d2h
 
 
-def cpu_baseline(cfg, T, n_slots, device_ids=None):
-    """The oracle as it stands, on a bounded sample: the most-loaded expert's MLP
-    (quantise -> exact gate_up -> SwiGLU -> requant -> exact down) for n routed slots."""
-    import numpy as np
-    import torch
+def host_cpu():
+    """Host cores this process may use and the CPU model (from /proc/cpuinfo)."""
+    model = ""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        n = len(os.sched_getaffinity(0))
+    except AttributeError:
+        n = os.cpu_count() or 1
+    return {"nproc": n, "model": model}
 
-    import workloads as W
-    from oracle import gemm as G
-    from oracle import nvfp4 as N
-    from oracle import routing as R
-    from oracle import storage as S
 
-    ids, _ = W.routing(cfg, T) if device_ids is None else (device_ids, None)
-    ids = np.asarray(ids)
-    perm = R.permute(ids, cfg.E)
-    counts = np.diff(perm["expert_offsets"])
-    e = int(np.argmax(counts))
-    n = int(min(n_slots, counts[e]))
-    rows = perm["slot_token"][perm["expert_offsets"][e]:perm["expert_offsets"][e] + n]
-    x = W.layer_input_bf16(cfg, T).float().numpy()[rows]
-    n_seg = 2 if cfg.split_gate_up_global else 1
-    t0 = time.perf_counter()
-    gu = S.quantize_weight(W.expert_weights_bf16(cfg, e, "gate_up").float().numpy(), n_seg)
-    dn = S.quantize_weight(W.expert_weights_bf16(cfg, e, "down").float().numpy(), 1)
-    t_prep = time.perf_counter() - t0
-    g_in = np.float32(np.abs(x).max() / 2688.0)
-    t0 = time.perf_counter()
-    ac, asf = N.quantize_groups(x, g_in)
-    sc = gu["scale"].copy()
-    if n_seg == 2:
-        sc[cfg.I:] = S.fold_up_scales(sc[cfg.I:], gu["g"][0], gu["g"][1])
-    Wg = G.dequant_int(N.unpack_codes(S.decode(gu["packed"], gu["mask"])), sc)
-    acc, _ = G.grouped_gemm_exact([Wg], [gu["g"][0]], G.dequant_int(ac, asf), np.float32([g_in]),
-                                  np.array([0, n]))
-    h = G.swiglu(acc)
-    g_dn = np.float32(np.abs(h).max() / 2688.0)
-    hc, hs = N.quantize_groups(h.astype(np.float32), g_dn)
-    G.grouped_gemm_exact([G.weight_int(dn)], [dn["g"][0]], G.dequant_int(hc, hs), np.float32([g_dn]),
-                         np.array([0, n]))
-    dt = time.perf_counter() - t0
-    flops = 2.0 * n * (2 * cfg.I * cfg.H + cfg.H * cfg.I)
-    return dict(value=flops / dt / 1e12, unit=UNIT, cores=1, kind="oracle",
-                sample=(f"expert {e} ({counts[e]} routed slots) of the {cfg.name}-shaped layer at T={T}: "
-                        f"quantise, exact int64 gate_up, SwiGLU, requant, exact int64 down for {n} slots "
-                        f"({flops / 1e9:.1f} dense-equiv GFLOP in {dt:.1f} s; numpy int64 matmul is "
-                        f"single-threaded; weight export {t_prep:.1f} s excluded)"),
-                seconds=dt)
+class OracleSample:
+    """A bounded sample of the workload for timing the oracle: the most-loaded expert's
+    routed slots (up to n) of the layer at T tokens, with that expert's weights exported
+    to pair-bitmask storage by the oracle (preparation, not timed)."""
+
+    def __init__(self, cfg, T, n_slots):
+        import numpy as np
+
+        import workloads as W
+        from oracle import routing as R
+        from oracle import storage as S
+        ids, _ = W.routing(cfg, T)
+        perm = R.permute(np.asarray(ids), cfg.E)
+        counts = np.diff(perm["expert_offsets"])
+        self.e = e = int(np.argmax(counts))
+        self.count = int(counts[e])
+        self.n = n = int(min(n_slots, counts[e]))
+        rows = perm["slot_token"][perm["expert_offsets"][e]:perm["expert_offsets"][e] + n]
+        self.x = W.layer_input_bf16(cfg, T).float().numpy()[rows]
+        self.n_seg = 2 if cfg.split_gate_up_global else 1
+        self.gu = S.quantize_weight(W.expert_weights_bf16(cfg, e, "gate_up").float().numpy(), self.n_seg)
+        self.dn = S.quantize_weight(W.expert_weights_bf16(cfg, e, "down").float().numpy(), 1)
+        self.cfg, self.T = cfg, T
+        self.flops = 2.0 * n * (2 * cfg.I * cfg.H + cfg.H * cfg.I)
+
+    def run(self, threads=None):
+        """quantise -> exact gate_up -> SwiGLU -> requant -> exact down for the sample's
+        slots.  threads: BLAS threads of numpy's float64 products (None: all host cores).
+        Returns (seconds, threads used)."""
+        import numpy as np
+        from threadpoolctl import threadpool_info, threadpool_limits
+
+        from oracle import gemm as G
+        from oracle import nvfp4 as N
+        from oracle import storage as S
+        cfg, gu, dn, n = self.cfg, self.gu, self.dn, self.n
+        with threadpool_limits(limits=threads):
+            blas = [i for i in threadpool_info() if i.get("user_api") == "blas"]
+            used = max((int(i.get("num_threads", 1)) for i in blas), default=1)
+            t0 = time.perf_counter()
+            g_in = np.float32(np.abs(self.x).max() / 2688.0)
+            ac, asf = N.quantize_groups(self.x, g_in)
+            sc = gu["scale"].copy()
+            if self.n_seg == 2:
+                sc[cfg.I:] = S.fold_up_scales(sc[cfg.I:], gu["g"][0], gu["g"][1])
+            Wg = G.dequant_int(N.unpack_codes(S.decode(gu["packed"], gu["mask"])), sc)
+            acc, _ = G.grouped_gemm_exact([Wg], [gu["g"][0]], G.dequant_int(ac, asf), np.float32([g_in]),
+                                          np.array([0, n]))
+            h = G.swiglu(acc)
+            g_dn = np.float32(np.abs(h).max() / 2688.0)
+            hc, hs = N.quantize_groups(h.astype(np.float32), g_dn)
+            G.grouped_gemm_exact([G.weight_int(dn)], [dn["g"][0]], G.dequant_int(hc, hs), np.float32([g_dn]),
+                                 np.array([0, n]))
+            return time.perf_counter() - t0, used
+
+    def describe(self, dt, used):
+        return (f"expert {self.e} ({self.count} routed slots) of the {self.cfg.name}-shaped layer at T={self.T}: "
+                f"quantise, exact gate_up (integer products through float64), SwiGLU, requant, exact down for "
+                f"{self.n} slots ({self.flops / 1e9:.1f} dense-equiv GFLOP in {dt:.2f} s on {used} BLAS "
+                f"thread(s); weight export not timed)")
+
+
+def cpu_baseline(cfg, T, n_slots, threads=None):
+    """The oracle as it stands, timed once on a bounded sample (OracleSample)."""
+    smp = OracleSample(cfg, T, n_slots)
+    smp.run(threads)                 # first call pages in the BLAS
+    dt, used = smp.run(threads)
+    hc = host_cpu()
+    return dict(value=smp.flops / dt / 1e12, unit=UNIT, cores=used, kind="oracle", sample=smp.describe(dt, used),
+                nproc=hc["nproc"], cpu_model=hc["model"], seconds=dt)
 
 
 def traffic_record():
     """ncu DRAM bytes per launch, valid only for the kernel source it was taken on."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
-    src = os.path.join(ROOT, "sparse_nvfp4_moe_b200", "csrc", "gemm_sp.cu")
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
-    return d if d.get("gemm_sp_sha256") == sha else None
+    return d if d.get("gemm_sp_sha256") == gemm_source_sha() else None
+
+
+def gemm_source_sha():
+    src = os.path.join(ROOT, "sparse_nvfp4_moe_b200", "csrc", "gemm_sp.cu")
+    return hashlib.sha256(open(src, "rb").read()).hexdigest()
+
+
+def write_traffic(csv_path, command, workload):
+    """profiles/traffic.json from an ncu CSV of the grouped-GEMM launches (metrics
+    dram__bytes_read.sum and dram__bytes_write.sum, one row per launch and metric):
+    mean DRAM bytes per launch of the gate_up (SwiGLU epilogue) and down (bf16) GEMMs,
+    stamped with the hash of the kernel source they were taken on."""
+    import collections
+    import csv
+    rows = list(csv.reader(open(csv_path)))
+    hi = next(i for i, r in enumerate(rows) if "Kernel Name" in r)
+    hdr, data = rows[hi], rows[hi + 1:]
+    ki, mi, vi, ui, idi = (hdr.index(c) for c in ("Kernel Name", "Metric Name", "Metric Value", "Metric Unit", "ID"))
+    unit = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "Tbyte": 1e12}
+    per = collections.defaultdict(dict)
+    for r in data:
+        if len(r) <= vi or not r[vi]:
+            continue
+        per[(r[idi], r[ki])][r[mi]] = float(r[vi].replace(",", "")) * unit.get(r[ui], 1)
+    res = {}
+    for (_, name), m in per.items():
+        key = "gate_up" if "k_grouped_gemm_sp<2," in name else ("down" if "k_grouped_gemm_sp<1," in name else None)
+        if key is None or "dram__bytes_read.sum" not in m:
+            continue
+        res.setdefault(key, []).append(m["dram__bytes_read.sum"] + m.get("dram__bytes_write.sum", 0.0))
+    out = {"workload": workload, "gemm_sp_sha256": gemm_source_sha(), "command": command,
+           "launches": {k: len(v) for k, v in res.items()}}
+    for k, v in res.items():
+        out[k] = sum(v) / len(v)
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    json.dump(out, open(path, "w"), indent=1)
+    return out
 
 
 def max_over_ranks(ms, world, device):
@@ -478,29 +672,83 @@ def whole_job_value(world, steps, flops_step, max_ms):
     return world * steps * flops_step / (max_ms * 1e-3) / 1e12
 
 
+def gemm_row(b, key, ms, isolated_ms, peaks, rot=None):
+    """One GEMM's figures on one layer shape and token count."""
+    cfg = b.cfg
+    fl = step_flops(b.S, cfg.H, cfg.I)[key]
+    by = step_bytes(b.S, b.T, cfg.H, cfg.I, b.n_touched)[key]
+    wb = b.n_touched * (2 * cfg.I * cfg.H if key == "gate_up" else cfg.H * cfg.I) * B_W
+    bound, t_roof, cls, target = classify(fl, by, wb, peaks)
+    p_burst, p_sust = fp4_peaks(peaks)
+    d = ms * 1e-3
+    row = {"ms": ms, "isolated_ms": isolated_ms, "TFLOPs": fl / d / 1e12, "GBps": by / d / 1e9,
+           "hbm_frac": by / d / 1e9 / peaks["hbm_gbs"], "tensor_frac": fl / d / 1e12 / p_burst,
+           "roofline_frac": t_roof / d, "bound": bound, "class": cls, "target": target,
+           "meets_target": (by / d / 1e9 / peaks["hbm_gbs"] if cls == "decode-sized" else t_roof / d) >= target,
+           "algorithmic_bytes": by, "weight_bytes": wb, "flops": fl}
+    if rot is not None:
+        row["rotation"] = {"slots": rot[0], "weight_copies": rot[1]}
+    return row
+
+
+def shape_rows(b_main, cfg_names, flush, peaks, dev):
+    """GEMM and step rows of every layer shape and token count (one GPU)."""
+    import torch
+
+    import workloads as W
+    rows = []
+    for name in cfg_names:
+        cfg = W.CONFIGS[name]
+        lin = b_main.lin if cfg.name == b_main.cfg.name else None
+        for T in cfg.tokens:
+            if cfg.name == b_main.cfg.name and T == b_main.T:
+                bb = b_main
+            else:
+                bb = Bench(cfg, T, dev, lin=lin)
+                lin = bb.lin
+            st_t, per_t = bb.run(5, 3, flush)
+            iso = {s: statistics.median(v) for s, v in per_t.items()}
+            ms_t = statistics.median(st_t)
+            f2 = step_flops(bb.S, cfg.H, cfg.I)
+            row = {"config": cfg.name, "tokens": T, "slots": bb.S, "experts_touched": bb.n_touched,
+                   "max_group": bb.max_group, "ms_per_step": ms_t,
+                   "TFLOPs": (f2["gate_up"] + f2["down"]) / (ms_t * 1e-3) / 1e12,
+                   "tokens_per_s": T / (ms_t * 1e-3)}
+            for st, key in (("gemm_gate_up", "gate_up"), ("gemm_down", "down")):
+                ms_r, R, C = bb.rotated_gemm_ms(key)
+                row[key] = gemm_row(bb, key, ms_r, iso[st], peaks, (R, C))
+            rows.append(row)
+            if bb is not b_main:
+                del bb
+            torch.cuda.empty_cache()
+        del lin
+        torch.cuda.empty_cache()
+    return rows
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
-    import torch.distributed as dist
 
     import workloads as W
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     cfg = W.CONFIGS[args.config]
     peaks = load_peaks()
+    p_burst, p_sust = fp4_peaks(peaks)
     b = Bench(cfg, args.tokens, dev)
     ok = b.check_against_forward()
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     if world > 1:
-        dist.barrier()
+        torch.distributed.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clk:
         if world > 1:
-            dist.barrier()
+            torch.distributed.barrier()
         torch.cuda.synchronize()
         step_ms, per = b.run(args.steps, max(args.warmup, 3), flush)
         torch.cuda.synchronize()
         if world > 1:
-            dist.barrier()
+            torch.distributed.barrier()
     clocks = clk.summary()
     total_ms = max_over_ranks(sum(step_ms), world, dev)
     S, H, I = b.S, cfg.H, cfg.I
@@ -508,46 +756,50 @@ def run_ours(args, rank, world, local_rank):
     by = step_bytes(S, args.tokens, H, I, b.n_touched)
     flops_step = fl["gate_up"] + fl["down"]
     value = whole_job_value(world, args.steps, flops_step, total_ms)
-    # roofline of the dominant kernel
+    # roofline of the dominant kernel, timed alone in its own graph after an L2 flush
     avg = {s: sum(v) / len(v) for s, v in per.items()}
     dom = max(("gemm_gate_up", "gemm_down"), key=lambda s: avg[s])
     key = "gate_up" if dom == "gemm_gate_up" else "down"
-    p_fp4 = FP4_SPARSE_OVER_BF16 * peaks["bf16_tflops_sustained"]
-    t_fl = fl[key] / (p_fp4 * 1e12)
-    t_by = by[key] / (peaks["hbm_gbs"] * 1e9)
+    wb = b.n_touched * (2 * I * H if key == "gate_up" else H * I) * B_W
+    bound, _, cls, target = classify(fl[key], by[key], wb, peaks)
     dur = avg[dom] * 1e-3
     tr = traffic_record()
     traffic = None
     if tr and tr.get("workload") == f"{cfg.name}:T={args.tokens}":
         traffic = tr.get(key)
-    if t_fl >= t_by:
-        roof = {"bound": "tensor", "achieved": fl[key] / dur / 1e12, "peak": p_fp4, "unit": "TFLOP/s"}
+    if bound == "tensor":
+        roof = {"bound": "tensor", "achieved": fl[key] / dur / 1e12, "peak": p_burst, "unit": "TFLOP/s"}
+        roof["frac_of_sustained_peak"] = roof["achieved"] / p_sust
     else:
         roof = {"bound": "hbm", "achieved": by[key] / dur / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = traffic
     roof.update(kernel=f"k_grouped_gemm_sp ({key})", algorithmic_bytes=by[key], algorithmic_flops=fl[key],
-                avg_launch_ms=avg[dom], peak_source=(f"{peaks['source']}: sparse FP4 = 8 x bf16 sustained "
-                                                   f"{peaks['bf16_tflops_sustained']} TFLOP/s; HBM "
-                                                   f"{peaks['hbm_gbs']} GB/s copy"))
+                avg_launch_ms=avg[dom], row_class=cls, target=target,
+                peak_source=(f"{peaks['source']}: sparse FP4 (dense-equivalent) = 8 x bf16 GEMM burst "
+                             f"{peaks['bf16_tflops']} TFLOP/s = {p_burst:.0f} TFLOP/s (sustained: 8 x "
+                             f"{peaks['bf16_tflops_sustained']} = {p_sust:.0f}); HBM {peaks['hbm_gbs']} GB/s copy"))
     kernels = {}
-    for s in b.STAGES:
+    for s_ in b.STAGES:
         k = {"permute": "permute", "quant_act": "quant_act", "gemm_gate_up": "gate_up", "gemm_down": "down",
-             "combine": "combine"}[s]
-        d = avg[s] * 1e-3
-        ent = {"ms": avg[s], "bytes_GBps": by[k] / d / 1e9, "hbm_frac": by[k] / d / 1e9 / peaks["hbm_gbs"]}
+             "combine": "combine"}[s_]
+        d = avg[s_] * 1e-3
+        ent = {"ms": avg[s_], "bytes_GBps": by[k] / d / 1e9, "hbm_frac": by[k] / d / 1e9 / peaks["hbm_gbs"]}
         if k in fl:
             ent["TFLOPs"] = fl[k] / d / 1e12
-            ent["tensor_frac"] = fl[k] / d / 1e12 / p_fp4
-            ent["roofline_frac"] = max(fl[k] / (p_fp4 * 1e12), by[k] / (peaks["hbm_gbs"] * 1e9)) / d
-        kernels[s] = ent
+            ent["tensor_frac"] = fl[k] / d / 1e12 / p_burst
+            ent["roofline_frac"] = max(fl[k] / (p_burst * 1e12), by[k] / (peaks["hbm_gbs"] * 1e9)) / d
+        kernels[s_] = ent
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": total_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e4m3 block scales) -> fp32 accumulate",
-        "data": "synthetic (seeded bf16 N(0,0.02) weights pruned/quantised by the library; bf16 N(0,1) "
-                "inputs with 1% x20 outlier channels; uniform random router logits)",
-        "config": {"workload": f"{cfg.name}-shaped MoE expert layer, full path (moe_forward stages)",
+        "data": ("synthetic (seeded bf16 N(0,0.02) weights pruned/quantised by the library; bf16 N(0,1) inputs"
+                 + ("; 1% x20 outlier channels" if cfg.outlier_channels else "")
+                 + f"; {cfg.routing} router logits)"),
+        "config": {"workload": (f"{cfg.name}-shaped MoE expert layer ({cfg.E} experts, top-{cfg.k}, hidden {H}, "
+                                f"intermediate {I}) at {args.tokens} tokens, the full moe_forward path: permute, "
+                                f"activation quant, gate_up + SwiGLU + NVFP4 requant, down, weighted combine"),
                    "E": cfg.E, "k": cfg.k, "H": H, "I": I, "tokens": args.tokens, "slots": S,
                    "experts_touched": b.n_touched, "max_group": b.max_group,
                    "l2": "flushed between timed steps (256 MiB write)", "parallelism": f"replicas x{world}"},
@@ -562,48 +814,46 @@ def run_ours(args, rank, world, local_rank):
         e2e_val = whole_job_value(world, 1, flops_step, max_over_ranks(ms, world, dev))
         out["e2e"] = {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                       "ms_per_step": ms, "api": "moesq_moe_forward_host (pinned host buffers)"}
-    if not args.no_sweep and world == 1:
-        sweep = []
-        for T in cfg.tokens:
-            if T == args.tokens:
-                continue
-            bb = Bench(cfg, T, dev, lin=b.lin)
-            st_t, per_t = bb.run(10, 3, flush)
-            a = {s: sum(v) / len(v) for s, v in per_t.items()}
-            f2 = step_flops(bb.S, H, I)
-            y2 = step_bytes(bb.S, T, H, I, bb.n_touched)
-            ms_t = sum(st_t) / len(st_t)
-            row = {"tokens": T, "ms_per_step": ms_t,
-                   "TFLOPs": (f2["gate_up"] + f2["down"]) / (ms_t * 1e-3) / 1e12}
-            for s, k in (("gemm_gate_up", "gate_up"), ("gemm_down", "down")):
-                d = a[s] * 1e-3
-                row[k] = {"ms": a[s], "TFLOPs": f2[k] / d / 1e12, "GBps": y2[k] / d / 1e9,
-                          "roofline_frac": max(f2[k] / (p_fp4 * 1e12), y2[k] / (peaks["hbm_gbs"] * 1e9)) / d,
-                          "bound": ("tensor" if f2[k] / (p_fp4 * 1e12) > y2[k] / (peaks["hbm_gbs"] * 1e9)
-                                    else "hbm")}
-            sweep.append(row)
-            del bb
-            torch.cuda.empty_cache()
-        out["sweep"] = sweep
-    if not args.no_sweep and world == 1:
+    if world == 1 and not args.no_dense:
         d = b.dense_comparison(10, flush)
-        fl_d = step_flops(b.S, H, I)
         by_w = {"gate_up": b.n_touched * 2 * I * H, "down": b.n_touched * H * I}
         out["dense_comparison"] = {
             "what": "the same gate_up (SwiGLU + requant) and down (bf16) GEMMs on the decoded dense NVFP4 "
                     "weights (dense tcgen05 MMA, 16-element scale blocks), same workload and inputs",
             **{f"{k}_ms": d[k] for k in d},
-            **{f"{k}_TFLOPs": fl_d[k] / (d[k] * 1e-3) / 1e12 for k in d},
+            **{f"{k}_TFLOPs": fl[k] / (d[k] * 1e-3) / 1e12 for k in d},
             "sparse_speedup": {k: d[k] / avg["gemm_" + k] for k in d},
             "weight_bytes_per_dense_element": {"sparse": 0.34375, "dense": 0.53125},
             "weight_bytes_touched_GB": {k: {"sparse": by_w[k] * 0.34375 / 1e9, "dense": by_w[k] * 0.53125 / 1e9}
                                         for k in by_w},
         }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = {k: v for k, v in cpu_baseline(cfg, args.tokens, args.cpu_slots).items()
-                               if k != "seconds"}
+        one = cpu_baseline(cfg, args.tokens, args.cpu_slots, threads=1)
+        allc = cpu_baseline(cfg, args.tokens, 8 * args.cpu_slots, threads=None)
+        cb = {k: v for k, v in allc.items() if k != "seconds"}
+        cb["single_thread"] = {k: v for k, v in one.items() if k not in ("seconds", "kind", "nproc", "cpu_model")}
+        out["cpu_baseline"] = cb
+    if world == 1 and not args.no_shapes:
+        names = [n for n in args.shape_configs.split(",") if n]
+        out["shapes"] = shape_rows(b, names, flush, peaks, dev)
+        out["shapes_method"] = (
+            "per row: ms_per_step = the whole path as one CUDA graph after an L2 flush (median of 5); per GEMM: "
+            "ms = one launch of a CUDA graph of >= 40 back-to-back launches that cycle through rotation slots "
+            "(relabelled routings and weight copies, >= 3 x L2 of distinct operands); isolated_ms = the GEMM "
+            "alone in its own graph after an L2 flush (includes graph launch and cold start); fractions against "
+            "the measured HBM copy and 8 x the measured bf16 burst peak; decode-sized rows (HBM-bound, weights "
+            ">= half the bytes) target 70% of HBM, the others 60% of their roofline")
     if int(b.status.item()) != 0:
         out["device_status"] = int(b.status.item())
+    del b
+    torch.cuda.empty_cache()
+    if world == 1 and not args.no_storage:
+        a2 = argparse.Namespace(**vars(args))
+        a2.config, a2.steps, a2.warmup = "kimi_k2", 5, 3
+        st = run_storage(a2)
+        out["storage"] = {k: st[k] for k in ("metric", "value", "unit", "ms_per_step", "round_trip_bit_exact",
+                                             "per_op", "config", "device_status")}
+        out["storage"]["hbm_frac"] = st["roofline"]["frac"]
     return out
 
 
@@ -614,19 +864,22 @@ def run_reference(args, rank, world):
     import workloads as W
     cfg = W.CONFIGS[args.config]
     slots = 128
-    vals = []
-    for i in range(max(args.warmup, 0) + args.steps):
-        r = cpu_baseline(cfg, args.tokens, slots)
-        if i >= args.warmup:
-            vals.append(r)
-    tot_flops = sum(v["value"] * v["seconds"] for v in vals)
-    tot_s = sum(v["seconds"] for v in vals)
-    value = tot_flops / tot_s
-    cb = dict(vals[-1])
-    cb.pop("seconds", None)
-    cb["value"] = value
+    smp = OracleSample(cfg, args.tokens, slots)
+    for _ in range(max(args.warmup, 0)):
+        smp.run()
+    times = []
+    used = 1
+    for _ in range(args.steps):
+        dt, used = smp.run()
+        times.append(dt)
+    tot_s = sum(times)
+    value = smp.flops * len(times) / tot_s / 1e12
+    hc = host_cpu()
+    cb = {"value": value, "unit": UNIT, "cores": used, "kind": "oracle",
+          "sample": smp.describe(tot_s / len(times), used) + " per step", "nproc": hc["nproc"],
+          "cpu_model": hc["model"]}
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_s / len(vals) * 1e3,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_s / len(times) * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64/f64 (exact)",
             "data": "synthetic", "config": {"workload": f"{cfg.name}-shaped MoE expert layer (oracle sample)",
                                               "tokens": args.tokens, "slots_per_step": slots},
@@ -650,8 +903,7 @@ def run_storage(args):
 
     import sparse_nvfp4_moe_b200 as M
     import workloads as W
-    cfg_name = args.config if args.config != "qwen3_30b_a3b" else "kimi_k2"
-    cfg = W.CONFIGS[cfg_name]
+    cfg = W.CONFIGS[args.config]
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     peaks = load_peaks()
@@ -730,6 +982,9 @@ def run_storage(args):
 
 def main():
     args = parse_args()
+    if args.traffic_csv:
+        print(json.dumps(write_traffic(args.traffic_csv, args.traffic_cmd, f"{args.config}:T={args.tokens}")))
+        return 0
     if args.storage and args.impl == "ours":
         print(json.dumps(run_storage(args)))
         return 0
