@@ -167,12 +167,26 @@ struct TileWalk {
   }
 };
 
-// The current item of `w` (empty experts are stepped over: their tiles end
-// where they start).
+// The current item of `w`.  Empty experts end their tiles where they start; when
+// the next expert does not hold tile q either, a binary search over the tile-end
+// prefix sums finds the first expert that does, so a walk over thousands of empty
+// experts (decode batches of a layer with many experts) costs log2(E) loads, not E.
 __device__ __forceinline__ Tile decode_tile(const Smem& s, TileWalk& w, int E) {
-  while (w.cur.x <= w.q && w.e + 1 < E) {
-    ++w.e;
-    w.cur = w.nxt;
+  if (w.cur.x <= w.q && w.e + 1 < E) {
+    if (w.nxt.x > w.q) {
+      ++w.e;
+      w.cur = w.nxt;
+    } else {
+      // rec[e + 1].x <= q < rec[E - 1].x (q is below the total tile count)
+      int lo = w.e + 2, hi = E - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (s.rec[mid].x > w.q) hi = mid;
+        else lo = mid + 1;
+      }
+      w.e = lo;
+      w.cur = s.rec[lo];
+    }
     w.nxt = w.e + 1 < E ? s.rec[w.e + 1] : w.cur;
   }
   const int4 r = w.cur;
