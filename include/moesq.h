@@ -201,9 +201,11 @@ moesq_status moesq_permute_workspace_size(int64_t T, int32_t k, int32_t E, size_
  *   MOESQ_ERR_CAPACITY is returned and nothing is enqueued (e.g. E = 512 allows
  *   T*k up to 524288).
  *   The first call on a device looks up the array's device address with that device
- *   current (cudaGetSymbolAddress) and caches it; make that first call before any
- *   stream capture.  Every GPU that loads the library holds the array until the
- *   process exits.  All calls share it, and each call overwrites the parts it reads,
+ *   current (cudaGetSymbolAddress) and caches it for the process; make that first call
+ *   before any stream capture.  The cached address belongs to the device's primary
+ *   context: calls after cudaDeviceReset in the same process are not supported.
+ *   Every GPU that loads the library holds the array until the process exits.  All
+ *   calls share it, and each call overwrites the parts it reads,
  *   so calls whose executions overlap on the GPU (other streams, other host threads)
  *   race and must be ordered by the caller. */
 #define MOESQ_PERMUTE_NOALLOC_MAX_COUNTS 262144
