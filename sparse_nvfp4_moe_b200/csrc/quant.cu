@@ -166,6 +166,81 @@ __global__ void k_quant_act_routed(const uint16_t* __restrict__ x, int64_t T, in
   }
 }
 
+// Warp form of the routed quantisation for K % 1024 == 0 (a warp covers 32 groups =
+// 1024 elements of one token).  Lanes 0..k-1 load the token's routing once (expert,
+// slot, the expert's global and padded row) and the warp shares it by shuffles, so a
+// thread waits for one round of index loads per token instead of two per slot.  Each
+// lane quantises its group and stores 16 code bytes per slot (512 contiguous bytes per
+// warp and slot); lanes 4m..4m+3 hold the four scales that share a 512-byte block
+// position and lane 4m stores them as one 32-bit word.
+__global__ void k_quant_act_routed_warp(const uint16_t* __restrict__ x, int64_t T, int64_t K,
+                                        const int32_t* __restrict__ topk_ids,
+                                        const int32_t* __restrict__ token_slot, int k,
+                                        const int32_t* __restrict__ expert_offsets,
+                                        const int32_t* __restrict__ pad_offsets, int E,
+                                        const float* __restrict__ g_in, uint8_t* __restrict__ codes,
+                                        uint8_t* __restrict__ sf) {
+  pdl_wait();  // the previous kernel's outputs are complete past here
+  pdl_trigger();
+  const int lane = threadIdx.x & 31;
+  const int64_t W = K / 1024;  // warp chunks per token
+  const int64_t nw = T * W;
+  const int64_t wstride = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; w < nw; w += wstride) {
+    const int64_t t = w / W;
+    const int64_t grp = 32 * (w - t * W) + lane;
+    // routing of token t: lane j < k holds slot j's global and padded row
+    float gj = 0.0f;
+    int rowj = 0;
+    if (lane < k) {
+      int e = topk_ids[t * k + lane];
+      if (e < 0 || e >= E) e = 0;
+      gj = g_in[e];
+      rowj = pad_offsets[e] + (token_slot[t * k + lane] - expert_offsets[e]);
+    }
+    float v[32];
+    const uint4* q = reinterpret_cast<const uint4*>(x + t * K + 32 * grp);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint4 u = q[c];
+      const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        v[8 * c + 2 * j] = bf16_bits_to_float(wd[j] & 0xFFFF);
+        v[8 * c + 2 * j + 1] = bf16_bits_to_float(wd[j] >> 16);
+      }
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(v[j]));
+    // the codes and scale depend on the slot only through its expert's global: a slot
+    // whose global equals the previous slot's (bit for bit) reuses them (warp-uniform)
+    float g_prev = 0.0f;
+    GroupScale gs = {0u, 0.0f};
+    uint32_t o[4] = {0u, 0u, 0u, 0u};
+    uint32_t word = 0u;
+    for (int j = 0; j < k; ++j) {
+      const float g = __shfl_sync(0xffffffffu, gj, j);
+      const int64_t row = __shfl_sync(0xffffffffu, rowj, j);
+      if (j == 0 || __float_as_uint(g) != __float_as_uint(g_prev)) {
+        g_prev = g;
+        gs = nvfp4_group_scale(amax, g);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) o[c] = nvfp4_word(v + 8 * c, gs.inv);
+        const uint32_t b1 = __shfl_down_sync(0xffffffffu, gs.sc, 1);
+        const uint32_t b2 = __shfl_down_sync(0xffffffffu, gs.sc, 2);
+        const uint32_t b3 = __shfl_down_sync(0xffffffffu, gs.sc, 3);
+        word = (gs.sc & 0xFFu) | ((b1 & 0xFFu) << 8) | ((b2 & 0xFFu) << 16) | ((b3 & 0xFFu) << 24);
+      }
+      *reinterpret_cast<uint4*>(codes + row * (K / 2) + 16 * grp) = make_uint4(o[0], o[1], o[2], o[3]);
+      if ((lane & 3) == 0) {
+        const int64_t blk = (row / 128) * (K / 128) + grp / 4;
+        *reinterpret_cast<uint32_t*>(sf + blk * 512 + sf_block_offset((uint32_t)(row % 128), 0u)) = word;
+      }
+    }
+  }
+}
+
 // Routed NVFP4 rows quantised elsewhere (codes [n, K/2], linear scales [n, K/32], e.g.
 // received from another GPU) into the grouped GEMM's padded operand layout: slot s of
 // the expert-ordered list takes input row gather[s] and lands on padded row
@@ -261,7 +336,15 @@ extern "C" moesq_status moesq_quant_act_routed(const uint16_t* x, int64_t T, int
   const int64_t n = T * (K / 32);
   int64_t g = (n + 127) / 128;
   if (g > 148 * 32) g = 148 * 32;
-  // small batches (decode): every slot's index loads in flight at once; large: more warps
+  // a warp per 1024 elements of a token when K allows it and k fits a warp; otherwise
+  // thread per group: for small batches (decode) every slot's index loads in flight at
+  // once, for large ones more warps
+  if (K % 1024 == 0 && k <= 32) {
+    if (moesq_launch(k_quant_act_routed_warp, dim3((unsigned)g), dim3(128), 0, (cudaStream_t)stream, x, T, K, topk_ids,
+                     token_slot, k, expert_offsets, pad_offsets, E, g_in, codes, sf) != cudaSuccess)
+      return MOESQ_ERR_CUDA;
+    return MOESQ_OK;
+  }
   const cudaError_t err =
       T <= 512 ? moesq_launch(k_quant_act_routed<true>, dim3((unsigned)g), dim3(128), 0, (cudaStream_t)stream, x, T, K,
                               topk_ids, token_slot, k, expert_offsets, pad_offsets, E, g_in, codes, sf)
