@@ -22,8 +22,11 @@ weight and activation copies (so that every launch streams its operands from HBM
 not L2); its `storage` key holds the Kimi-K2 storage benchmark.
 
 Metric: dense-equivalent TFLOP/s (2*S*2I*H + 2*S*H*I per step, S = tokens*k),
-whole job over all ranks.  Multi-GPU runs are replicas (weak scaling): every
-rank runs the same layer on its own batch, no collective on the data path.
+whole job over all ranks.  Multi-GPU runs (one process per GPU under torchrun) are
+expert parallel by default (weak scaling): rank r holds a contiguous 1/N of the
+experts and routes its own batch of --tokens tokens, and every step sends each
+routed slot's NVFP4 codes and scales to its expert's rank and the bf16 outputs back
+(NCCL all-to-all).  --replicas runs N independent copies of the one-GPU path instead.
 
 --impl reference times the CPU oracle (numpy, exact integer products through
 float64) on a bounded sample of the same workload on the host cores; it is a
@@ -76,6 +79,10 @@ def parse_args():
                     help="write profiles/traffic.json from this ncu CSV (dram__bytes_read.sum and "
                          "dram__bytes_write.sum of the GEMM launches) and exit")
     ap.add_argument("--traffic-cmd", default="", help="the command the ncu CSV came from (recorded)")
+    ap.add_argument("--ep", action="store_true",
+                    help="expert-parallel mode even on one rank (under torchrun), the default for N > 1")
+    ap.add_argument("--replicas", action="store_true",
+                    help="with N > 1 GPUs: N independent replicas of the one-GPU path instead of expert parallelism")
     a = ap.parse_args()
     if a.config is None:
         a.config = "kimi_k2" if a.storage else DEFAULT_CONFIG
@@ -857,6 +864,128 @@ def run_ours(args, rank, world, local_rank):
     return out
 
 
+def ep_launches(T, k, n_recv):
+    """Library kernels one expert-parallel step launches on a rank: permute of its
+    tokens (1 kernel up to 1024 slots, else 3), quantisation, permute of the received
+    slots (same rule), gather into the operand layout, the two GEMMs, the gather back
+    to the received order and the weighted combine."""
+    perm = lambda n: 1 if n <= 1024 else 3
+    return perm(T * k) + 1 + (perm(n_recv) + 1 + 2 + 1 if n_recv > 0 else 0) + 1
+
+
+def run_ep(args, rank, world, local_rank):
+    """Expert parallelism over the ranks (one process per GPU, NCCL): rank r holds the
+    contiguous expert range [E r / N, E (r+1) / N) and routes its own batch of T tokens;
+    each step dispatches every routed slot's NVFP4 codes and scales to its expert's rank
+    and brings the bf16 down outputs back for the j-order combine
+    (sparse_nvfp4_moe_b200.ep.ExpertParallelMoE).  Weak scaling: T tokens per rank."""
+    import dataclasses
+
+    import torch
+    import torch.distributed as dist
+
+    import sparse_nvfp4_moe_b200 as M
+    import workloads as W
+    from sparse_nvfp4_moe_b200.ep import DeviceCompute, ExpertParallelMoE, expert_ranges
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cfg = W.CONFIGS[args.config]
+    T, H, I, E, k = args.tokens, cfg.H, cfg.I, cfg.E, cfg.k
+    lo, hi = expert_ranges(E, world)[rank]
+    n_seg = 2 if cfg.split_gate_up_global else 1
+    lin = {}
+    for which, ns, kd in (("gate_up", n_seg, M.KIND_GATE_UP_SPLIT if n_seg == 2 else M.KIND_GATE_UP),
+                          ("down", 1, M.KIND_DOWN)):
+        w = W.all_expert_weights_bf16(cfg, which, device=dev, experts=range(lo, hi))
+        st = M.quantize_expert_weights(w, ns)
+        del w
+        lin[which] = M.ExpertLinear.from_storage(st, kd)
+        del st
+    # this rank's tokens: the layer's generator reseeded per rank (the weights keep the layer's seed)
+    tcfg = dataclasses.replace(cfg, seed=cfg.seed + 7919 * (rank + 1))
+    x = W.layer_input_bf16(tcfg, T, device=dev)
+    ids, tw = W.routing(tcfg, T, device=dev)
+    ids, tw = ids.contiguous(), tw.contiguous()
+    # one static input global for every rank (the largest amax/(6*448) over the ranks'
+    # batches) and fixed down-input globals: the values do not change the work
+    g = torch.tensor([W.activation_global_scale_input(x)], dtype=torch.float32, device=dev)
+    dist.all_reduce(g, op=dist.ReduceOp.MAX)
+    g_all = g.expand(E).contiguous()
+    g_dn = torch.full((hi - lo,), 0.01, dtype=torch.float32, device=dev)
+    local = M.MoELayer(k, lin["gate_up"], lin["down"], g_all[lo:hi].contiguous(), g_dn)
+    moe = ExpertParallelMoE(E, k, H, DeviceCompute(local, g_all))
+    # slots this rank sends to every rank (its routing is fixed over the steps)
+    owner = torch.bucketize(ids.long().flatten(), torch.tensor([h for _, h in expert_ranges(E, world)], device=dev),
+                            right=True)
+    send = torch.bincount(owner, minlength=world).to(torch.int64)
+    recv = torch.empty_like(send)
+    dist.all_to_all_single(recv, send)
+    send_h, recv_h = send.cpu().tolist(), recv.cpu().tolist()
+    remote_out = sum(send_h) - send_h[rank]
+    remote_in = sum(recv_h) - recv_h[rank]
+    for _ in range(max(args.warmup, 3)):
+        moe.forward(x, ids, tw)
+    torch.cuda.synchronize()
+    dist.barrier()
+    stream = torch.cuda.current_stream()
+    with ClockSampler(local_rank) as clk:
+        dist.barrier()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            moe.forward(x, ids, tw)
+        b.record(stream)
+        b.synchronize()
+        dist.barrier()
+    clocks = clk.summary()
+    total_ms = max_over_ranks(a.elapsed_time(b), world, dev)
+    fl = step_flops(T * k, H, I)
+    flops_step = fl["gate_up"] + fl["down"]
+    value = whole_job_value(world, args.steps, flops_step, total_ms)
+    # end to end: the batch and its routing from pinned host memory, the output back
+    hx, hids, hw = x.cpu().pin_memory(), ids.cpu().pin_memory(), tw.cpu().pin_memory()
+    hout = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
+    n_e2e = max(3, args.steps // 4)
+    for _ in range(2):
+        hout.copy_(moe.forward(hx.to(dev, non_blocking=True), hids.to(dev, non_blocking=True),
+                               hw.to(dev, non_blocking=True)), non_blocking=True)
+    torch.cuda.synchronize()
+    dist.barrier()
+    a2, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a2.record(stream)
+    for _ in range(n_e2e):
+        hout.copy_(moe.forward(hx.to(dev, non_blocking=True), hids.to(dev, non_blocking=True),
+                               hw.to(dev, non_blocking=True)), non_blocking=True)
+    b2.record(stream)
+    b2.synchronize()
+    e2e_ms = max_over_ranks(a2.elapsed_time(b2) / n_e2e, world, dev)
+    per_slot_dispatch = H // 2 + H // 32 + 4      # codes, scales, local expert id
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e4m3 block scales) -> fp32 accumulate",
+        "data": "synthetic (seeded per rank; bf16 N(0,0.02) weights pruned/quantised by the library)",
+        "config": {"workload": (f"{cfg.name}-shaped MoE expert layer ({E} experts, top-{k}, hidden {H}, "
+                                f"intermediate {I}), expert parallel over {world} GPUs: {T} tokens per rank, "
+                                f"experts [{lo}, {hi}) on rank {rank} of a contiguous split"),
+                   "E": E, "k": k, "H": H, "I": I, "tokens_per_rank": T, "slots_per_rank": T * k,
+                   "l2": "not flushed: every step's operands exceed L2", "parallelism": f"ep{world}"},
+        "ep": {"dispatch_bytes_rank0": remote_out * per_slot_dispatch, "combine_bytes_rank0": remote_in * H * 2,
+               "slots_sent_rank0": send_h, "slots_received_rank0": recv_h,
+               "exchange": "torch.distributed.all_to_all_single (NCCL) of NVFP4 codes+scales out, bf16 rows back"},
+        "e2e": {"value": whole_job_value(world, 1, flops_step, e2e_ms), "unit": UNIT,
+                "h2d_bytes_per_step": hx.numel() * 2 + hids.numel() * 4 + hw.numel() * 4,
+                "d2h_bytes_per_step": hout.numel() * 2, "ms_per_step": e2e_ms,
+                "api": "ExpertParallelMoE.forward on host-copied inputs (pinned)"},
+        "gpu_launches": args.steps * ep_launches(T, k, sum(recv_h)),
+        "clocks": clocks,
+    }
+    if int(moe.compute.status.item()) != 0:
+        out["device_status"] = int(moe.compute.status.item())
+    return out
+
+
 def run_reference(args, rank, world):
     """The oracle as it stands, timed on the host cores, on a bounded per-step sample."""
     if rank != 0:
@@ -997,14 +1126,15 @@ def main():
             print(json.dumps(res))
         return 0
     import torch.distributed as dist
-    if world > 1:
+    if world > 1 or (args.ep and "RANK" in os.environ):
         import torch
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        res = run_ours(args, rank, world, local_rank)
+        use_ep = (world > 1 and not args.replicas) or (args.ep and dist.is_initialized())
+        res = run_ep(args, rank, world, local_rank) if use_ep else run_ours(args, rank, world, local_rank)
     finally:
-        if world > 1:
+        if dist.is_initialized():
             dist.barrier()
             dist.destroy_process_group()
     if rank == 0:

@@ -135,12 +135,15 @@ class ExpertParallelMoE:
         recv_t = torch.empty(self.world, dtype=torch.int64, device=codes.device)
         dist.all_to_all_single(recv_t, torch.tensor(send, dtype=torch.int64, device=codes.device), group=self.group)
         recv = recv_t.cpu().tolist()
-        # local expert id of every slot, in slot order (slots are grouped by rank already)
-        counts = torch.tensor([eo_h[e + 1] - eo_h[e] for e in range(self.E)], dtype=torch.int64)
-        e_of_slot = torch.repeat_interleave(torch.arange(self.E, dtype=torch.int64), counts)
-        lo_of_slot = torch.tensor([lo for lo, _ in self.ranges], dtype=torch.int64)[
-            torch.bucketize(e_of_slot, torch.tensor([hi for _, hi in self.ranges]), right=True)]
-        local_ids = (e_of_slot - lo_of_slot).to(torch.int32).to(codes.device)
+        # local expert id of every slot, in slot order (slots are grouped by rank already),
+        # built where the slots live
+        dv = codes.device
+        counts = (eo[1:] - eo[:-1]).to(torch.int64)
+        e_of_slot = torch.repeat_interleave(torch.arange(self.E, dtype=torch.int64, device=dv), counts.to(dv),
+                                            output_size=int(eo_h[-1]))
+        bounds = torch.tensor([hi for _, hi in self.ranges], dtype=torch.int64, device=dv)
+        lows = torch.tensor([lo for lo, _ in self.ranges], dtype=torch.int64, device=dv)
+        local_ids = (e_of_slot - lows[torch.bucketize(e_of_slot, bounds, right=True)]).to(torch.int32)
         r_codes = self._exchange(codes, send, recv)
         r_sf = self._exchange(sf, send, recv)
         r_ids = self._exchange(local_ids, send, recv)

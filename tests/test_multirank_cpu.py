@@ -73,3 +73,14 @@ def test_single_rank_helpers_need_no_process_group():
     import bench
     assert bench.max_over_ranks(12.5, 1, None) == 12.5
     assert bench.whole_job_value(1, 10, 1e12, 5.0) == pytest.approx(10 * 1.0 / 5e-3)
+
+
+def test_ep_launch_count():
+    """Kernels an expert-parallel step launches per rank: permute (1 kernel up to 1024
+    slots, else 3), quantisation, then for received slots permute, gather, 2 GEMMs,
+    gather back; and the combine."""
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.ep_launches(1, 8, 0) == 1 + 1 + 1
+    assert bench.ep_launches(1, 8, 3) == 1 + 1 + (1 + 1 + 2 + 1) + 1
+    assert bench.ep_launches(65536, 8, 524288) == 3 + 1 + (3 + 1 + 2 + 1) + 1
