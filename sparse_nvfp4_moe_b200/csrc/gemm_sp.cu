@@ -604,17 +604,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
         sb ^= 1;
       } else if constexpr (EPI == MOESQ_EPI_BF16) {
-        // Per 32-token column block kb, its four warps (one per lane quarter q) stage
-        // [32 tokens][128 outputs] bf16 as two 64-output halves [32 rows][128 B] in the
-        // TMA 128-byte swizzle (16-byte chunk c of row r at c ^ (r & 7)), then one lane
-        // writes them with two TMA stores, or the 128 threads copy the valid rows when
-        // the block reaches past the expert's tokens.  The interleaved weight rows put
-        // both outputs of a bf16 pair in one thread of a 16x256b TMEM load (down:
-        // lanes j and 8 + j of a 16-lane group; gate_up: gate or up of outputs
-        // 16q + 2j + {0,1} from the loads at lane 32q and 32q + 16), so each pair
-        // is one word and no lanes exchange values.  Words of one store land on 8
-        // consecutive pair slots of 4 rows two apart: no bank conflicts.
-        uint8_t* stg = reinterpret_cast<uint8_t*>(epi) + kb * 8192;  // [2 halves][32 rows][128 B]
+        // Per 32-token column block kb, its four warps (one per lane quarter q) write
+        // [32 tokens][128 outputs] bf16.  The interleaved weight rows put both outputs of
+        // a bf16 pair in one thread of a 16x256b TMEM load (down: lanes j and 8 + j of a
+        // 16-lane group; gate_up: gate or up of outputs 16q + 2j + {0,1} from the loads
+        // at lane 32q and 32q + 16), so each pair is one word and no lanes exchange values.
+        // nblk is the same for the block's four warps, so they take the same branch.
         const int64_t s0 = t.s0;
         int nvalid = t.n_rows;
         if (s0 + nvalid > p.S) nvalid = (int)(p.S - s0 > 0 ? p.S - s0 : 0);
@@ -629,15 +624,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         __syncwarp();
         if (lane == 0) release_acc(buf);
         decode_next();
-        const bool issuer = q == 2 && lane == 0;
-        if (issuer) bulk_wait_group_read0();  // this block's previous stores have read the staging
-        named_bar_sync(10 + kb, 128);         // (and its previous row copy is done)
         const bool gu = p.gate_up;
-        if (nblk > 0) {
-          const int j = lane >> 2;
-          // pair slots and halves of the thread's two words per column
-          const int w0 = gu ? 8 * q + j : 16 * (q & 1) + j;
-          const int w1 = gu ? w0 : w0 + 8;
+        const int j = lane >> 2;
+        // pair slots of the thread's two words per column
+        const int w0 = gu ? 8 * q + j : 16 * (q & 1) + j;
+        const int w1 = gu ? w0 : w0 + 8;
+        if (nblk == 32) {
+          // a full block: the four warps stage [32 tokens][128 outputs] as two 64-output
+          // halves [32 rows][128 B] in the TMA 128-byte swizzle (16-byte chunk c of row r
+          // at c ^ (r & 7)) and one lane writes them with two TMA stores.  Words of one
+          // staging store land on 8 consecutive pair slots of 4 rows two apart: no bank
+          // conflicts.
+          uint8_t* stg = reinterpret_cast<uint8_t*>(epi) + kb * 8192;  // [2 halves][32 rows][128 B]
+          const bool issuer = q == 2 && lane == 0;
+          if (issuer) bulk_wait_group_read0();  // this block's previous stores have read the staging
+          named_bar_sync(10 + kb, 128);
           uint8_t* h0 = stg + (gu ? 0 : (q >> 1) * 4096);
           uint8_t* h1 = stg + (gu ? 4096 : (q >> 1) * 4096);
 #pragma unroll
@@ -649,32 +650,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             // down: (a0, a1) and (c0, c1) are output pairs; gate_up: (a0, c0) gate, (a1, c1) up
             const float2 w0v = __fmul2_rn(make_float2(a0, gu ? c0 : a1), make_float2(alpha, alpha));
             const float2 w1v = __fmul2_rn(make_float2(gu ? a1 : c0, c1), make_float2(gu ? alpha_u : alpha, gu ? alpha_u : alpha));
-            const __nv_bfloat162 p0 = __floats2bfloat162_rn(w0v.x, w0v.y);
-            const __nv_bfloat162 p1 = __floats2bfloat162_rn(w1v.x, w1v.y);
-            *reinterpret_cast<__nv_bfloat162*>(h0 + row * 128 + (((w0 >> 2) ^ (row & 7)) << 4) + ((w0 & 3) << 2)) = p0;
-            *reinterpret_cast<__nv_bfloat162*>(h1 + row * 128 + (((w1 >> 2) ^ (row & 7)) << 4) + ((w1 & 3) << 2)) = p1;
+            *reinterpret_cast<__nv_bfloat162*>(h0 + row * 128 + (((w0 >> 2) ^ (row & 7)) << 4) + ((w0 & 3) << 2)) =
+                __floats2bfloat162_rn(w0v.x, w0v.y);
+            *reinterpret_cast<__nv_bfloat162*>(h1 + row * 128 + (((w1 >> 2) ^ (row & 7)) << 4) + ((w1 & 3) << 2)) =
+                __floats2bfloat162_rn(w1v.x, w1v.y);
           }
-        }
-        fence_proxy_async_smem();
-        named_bar_sync(10 + kb, 128);  // staging of the block complete
-        const int x0 = gu ? 64 * mt : BM * mt;            // first column of half 0
-        const int x1 = gu ? I + 64 * mt : BM * mt + 64;   // and of half 1
-        if (own_tile && nblk == 32) {
-          if (issuer) {
-            tma_store_2d(&tmap_y, stg, x0, (int32_t)(s0 + c_lo));
-            tma_store_2d(&tmap_y, stg + 4096, x1, (int32_t)(s0 + c_lo));
+          fence_proxy_async_smem();
+          named_bar_sync(10 + kb, 128);  // staging of the block complete
+          if (own_tile && issuer) {
+            tma_store_2d(&tmap_y, stg, gu ? 64 * mt : BM * mt, (int32_t)(s0 + c_lo));
+            tma_store_2d(&tmap_y, stg + 4096, gu ? I + 64 * mt : BM * mt + 64, (int32_t)(s0 + c_lo));
             bulk_commit_group();
           }
         } else if (own_tile && nblk > 0) {
-          // 16-byte chunk i: row i >> 4, half (i >> 3) & 1, chunk i & 7 of the half row
-          const int et = 32 * q + lane;  // 0..127 within the block
+          // a block past the expert's last tokens: each pair word goes straight to global
+          // memory; for a fixed (i, b) the eight lanes of equal lane & 3 hold 16
+          // consecutive outputs of one token row, so a warp store writes four tokens'
+          // 32-byte row segments (whole sectors), with no staging or block barrier
+          const int base0 = gu ? 64 * mt : BM * mt + 64 * (q >> 1);
+          const int base1 = gu ? I + 64 * mt : base0;
+          uint16_t* yb = (uint16_t*)p.out + (s0 + c_lo) * p.M;
 #pragma unroll
-          for (int i0 = 0; i0 < 4; ++i0) {
-            const int i = et + 128 * i0;
-            const int r = i >> 4, half = (i >> 3) & 1, jj = i & 7;
-            if (r < nblk) {
-              const uint4 v = *reinterpret_cast<const uint4*>(stg + half * 4096 + r * 128 + ((jj ^ (r & 7)) << 4));
-              *reinterpret_cast<uint4*>((uint16_t*)p.out + (s0 + c_lo + r) * p.M + (half ? x1 : x0) + 8 * jj) = v;
+          for (int v = 0; v < 8; ++v) {
+            const int i = v >> 1, b = v & 1;
+            const int row = 8 * i + 2 * (lane & 3) + b;
+            const float a0 = __uint_as_float(r0[4 * i + b]), a1 = __uint_as_float(r0[4 * i + 2 + b]);
+            const float c0 = __uint_as_float(r1[4 * i + b]), c1 = __uint_as_float(r1[4 * i + 2 + b]);
+            const float2 w0v = __fmul2_rn(make_float2(a0, gu ? c0 : a1), make_float2(alpha, alpha));
+            const float2 w1v = __fmul2_rn(make_float2(gu ? a1 : c0, c1), make_float2(gu ? alpha_u : alpha, gu ? alpha_u : alpha));
+            if (row < nblk) {
+              uint16_t* yr = yb + (int64_t)row * p.M;
+              *reinterpret_cast<__nv_bfloat162*>(yr + base0 + 2 * w0) = __floats2bfloat162_rn(w0v.x, w0v.y);
+              *reinterpret_cast<__nv_bfloat162*>(yr + base1 + 2 * w1) = __floats2bfloat162_rn(w1v.x, w1v.y);
             }
           }
         }
