@@ -326,6 +326,21 @@ moesq_status moesq_grouped_gemm_workspace_size(const moesq_linear* W, int64_t S,
 moesq_status moesq_set_gemm_pair_limit(int32_t max_pairs);
 moesq_status moesq_gemm_launch_pairs(int32_t dense, int32_t epilogue, int32_t* pairs);
 
+/* Work-item width of the sparse SwiGLU gate_up GEMM (the pages have no counterpart).
+ * A work item is one weight-tile pair times one 128-token tile, or, on large batches,
+ * two 128-token tiles of one expert computed by single MMAs of N <= 256 ("wide" items:
+ * the weight tile is read from shared memory once per 256 tokens).  Wide items need
+ * K % 512 == 0; without a forced width they are chosen when K >= 4096 and
+ * S >= 256 * E.  The result
+ * of a GEMM does not depend on the width.
+ *   moesq_set_gemm_tiles_per_item: 0 = choose (the default), 1 = one tile, 2 = wide
+ *     wherever the shape allows, for every later launch in the process; tiles in 0..2.
+ *   moesq_gemm_tiles_per_item: the width (1 or 2) that a launch with these arguments
+ *     would use now (dense != 0: the dense comparison kernel, always 1). */
+moesq_status moesq_set_gemm_tiles_per_item(int32_t tiles);
+moesq_status moesq_gemm_tiles_per_item(int32_t dense, int32_t epilogue, int64_t K, int64_t E, int64_t S,
+                                       int32_t* tiles);
+
 /* Dense comparison GEMM: the same grouped GEMM, epilogues and argument meanings on
  * dense NVFP4 weights, the pages' alternative storage ("--no-sparse-storage writes
  * dense packed NVFP4 with the pruned elements zeroed", Usage of the MoESQ repository

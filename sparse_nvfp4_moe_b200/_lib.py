@@ -64,6 +64,8 @@ _SIGS = {
     "moesq_sf_expand_block16": (ctypes.c_int, [c_vp, c_vp, c_i64, c_vp]),
     "moesq_set_gemm_pair_limit": (ctypes.c_int, [c_i32]),
     "moesq_gemm_launch_pairs": (ctypes.c_int, [c_i32, c_i32, ctypes.POINTER(c_i32)]),
+    "moesq_set_gemm_tiles_per_item": (ctypes.c_int, [c_i32]),
+    "moesq_gemm_tiles_per_item": (ctypes.c_int, [c_i32, c_i32, c_i64, c_i64, c_i64, ctypes.POINTER(c_i32)]),
     "moesq_selftest_wait_timeout": (ctypes.c_int, [c_vp, c_i64, c_vp, c_vp]),
     "moesq_gather_act": (ctypes.c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp]),
     "moesq_grouped_gemm_workspace_size": (ctypes.c_int, [ctypes.POINTER(Linear), c_i64,
@@ -274,4 +276,15 @@ def moesq_gemm_launch_pairs(dense, epilogue):
     """CTA pairs the next grouped-GEMM launch on the current device would use."""
     n = c_i32(0)
     _check("moesq_gemm_launch_pairs", lib().moesq_gemm_launch_pairs(dense, epilogue, ctypes.byref(n)))
+    return n.value
+
+
+def moesq_set_gemm_tiles_per_item(tiles):
+    _check("moesq_set_gemm_tiles_per_item", lib().moesq_set_gemm_tiles_per_item(tiles))
+
+
+def moesq_gemm_tiles_per_item(dense, epilogue, K, E, S):
+    """Token tiles per work item (1, or 2 for wide items) a grouped-GEMM launch would use."""
+    n = c_i32(0)
+    _check("moesq_gemm_tiles_per_item", lib().moesq_gemm_tiles_per_item(dense, epilogue, K, E, S, ctypes.byref(n)))
     return n.value

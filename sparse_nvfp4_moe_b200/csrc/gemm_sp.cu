@@ -28,7 +28,11 @@
 //     an output, or two neighbouring outputs) and no lanes exchange values;
 //   * fuses the epilogue: FP32 or bf16 output per slot, or SwiGLU followed by
 //     NVFP4 requantisation written straight into the next GEMM's B operand
-//     layout (codes + 512-byte scale blocks).
+//     layout (codes + 512-byte scale blocks);
+//   * on large batches runs the SwiGLU GEMM on wide items: two token tiles of an
+//     expert per item, one MMA of N <= 256 per K step, so the weight tile is read
+//     from shared memory once per 256 tokens (accumulators of consecutive items
+//     overlap in TMEM, see namespace wide).
 //
 // The same kernel, with a dense stage geometry (256-deep stages of four dense
 // kind::mxf4nvf4 MMAs, no metadata), is the dense comparison GEMM on decoded
@@ -83,6 +87,27 @@ constexpr int EPI_THREADS = 32 * EPI_WARPS;
 constexpr int THREADS = 64 + EPI_THREADS;  // producer warp, MMA warp, epilogue warps
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_ACC = 0, TM_E = 256, TM_SFA = 264, TM_SFB = 280;
+// Wide items (the SwiGLU gate_up GEMM on large batches): a work item is one weight-tile
+// pair and two 128-token tiles of an expert, and each 128-deep step is ONE MMA with
+// N = 256, so the weight tile is read from shared memory once for 256 tokens: a stage
+// moves 58 KB into each SM (weights 22 KB, the CTA's 128 token rows 32 KB, the two
+// 128-row token scale blocks 4 KB) and its MMAs read 48 KB, against 80 KB of copies
+// and reads for the same work in two one-tile items.  Two 256-column accumulators do
+// not fit in TMEM beside the metadata and scales, so the accumulators of consecutive
+// items overlap: items alternate between columns 0-255 and 128-383, and the next item's
+// MMAs start as soon as the epilogue has read the shared columns 128-255 (one token
+// tile), while the other tile's columns stay untouched until the item after it.
+namespace wide {
+constexpr int STAGES = 3;
+constexpr int A_BYTES = Geo<false>::A_BYTES, E_BYTES = Geo<false>::E_BYTES;
+constexpr int B_CHUNK = BN * 128;  // 128 token rows of one 256-deep chunk (SW128)
+constexpr int B_BYTES = 2 * B_CHUNK;
+constexpr int OFF_E = A_BYTES + B_BYTES, OFF_SFA = OFF_E + E_BYTES, OFF_SFB = OFF_SFA + SF_BYTES;
+constexpr int STAGE_BYTES = OFF_SFB + 2 * SF_BYTES;  // 59392
+constexpr int EPI_BYTES = 4096;                      // the SwiGLU epilogue's amax swaps and code multipliers
+constexpr uint32_t TM_E = 384, TM_SFA = 392, TM_SFB = 408;  // SFB: 8 columns per MMA (token rows 0-127, 128-255)
+static_assert(TM_SFB + 32 <= TMEM_COLS && STAGE_BYTES % 1024 == 0, "wide geometry");
+}  // namespace wide
 
 struct Params {
   const uint8_t* meta;
@@ -123,7 +148,12 @@ template <bool DENSE>
 constexpr size_t smem_bytes() {
   return 1024 /*align*/ + (size_t)Geo<DENSE>::STAGES * stage_bytes<DENSE>() + EPI_BYTES + sizeof(Smem);
 }
-static_assert(smem_bytes<false>() <= 227 * 1024 && smem_bytes<true>() <= 227 * 1024, "shared memory budget");
+constexpr size_t smem_bytes_wide() {
+  return 1024 /*align*/ + (size_t)wide::STAGES * wide::STAGE_BYTES + wide::EPI_BYTES + sizeof(Smem);
+}
+static_assert(smem_bytes<false>() <= 227 * 1024 && smem_bytes<true>() <= 227 * 1024 &&
+                  smem_bytes_wide() <= 227 * 1024,
+              "shared memory budget");
 static_assert(Geo<false>::STAGES <= MAX_STAGES && Geo<true>::STAGES <= MAX_STAGES, "barrier arrays");
 
 template <bool DENSE>
@@ -138,6 +168,7 @@ __device__ __forceinline__ uint32_t make_idesc(uint32_t n) {
 
 struct Tile {
   int e, nt, mt, n_rows;
+  int n_rows1;  // wide items: tokens of the second 128-token tile (0: none)
   int prow;  // first padded row of the token tile
   int s0;    // first routed slot of the token tile
 };
@@ -171,6 +202,7 @@ struct TileWalk {
 // the next expert does not hold tile q either, a binary search over the tile-end
 // prefix sums finds the first expert that does, so a walk over thousands of empty
 // experts (decode batches of a layer with many experts) costs log2(E) loads, not E.
+template <int NT = 1>
 __device__ __forceinline__ Tile decode_tile(const Smem& s, TileWalk& w, int E) {
   if (w.cur.x <= w.q && w.e + 1 < E) {
     if (w.nxt.x > w.q) {
@@ -193,11 +225,12 @@ __device__ __forceinline__ Tile decode_tile(const Smem& s, TileWalk& w, int E) {
   Tile t;
   t.e = w.e;
   t.mt = w.m;
-  t.nt = w.q - (r.x - (r.w + BN - 1) / BN);
-  const int rem = r.w - t.nt * BN;
+  t.nt = w.q - (r.x - (r.w + NT * BN - 1) / (NT * BN));
+  const int rem = r.w - t.nt * (NT * BN);
   t.n_rows = rem < BN ? rem : BN;
-  t.prow = r.z + t.nt * BN;
-  t.s0 = r.y + t.nt * BN;
+  t.n_rows1 = NT == 2 ? (rem - BN < 0 ? 0 : (rem - BN < BN ? rem - BN : BN)) : 0;
+  t.prow = r.z + t.nt * (NT * BN);
+  t.s0 = r.y + t.nt * (NT * BN);
   return t;
 }
 
@@ -209,7 +242,7 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-template <int EPI, bool DENSE>
+template <int EPI, bool DENSE, int NT = 1>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     k_grouped_gemm_sp(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                       const __grid_constant__ CUtensorMap tmap_b16, const __grid_constant__ CUtensorMap tmap_e,
@@ -217,12 +250,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                       const __grid_constant__ CUtensorMap tmap_y, const __grid_constant__ CUtensorMap tmap_b_3d,
                       const Params p) {
   using G = Geo<DENSE>;
-  constexpr int STAGES = G::STAGES, STAGE_BYTES = stage_bytes<DENSE>();
-  constexpr int A_BYTES = G::A_BYTES, B_BYTES = G::B_BYTES, E_BYTES = G::E_BYTES;
+  static_assert(NT == 1 || (NT == 2 && !DENSE && EPI == MOESQ_EPI_SWIGLU_NVFP4), "wide items: SwiGLU gate_up");
+  constexpr int STAGES = NT == 2 ? wide::STAGES : G::STAGES;
+  constexpr int STAGE_BYTES = NT == 2 ? wide::STAGE_BYTES : stage_bytes<DENSE>();
+  constexpr int A_BYTES = G::A_BYTES, B_BYTES = NT == 2 ? wide::B_BYTES : G::B_BYTES, E_BYTES = G::E_BYTES;
+  constexpr int EPI_SPACE = NT == 2 ? wide::EPI_BYTES : EPI_BYTES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   float* epi = (float*)(smem + STAGES * STAGE_BYTES);
-  Smem& S = *(Smem*)(smem + STAGES * STAGE_BYTES + EPI_BYTES);
+  Smem& S = *(Smem*)(smem + STAGES * STAGE_BYTES + EPI_SPACE);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();  // 0: issues the pair's MMAs
@@ -275,7 +311,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     for (int e0 = 0; e0 < E; e0 += 32) {
       const int e = e0 + lane;
       int v = 0;
-      if (e < E) v = (S.rec[e].w + BN - 1) / BN;
+      if (e < E) v = (S.rec[e].w + NT * BN - 1) / (NT * BN);
       int x = v;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -308,14 +344,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       for (int i = 0; i < STAGES; ++i) full_lead[i] = cluster_map(&S.full[i], 0);
       const bool b3d = !DENSE && (p.K % 256) == 0;  // both 256-deep token chunks of a stage in one 3-D box
       for (int id = pair_id; id < total; id += npairs, walk.advance(MT2)) {
-        const Tile t = decode_tile(S, walk, E);
+        const Tile t = decode_tile<NT>(S, walk, E);
         const int mt = min(2 * t.mt + (int)rank, MT - 1);  // an odd last tile is loaded twice
         int prow = t.prow;
         if (prow < 0 || (int64_t)prow + BN > p.P_cap) {  // inconsistent offsets: stay in bounds
           flag(p.d_status, MOESQ_DFLAG_CAPACITY);
           prow = 0;
         }
-        const int n_mma = max(16, (t.n_rows + 15) / 16 * 16);
+        const int n_mma = max(16, (t.n_rows + (NT == 2 ? t.n_rows1 : 0) + 15) / 16 * 16);
         const int brow = prow + (int)rank * (n_mma / 2);  // this CTA's half of the token rows
         const int wt = t.e * MT + mt;                   // weight tile
         // a tile of <= 32 tokens loads 16-row B boxes (decode-sized groups)
@@ -323,6 +359,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const void* tb = small ? (const void*)&tmap_b16 : (const void*)&tmap_b;
         const void* tb3 = &tmap_b_3d;
         const uint32_t b_box = small ? 16 * 128 : B_CHUNK;
+        // wide items holding two token tiles: this CTA's (up to) 128 token rows of both
+        // 256-deep chunks in one 3-D box of 128 rows, and the second tile's scale block
+        const bool two = NT == 2 && t.n_rows1 > 0;
         for (int kb = 0; kb < nkb; ++kb) {
           mbar_wait_spin(&S.empty[stage], phase ^ 1, abort, p.d_status);
           const int nk = min(4, kb128 - 4 * kb);  // 128-deep MMAs in this stage
@@ -332,13 +371,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int i = 1; i < STAGES; ++i)
             if (stage == i) bar = full_lead[i];
-          if (lead) mbar_arrive_expect_tx(&S.full[stage], 2u * (A_BYTES + nc * b_box + E_BYTES + 2 * SF_BYTES));
+          if constexpr (NT == 2) {
+            if (lead)
+              mbar_arrive_expect_tx(&S.full[stage], two ? 2u * (A_BYTES + B_BYTES + E_BYTES + 3 * SF_BYTES)
+                                                        : 2u * (A_BYTES + nc * b_box + E_BYTES + 2 * SF_BYTES));
+          } else {
+            if (lead) mbar_arrive_expect_tx(&S.full[stage], 2u * (A_BYTES + nc * b_box + E_BYTES + 2 * SF_BYTES));
+          }
           // weight tile in the repack's interleaved row order: gate and up rows of
           // outputs 64mt..64mt+63 in one 5-D box (byte, j, gate/up, h, 16-row group), or
           // down rows 128mt.. in one 4-D box (byte, j, p, 16-row group)
           if (p.gate_up) tma_load_5d_pair(st, &tmap_a, kb * 128, 0, 0, 0, t.e * (p.M / 16) + 4 * mt, bar);
           else tma_load_4d_pair(st, &tmap_a, kb * 128, 0, 0, (t.e * p.M + BM * mt) / 16, bar);
-          if (b3d && nc > 1 && !small) {  // 64-row chunks: chunk 1 lands at B_CHUNK as the MMA expects
+          if constexpr (NT == 2) {  // chunk 1 lands at wide::B_CHUNK (K % 512 == 0: nc == 2)
+            if (two) {
+              tma_load_3d_pair(st + A_BYTES, tb3, 0, brow, 2 * kb, bar);
+            } else {
+              tma_load_2d_pair(st + A_BYTES, tb, kb * 256, brow, bar);
+              tma_load_2d_pair(st + A_BYTES + wide::B_CHUNK, tb, kb * 256 + 128, brow, bar);
+            }
+          } else if (b3d && nc > 1 && !small) {  // 64-row chunks: chunk 1 lands at B_CHUNK as the MMA expects
             tma_load_3d_pair(st + A_BYTES, tb3, 0, brow, 2 * kb, bar);
           } else {
             tma_load_2d_pair(st + A_BYTES, tb, kb * (G::BK / 2), brow, bar);
@@ -350,6 +402,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           tma_load_2d_pair(st + A_BYTES + B_BYTES + E_BYTES, &tmap_sfa, 0, (wt * kb128 + 4 * kb) * 2, bar);
           tma_load_2d_pair(st + A_BYTES + B_BYTES + E_BYTES + SF_BYTES, &tmap_sfb, 0,
                            ((prow / 128) * kb128 + 4 * kb) * 2, bar);
+          if (two)
+            tma_load_2d_pair(st + A_BYTES + B_BYTES + E_BYTES + 2 * SF_BYTES, &tmap_sfb, 0,
+                             ((prow / 128 + 1) * kb128 + 4 * kb) * 2, bar);
           ++fills;
           if (++stage == STAGES) {
             stage = 0;
@@ -386,13 +441,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       const uint64_t dE2 = smem_desc(s0 + A_BYTES + B_BYTES, BM * 16, 128, SWZ_NONE);  // LBO = chunk stride
       const uint64_t dSFA0 = smem_desc(s0 + A_BYTES + B_BYTES + E_BYTES, 16, 128, SWZ_NONE);
       const uint64_t dSFB0 = dSFA0 + (SF_BYTES >> 4);
-      const uint32_t tE = tmem + TM_E, tSFA = tmem + TM_SFA, tSFB = tmem + TM_SFB;
+      const uint32_t tE = tmem + (NT == 2 ? wide::TM_E : TM_E), tSFA = tmem + (NT == 2 ? wide::TM_SFA : TM_SFA);
+      const uint32_t tSFB = tmem + TM_SFB;
       TileWalk walk(S, pair_id, npairs, MT2, E);
+      int wpar = 0;  // wide items: accumulator at columns 128 * wpar, alternating per item
       for (int id = pair_id; id < total; id += npairs, walk.advance(MT2)) {
-        const Tile t = decode_tile(S, walk, E);
-        const int n_mma = max(16, (t.n_rows + 15) / 16 * 16);
+        const Tile t = decode_tile<NT>(S, walk, E);
+        const int n_mma = max(16, (t.n_rows + (NT == 2 ? t.n_rows1 : 0) + 15) / 16 * 16);
         const uint32_t idesc = make_idesc<DENSE>((uint32_t)n_mma);
-        const uint32_t d_tmem = tmem + TM_ACC + buf * BN;
+        const uint32_t d_tmem = tmem + TM_ACC + (NT == 2 ? wpar * BN : buf * BN);
+        const bool two = NT == 2 && t.n_rows1 > 0;
         mbar_wait_spin(&S.acc_empty[buf], ((acc_phase >> buf) & 1u) ^ 1u, abort, p.d_status);
         tc_fence_after();
         for (int kb = 0; kb < nkb; ++kb) {
@@ -400,7 +458,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           tc_fence_after();
           const uint64_t so = (uint64_t)((stage * STAGE_BYTES) >> 4);
           const int nk = min(4, kb128 - 4 * kb);
-          if constexpr (DENSE) {
+          if constexpr (NT == 2) {
+            // one MMA of N <= 256 per 128 dense K.  The token scales of MMA j take eight
+            // TMEM columns: column c holds rows 32c..32c+31 (lane = row % 32, byte =
+            // scale), so the second tile's block (rows 128..255) goes to columns 4..7.
+            const uint32_t tSFBw = tmem + wide::TM_SFB;
+            tc_cp_pair_128x256b(tE, dE2 + so);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              tc_cp_pair_32x128b_warpx4(tSFA + 4 * j, dSFA0 + so + (uint64_t)(j * (512 >> 4)));
+              tc_cp_pair_32x128b_warpx4(tSFBw + 8 * j, dSFB0 + so + (uint64_t)(j * (512 >> 4)));
+              if (two)
+                tc_cp_pair_32x128b_warpx4(tSFBw + 8 * j + 4, dSFB0 + so + (uint64_t)((SF_BYTES + j * 512) >> 4));
+              tc_mma_pair_sp_nvf4(d_tmem, dA0 + so + (uint64_t)(j * 2),
+                                  dB0 + so + (uint64_t)((j >> 1) * (wide::B_CHUNK >> 4) + (j & 1) * 4), tE + 2 * j,
+                                  idesc, tSFA + 4 * j, tSFBw + 8 * j, (kb > 0 || j > 0) ? 1u : 0u);
+            }
+          } else if constexpr (DENSE) {
             // dense MMAs of 64 dense K: A and B each advance 32 B inside their
             // 128-byte swizzle rows; one scale block per MMA and operand
 #pragma unroll
@@ -449,7 +523,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
         tc_commit_pair_mc(&S.acc_full[buf], 0x3);
         acc_phase ^= 1u << buf;
-        buf ^= 1;
+        if constexpr (NT == 1) buf ^= 1;  // wide items: one barrier pair, alternating columns
+        wpar ^= 1;
       }
       // drain: all tensor-core work of the pair complete before TMEM is freed
       tc_commit_pair_mc(&S.done, 0x1);
@@ -477,15 +552,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     };
     TileWalk walk(S, pair_id, npairs, MT2, E);
     int sb = 0;  // SwiGLU staging buffer of this tile
+    [[maybe_unused]] int wpar = 0;  // wide items: accumulator at columns 128 * wpar
     // the next tile is decoded while this one drains (a chain of shared-memory
     // loads that would otherwise stand alone between tiles)
-    Tile tn = pair_id < total ? decode_tile(S, walk, E) : Tile{};
+    Tile tn = pair_id < total ? decode_tile<NT>(S, walk, E) : Tile{};
     for (int id = pair_id; id < total; id += npairs) {
       const Tile t = tn;
       auto decode_next = [&]() {
         if (id + npairs < total) {
           walk.advance(MT2);
-          tn = decode_tile(S, walk, E);
+          tn = decode_tile<NT>(S, walk, E);
         }
       };
       const int mt = 2 * t.mt + (int)rank;  // this CTA's weight tile
@@ -508,101 +584,154 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // = alpha g / (1 + 2^(g * (-alpha log2 e))), so alpha enters the exponent's
         // multiplier and the product alpha * alpha_u enters the amax and the code
         // multiplier below (a few ulp of reassociation, no multiply per element)
-        float hv[2][8];  // [h][v]: v = 2i + b
         const float ch = __fmul_rn(alpha, alpha_u);
-        if (live) {
+        const float ce = __fmul_rn(alpha, -1.4426950408889634f);
+        auto load_h = [&](uint32_t tcol, float (&h_)[2][8]) {
           uint32_t r[16];
-          const float ce = __fmul_rn(alpha, -1.4426950408889634f);
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            tmem_ld_16x256b_x4(tbase + ((uint32_t)(16 * h) << 16) + c_lo, r);
+            tmem_ld_16x256b_x4(tcol + ((uint32_t)(16 * h) << 16), r);
             tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 4; ++i) {  // columns b = 0, 1 as one packed pair
               const float2 g = make_float2(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]));
               const float2 u = make_float2(__uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
               const float2 hh = __fmul2_rn(sigmoid_scaled2(g, ce), u);
-              hv[h][2 * i] = hh.x;
-              hv[h][2 * i + 1] = hh.y;
+              h_[h][2 * i] = hh.x;
+              h_[h][2 * i + 1] = hh.y;
             }
           }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) release_acc(buf);
-        decode_next();
-        if (live) {
-          // amax of each column over this warp's 16 outputs: per thread over its two,
-          // then over the 8 lanes of equal t%4 (lane bits 2..4) by three halving
-          // exchanges; lane t ends with column v = (t >> 2) & 7 of its own t%4
-          float m[8];
-#pragma unroll
-          for (int v = 0; v < 8; ++v) m[v] = fmaxf(fabsf(hv[0][v]), fabsf(hv[1][v]));
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const bool hi = lane & 16;
-            const float x = __shfl_xor_sync(0xffffffffu, hi ? m[k] : m[k + 4], 16);
-            m[k] = fmaxf(hi ? m[k + 4] : m[k], x);
+        };
+        float hv[2][8];  // [h][v]: v = 2i + b
+        [[maybe_unused]] const bool live1 = NT == 2 && c_lo < t.n_rows1;
+        if constexpr (NT == 2) {
+          // the tile in the shared columns 128-255 (tile 1 at wpar 0, tile 0 at wpar 1)
+          // is read first, raw, and the accumulator released; then SiLU, and the other tile
+          const uint32_t tsh = tmem + TM_ACC + BN + ((uint32_t)(32 * q) << 16) + c_lo;
+          const bool live_sh = wpar ? live : live1;
+          uint32_t ra[16], rb[16];
+          if (live_sh) {
+            tmem_ld_16x256b_x4(tsh, ra);
+            tmem_ld_16x256b_x4(tsh + (16u << 16), rb);
+            tmem_ld_wait();
           }
-#pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            const bool hi = lane & 8;
-            const float x = __shfl_xor_sync(0xffffffffu, hi ? m[k] : m[k + 2], 8);
-            m[k] = fmaxf(hi ? m[k + 2] : m[k], x);
-          }
-          {
-            const bool hi = lane & 4;
-            const float x = __shfl_xor_sync(0xffffffffu, hi ? m[0] : m[1], 4);
-            m[0] = fmaxf(hi ? m[1] : m[0], x);
-          }
-          // the scale group (32 outputs) spans quarters q and q ^ 1, which use the
-          // same lane -> column map: swap the partial amax through shared memory
-          float* xa = epi + (kb * 4 + q) * 32;
-          xa[lane] = m[0];
-          named_bar_sync(2 + (q >> 1) + 2 * kb, 64);
-          const float amax = __fmul_rn(fmaxf(m[0], epi[(kb * 4 + (q ^ 1)) * 32 + lane]), fabsf(ch));
-          const GroupScale gs = nvfp4_group_scale(amax, ag.y);
-          // code multiplier of column (lane >> 2) & 7 for the scaled hv, transposed through
-          // shared memory so that each thread reads its 8 columns with two vector loads
-          float* xi = epi + 512 + ew * 32;
-          xi[(lane & 3) * 8 + ((lane >> 2) & 7)] = __fmul_rn(gs.inv, ch);
+          tc_fence_before();
           __syncwarp();
-          const float4 iv0 = *reinterpret_cast<const float4*>(xi + (lane & 3) * 8);
-          const float4 iv1 = *reinterpret_cast<const float4*>(xi + (lane & 3) * 8 + 4);
-          const float ivs[8] = {iv0.x, iv0.y, iv0.z, iv0.w, iv1.x, iv1.y, iv1.z, iv1.w};
-          const int vc = (lane >> 2) & 7;
-          const int rc = 8 * (vc >> 1) + 2 * (lane & 3) + (vc & 1);  // this lane's column (row of the block)
-          if ((q & 1) == 0) S.sstg[sb][kb][rc][q >> 1] = (uint8_t)gs.sc;
-          // codes: byte 8q + t/4 of each of this thread's 8 token rows (outputs 2(t/4) + {0,1})
-          uint8_t* stg = &S.hstg[sb][kb][0][8 * q + (lane >> 2)];
+          if (lane == 0) release_acc(0);
+          decode_next();
+          auto silu = [&](const uint32_t (&r)[16], float (&h_)[8]) {
 #pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            const float inv = ivs[v];
-            const float2 x = __fmul2_rn(make_float2(hv[0][v], hv[1][v]), make_float2(inv, inv));
-            const uint32_t byte = inv == 0.0f ? 0u : e2m1x2(x.x, x.y);
-            stg[(8 * (v >> 1) + 2 * (lane & 3) + (v & 1)) * 32] = (uint8_t)byte;
+            for (int i = 0; i < 4; ++i) {
+              const float2 g = make_float2(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]));
+              const float2 u = make_float2(__uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+              const float2 hh = __fmul2_rn(sigmoid_scaled2(g, ce), u);
+              h_[2 * i] = hh.x;
+              h_[2 * i + 1] = hh.y;
+            }
+          };
+          if (live_sh) {
+            silu(ra, hv[0]);
+            silu(rb, hv[1]);
           }
+        } else {
+          if (live) load_h(tbase + c_lo, hv);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) release_acc(buf);
+          decode_next();
         }
-        // the four warps of this column block hold all 64 outputs of its 32 tokens:
-        // one TMA store of [32 rows][32 B] codes (rows past the expert's tokens are its
-        // own padding, never read as tokens) and 2-byte scale pairs
-        fence_proxy_async_smem();
-        if (q == 2 && lane == 0) bulk_wait_group_read0();  // the store two tiles back has read its buffer
-        named_bar_sync(10 + kb, 128);  // also: both amax slots of every pair are read
-        if (live) {
-          const int64_t prow0 = (int64_t)t.prow + c_lo;
-          if (q == 2 && lane == 0) {
-            tma_store_2d(&tmap_y, &S.hstg[sb][kb][0][0], 32 * mt, (int32_t)prow0);
-            bulk_commit_group();
+        // amax, scales, codes and stores of one token tile (rows prow_t.., n_t tokens)
+        auto finish = [&](const float (&hv)[2][8], int prow_t, int n_t, bool live) {
+          if (live) {
+            // amax of each column over this warp's 16 outputs: per thread over its two,
+            // then over the 8 lanes of equal t%4 (lane bits 2..4) by three halving
+            // exchanges; lane t ends with column v = (t >> 2) & 7 of its own t%4
+            float m[8];
+#pragma unroll
+            for (int v = 0; v < 8; ++v) m[v] = fmaxf(fabsf(hv[0][v]), fabsf(hv[1][v]));
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const bool hi = lane & 16;
+              const float x = __shfl_xor_sync(0xffffffffu, hi ? m[k] : m[k + 4], 16);
+              m[k] = fmaxf(hi ? m[k + 4] : m[k], x);
+            }
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+              const bool hi = lane & 8;
+              const float x = __shfl_xor_sync(0xffffffffu, hi ? m[k] : m[k + 2], 8);
+              m[k] = fmaxf(hi ? m[k + 2] : m[k], x);
+            }
+            {
+              const bool hi = lane & 4;
+              const float x = __shfl_xor_sync(0xffffffffu, hi ? m[0] : m[1], 4);
+              m[0] = fmaxf(hi ? m[1] : m[0], x);
+            }
+            // the scale group (32 outputs) spans quarters q and q ^ 1, which use the
+            // same lane -> column map: swap the partial amax through shared memory
+            float* xa = epi + (kb * 4 + q) * 32;
+            xa[lane] = m[0];
+            named_bar_sync(2 + (q >> 1) + 2 * kb, 64);
+            const float amax = __fmul_rn(fmaxf(m[0], epi[(kb * 4 + (q ^ 1)) * 32 + lane]), fabsf(ch));
+            const GroupScale gs = nvfp4_group_scale(amax, ag.y);
+            // code multiplier of column (lane >> 2) & 7 for the scaled hv, transposed through
+            // shared memory so that each thread reads its 8 columns with two vector loads
+            float* xi = epi + 512 + ew * 32;
+            xi[(lane & 3) * 8 + ((lane >> 2) & 7)] = __fmul_rn(gs.inv, ch);
+            __syncwarp();
+            const float4 iv0 = *reinterpret_cast<const float4*>(xi + (lane & 3) * 8);
+            const float4 iv1 = *reinterpret_cast<const float4*>(xi + (lane & 3) * 8 + 4);
+            const float ivs[8] = {iv0.x, iv0.y, iv0.z, iv0.w, iv1.x, iv1.y, iv1.z, iv1.w};
+            const int vc = (lane >> 2) & 7;
+            const int rc = 8 * (vc >> 1) + 2 * (lane & 3) + (vc & 1);  // this lane's column (row of the block)
+            if ((q & 1) == 0) S.sstg[sb][kb][rc][q >> 1] = (uint8_t)gs.sc;
+            // codes: byte 8q + t/4 of each of this thread's 8 token rows (outputs 2(t/4) + {0,1})
+            uint8_t* stg = &S.hstg[sb][kb][0][8 * q + (lane >> 2)];
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              const float inv = ivs[v];
+              const float2 x = __fmul2_rn(make_float2(hv[0][v], hv[1][v]), make_float2(inv, inv));
+              const uint32_t byte = inv == 0.0f ? 0u : e2m1x2(x.x, x.y);
+              stg[(8 * (v >> 1) + 2 * (lane & 3) + (v & 1)) * 32] = (uint8_t)byte;
+            }
           }
-          if (q == 3 && lane < t.n_rows - c_lo) {
-            const int64_t prow = prow0 + lane;
-            const int64_t blk = (prow / 128) * (I / 128) + (64 * mt) / 128;
-            *reinterpret_cast<uint16_t*>(p.out_sf + blk * 512 + sf_block_offset((uint32_t)(prow % 128), 2u * (mt & 1))) =
-                *reinterpret_cast<const uint16_t*>(&S.sstg[sb][kb][lane][0]);
+          // the four warps of this column block hold all 64 outputs of its 32 tokens:
+          // one TMA store of [32 rows][32 B] codes (rows past the expert's tokens are its
+          // own padding, never read as tokens) and 2-byte scale pairs
+          fence_proxy_async_smem();
+          if (q == 2 && lane == 0) bulk_wait_group_read0();  // the store two tiles back has read its buffer
+          named_bar_sync(10 + kb, 128);  // also: both amax slots of every pair are read
+          if (live) {
+            const int64_t prow0 = (int64_t)prow_t + c_lo;
+            if (q == 2 && lane == 0) {
+              tma_store_2d(&tmap_y, &S.hstg[sb][kb][0][0], 32 * mt, (int32_t)prow0);
+              bulk_commit_group();
+            }
+            if (q == 3 && lane < n_t - c_lo) {
+              const int64_t prow = prow0 + lane;
+              const int64_t blk = (prow / 128) * (I / 128) + (64 * mt) / 128;
+              *reinterpret_cast<uint16_t*>(p.out_sf + blk * 512 + sf_block_offset((uint32_t)(prow % 128), 2u * (mt & 1))) =
+                  *reinterpret_cast<const uint16_t*>(&S.sstg[sb][kb][lane][0]);
+            }
           }
+          sb ^= 1;
+        };
+        if constexpr (NT == 2) {
+          // the shared-column tile first (its values are in hv), then the other one
+          if (wpar) {
+            finish(hv, t.prow, t.n_rows, live);
+            if (t.n_rows1 > 0) {
+              if (live1) load_h(tbase + 2 * BN + c_lo, hv);
+              finish(hv, t.prow + BN, t.n_rows1, live1);
+            }
+          } else {
+            if (t.n_rows1 > 0) finish(hv, t.prow + BN, t.n_rows1, live1);
+            if (live) load_h(tbase + c_lo, hv);
+            finish(hv, t.prow, t.n_rows, live);
+          }
+          wpar ^= 1;
+        } else {
+          finish(hv, t.prow, t.n_rows, live);
         }
-        sb ^= 1;
       } else if constexpr (EPI == MOESQ_EPI_BF16) {
         // Per 32-token column block kb, its four warps (one per lane quarter q) write
         // [32 tokens][128 outputs] bf16.  The interleaved weight rows put both outputs of
@@ -742,7 +871,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
       }
       acc_phase ^= 1u << buf;
-      buf ^= 1;
+      if constexpr (NT == 1) buf ^= 1;
     }
   }
 
@@ -822,17 +951,34 @@ extern "C" moesq_status moesq_grouped_gemm_workspace_size(const moesq_linear* W,
 
 // Upper bound on the CTA pairs a grouped GEMM launches (0: none), process-wide.
 static std::atomic<int> g_pair_limit{0};
+// Token tiles per work item of the sparse SwiGLU GEMM: 0 chooses, 1 or 2 forces
+// (2 where the shape allows wide items), process-wide.
+static std::atomic<int> g_tiles_per_item{0};
+
+// Wide items (two 128-token tiles, one N <= 256 MMA per K step) for the sparse SwiGLU
+// gate_up GEMM: K a multiple of 512 (whole stages, so both token chunks of every
+// stage are loaded).  Unless forced they are chosen for K >= 4096 and an average of
+// 256 or more routed slots per expert, where most items hold two full tiles: with
+// K = 2048 an item's main loop is too short to cover the two-tile SwiGLU epilogue,
+// which then bounds the GEMM (measured 10 % slower than one-tile items there).
+static int tiles_per_item(bool dense, int32_t epilogue, int64_t K, int64_t E, int64_t S) {
+  if (dense || epilogue != MOESQ_EPI_SWIGLU_NVFP4 || K % 512 != 0) return 1;
+  const int f = g_tiles_per_item.load(std::memory_order_relaxed);
+  if (f) return f;
+  return K >= 4096 && S >= 256 * E ? 2 : 1;
+}
 
 // CTA pairs of a launch: clusters of 2 CTAs, one CTA per SM, as many pairs as the
-// device can hold at once (cached per device and epilogue), capped by g_pair_limit.
+// device can hold at once (cached per device and kernel), capped by g_pair_limit.
 template <bool DENSE>
-static moesq_status launch_pairs(int dev, int sms, int32_t epilogue, int* pairs_out) {
-  constexpr size_t smem = sp::smem_bytes<DENSE>();
-  static int pairs_cache[64][3] = {{0}};
-  const int ei = epilogue - MOESQ_EPI_F32;
+static moesq_status launch_pairs(int dev, int sms, int32_t epilogue, int* pairs_out, bool wide = false) {
+  const size_t smem = wide ? sp::smem_bytes_wide() : sp::smem_bytes<DENSE>();
+  static int pairs_cache[64][4] = {{0}};
+  const int ei = wide ? 3 : epilogue - MOESQ_EPI_F32;
   int pairs = dev < 64 ? pairs_cache[dev][ei] : 0;
   if (pairs == 0) {
-    const void* fn = epilogue == MOESQ_EPI_F32 ? (const void*)sp::k_grouped_gemm_sp<MOESQ_EPI_F32, DENSE>
+    const void* fn = wide ? (const void*)sp::k_grouped_gemm_sp<MOESQ_EPI_SWIGLU_NVFP4, false, 2>
+                     : epilogue == MOESQ_EPI_F32 ? (const void*)sp::k_grouped_gemm_sp<MOESQ_EPI_F32, DENSE>
                      : epilogue == MOESQ_EPI_BF16 ? (const void*)sp::k_grouped_gemm_sp<MOESQ_EPI_BF16, DENSE>
                                                   : (const void*)sp::k_grouped_gemm_sp<MOESQ_EPI_SWIGLU_NVFP4, DENSE>;
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
@@ -936,6 +1082,14 @@ static moesq_status grouped_gemm_impl(const moesq_linear* W, const uint8_t* act_
     const cuuint32_t box64[3] = {128, 64, 2};
     if (!make_tmap_u8(&tb3, act_codes, 3, dims, strides, box64, CU_TENSOR_MAP_SWIZZLE_128B)) return MOESQ_ERR_CUDA;
   }
+  // wide items: a CTA's 128 rows of both chunks in one box (32 KB)
+  const bool wide = tiles_per_item(DENSE, epilogue, W->K, W->E, S) == 2;
+  if (wide) {
+    const cuuint64_t dims[3] = {128, (uint64_t)P_cap, (uint64_t)(W->K / 256)};
+    const cuuint64_t strides[2] = {(uint64_t)(W->K / 2), 128};
+    const cuuint32_t box128[3] = {128, 128, 2};
+    if (!make_tmap_u8(&tb3, act_codes, 3, dims, strides, box128, CU_TENSOR_MAP_SWIZZLE_128B)) return MOESQ_ERR_CUDA;
+  }
   // metadata and scale blocks seen as 256-byte rows (no swizzle: contiguous copies)
   te = ta;  // unused by the dense kernel
   if ((!DENSE && !make_tmap_rows(&te, W->meta, 256, (uint64_t)(W->E * MT * nkb256 * 8), 256, 16,
@@ -965,9 +1119,9 @@ static moesq_status grouped_gemm_impl(const moesq_linear* W, const uint8_t* act_
       return MOESQ_ERR_CUDA;
   }
 
-  constexpr size_t smem = sp::smem_bytes<DENSE>();
+  const size_t smem = wide ? sp::smem_bytes_wide() : sp::smem_bytes<DENSE>();
   int pairs = 0;
-  const moesq_status pst = launch_pairs<DENSE>(dev, sms, epilogue, &pairs);
+  const moesq_status pst = launch_pairs<DENSE>(dev, sms, epilogue, &pairs, wide);
   if (pst != MOESQ_OK) return pst;
   sp::Params prm;
   prm.meta = W->meta;
@@ -1002,8 +1156,12 @@ static moesq_status grouped_gemm_impl(const moesq_linear* W, const uint8_t* act_
                          tb16, te, tsfa, tsfb, ty, tb3, prm);
       break;
     default:
-      err = moesq_launch(sp::k_grouped_gemm_sp<MOESQ_EPI_SWIGLU_NVFP4, DENSE>, grid, dim3(sp::THREADS), smem, st,
-                         ta, tb, tb16, te, tsfa, tsfb, ty, tb3, prm);
+      if (wide)
+        err = moesq_launch(sp::k_grouped_gemm_sp<MOESQ_EPI_SWIGLU_NVFP4, false, 2>, grid, dim3(sp::THREADS), smem,
+                           st, ta, tb, tb16, te, tsfa, tsfb, ty, tb3, prm);
+      else
+        err = moesq_launch(sp::k_grouped_gemm_sp<MOESQ_EPI_SWIGLU_NVFP4, DENSE>, grid, dim3(sp::THREADS), smem, st,
+                           ta, tb, tb16, te, tsfa, tsfb, ty, tb3, prm);
   }
   if (err != cudaSuccess) {
     (void)cudaGetLastError();
@@ -1052,4 +1210,18 @@ extern "C" moesq_status moesq_gemm_launch_pairs(int32_t dense, int32_t epilogue,
       dense ? launch_pairs<true>(dev, sms, epilogue, &n) : launch_pairs<false>(dev, sms, epilogue, &n);
   if (st == MOESQ_OK) *pairs = n;
   return st;
+}
+
+extern "C" moesq_status moesq_set_gemm_tiles_per_item(int32_t tiles) {
+  MOESQ_REQUIRE(tiles >= 0 && tiles <= 2, MOESQ_ERR_INVALID_ARG);
+  g_tiles_per_item.store(tiles, std::memory_order_relaxed);
+  return MOESQ_OK;
+}
+
+extern "C" moesq_status moesq_gemm_tiles_per_item(int32_t dense, int32_t epilogue, int64_t K, int64_t E, int64_t S,
+                                                  int32_t* tiles) {
+  MOESQ_REQUIRE(tiles && epilogue >= MOESQ_EPI_F32 && epilogue <= MOESQ_EPI_SWIGLU_NVFP4 && K > 0 && E > 0 && S >= 0,
+                MOESQ_ERR_INVALID_ARG);
+  *tiles = tiles_per_item(dense != 0, epilogue, K, E, S);
+  return MOESQ_OK;
 }

@@ -13,7 +13,14 @@ walk.  The other GEMM tests have fewer items than the device has pairs, so here:
   kernel);
 * a layer whose item list is many times the device's own pair count (32 experts,
   top-4, H = 512, I = 256, 8192 tokens: 512 items per GEMM) runs at the uncapped
-  launch, and the whole layer is compared element by element.
+  launch, and the whole layer is compared element by element;
+* wide items of the SwiGLU gate_up GEMM (two 128-token tiles of one expert, one MMA
+  of N <= 256 per K step, a single 256-column accumulator): forced on layers whose
+  experts hold 0, 7, 40, 128, 129, 250, 256, 300, 517 and 700 tokens, so items with a
+  full and a ragged second tile (N = 144 .. 256), single-tile items of <= 16, <= 64
+  and 128 tokens and empty experts all occur, at 1, 3 and all pairs, with the fold
+  and with separate gate and up globals; the many-item layer runs forced to wide
+  items as well (256 items per pair: the accumulator columns alternate many times).
 
 Tolerances are those of tests/test_gpu_gemm.py (1e-5 * sum|a w| in FP32, one bf16 ulp
 beyond it; requantised codes bit-exact where the NVFP4 rule fixes them).  The grouped
@@ -33,6 +40,12 @@ pytestmark = pytest.mark.gpu
 LIMITS = (1, 2, 3)
 CAPPED = ("tiny", "ragged_multi_tile", "sparse_routing", "mid_ktail", "deep_k", "exact_per_half_alpha")
 MANY = W.LayerConfig("many_items", 46, 32, 4, 512, 256, (8192,), "uniform", True)
+# tokens per expert of the wide-item layers (top-1 routing, built directly)
+WIDE_COUNTS = (0, 7, 40, 128, 129, 250, 256, 300, 517, 700)
+WIDE = {
+    "fold": (W.LayerConfig("wide_fold", 47, 10, 1, 1024, 384, (2327,), "uniform", True), {}),
+    "exact": (W.LayerConfig("wide_exact", 48, 10, 1, 512, 256, (2327,), "uniform", True), dict(exact=True)),
+}
 
 
 def items(layer, out_rows):
@@ -40,6 +53,18 @@ def items(layer, out_rows):
     counts = np.diff(layer.perm["expert_offsets"])
     mt = out_rows // 128
     return int(((counts + 127) // 128).sum()) * ((mt + 1) // 2)
+
+
+class TilesPerItem:
+    def __init__(self, n):
+        self.n = n
+
+    def __enter__(self):
+        M.moesq_set_gemm_tiles_per_item(self.n)
+        return self
+
+    def __exit__(self, *a):
+        M.moesq_set_gemm_tiles_per_item(0)
 
 
 class PairLimit:
@@ -150,3 +175,59 @@ def test_pair_limit_arguments():
     with PairLimit(full + 100):
         assert M.moesq_gemm_launch_pairs(0, M.EPI_BF16) == full
     torch.cuda.synchronize()
+
+
+def test_many_items_swiglu_requant_wide(many_layer):
+    assert M.moesq_gemm_tiles_per_item(0, M.EPI_SWIGLU_NVFP4, MANY.H, MANY.E, many_layer.S) == 1
+    with TilesPerItem(2):
+        assert M.moesq_gemm_tiles_per_item(0, M.EPI_SWIGLU_NVFP4, MANY.H, MANY.E, many_layer.S) == 2
+        TG.test_swiglu_requant_epilogue(many_layer)
+        TG.test_moe_forward_end_to_end(many_layer)
+
+
+def wide_routing(cfg, seed):
+    """Top-1 routing with WIDE_COUNTS tokens per expert, in a seeded token order."""
+    ids = np.repeat(np.arange(cfg.E), WIDE_COUNTS)
+    np.random.default_rng(seed).shuffle(ids)
+    return ids.reshape(-1, 1), np.ones((ids.size, 1), np.float32)
+
+
+@pytest.fixture(scope="module", params=sorted(WIDE))
+def wide_layer(request):
+    cfg, opt = WIDE[request.param]
+    T = int(sum(WIDE_COUNTS))
+    assert cfg.E == len(WIDE_COUNTS) and cfg.H % 512 == 0
+    return TG.Layer(cfg, T, routing=wide_routing(cfg, cfg.seed), **opt)
+
+
+@pytest.mark.parametrize("limit", (0, 1, 3))
+def test_wide_items_swiglu_requant(wide_layer, limit):
+    L = wide_layer
+    with TilesPerItem(2), PairLimit(limit):
+        assert M.moesq_gemm_tiles_per_item(0, M.EPI_SWIGLU_NVFP4, L.cfg.H, L.cfg.E, L.S) == 2
+        TG.test_swiglu_requant_epilogue(L)
+
+
+@pytest.mark.parametrize("limit", (0, 3))
+def test_wide_items_forward(wide_layer, limit):
+    with TilesPerItem(2), PairLimit(limit):
+        TG.test_moe_forward_end_to_end(wide_layer)
+        TG.test_forward_is_deterministic(wide_layer)
+
+
+def test_tiles_per_item_arguments():
+    sw, bf = M.EPI_SWIGLU_NVFP4, M.EPI_BF16
+    for bad in (-1, 3):
+        with pytest.raises(M.MoesqError):
+            M.moesq_set_gemm_tiles_per_item(bad)
+    assert M.moesq_gemm_tiles_per_item(0, sw, 4096, 128, 256 * 128) == 2      # 256 slots per expert
+    assert M.moesq_gemm_tiles_per_item(0, sw, 4096, 128, 256 * 128 - 1) == 1
+    assert M.moesq_gemm_tiles_per_item(0, sw, 4096 + 256, 128, 1 << 20) == 1  # K % 512 != 0
+    assert M.moesq_gemm_tiles_per_item(0, sw, 2048, 128, 1 << 20) == 1        # K < 4096
+    assert M.moesq_gemm_tiles_per_item(0, bf, 4096, 128, 1 << 20) == 1        # SwiGLU only
+    assert M.moesq_gemm_tiles_per_item(1, sw, 4096, 128, 1 << 20) == 1        # sparse only
+    with TilesPerItem(2):
+        assert M.moesq_gemm_tiles_per_item(0, sw, 4096, 128, 1) == 2
+        assert M.moesq_gemm_tiles_per_item(0, sw, 4096 + 256, 128, 1) == 1
+    with TilesPerItem(1):
+        assert M.moesq_gemm_tiles_per_item(0, sw, 4096, 128, 1 << 20) == 1
