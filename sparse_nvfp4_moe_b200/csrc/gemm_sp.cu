@@ -79,6 +79,7 @@ __host__ __device__ constexpr int stage_bytes() {
 }
 constexpr int EPI_BYTES = 32768;  // epilogue space: bf16 staging, f32 transposes, SwiGLU amax swaps
 constexpr int MAX_E = 1024;
+constexpr int ITEM_TAB = 128;  // work items per pair whose expert is looked up, not searched
 // Sixteen epilogue warps, four per sub-partition: the epilogue is bound by issue
 // and latency (TMEM loads, MUFU-heavy SiLU, lane exchanges), so it wants warps;
 // 18 warps leave 112 registers a thread.
@@ -141,7 +142,12 @@ struct Smem {
   // {end of its token tiles (prefix sum), first routed slot, first padded row,
   // routed-slot count}
   int4 rec[MAX_E];
-  float2 ag[MAX_E];  // {g_act[e] * alpha_w[e] (the accumulator's scale), global scale of the requantised output}
+  float2 ag[MAX_E];
+  // the expert of each of this pair's work items when the pair has at most ITEM_TAB of
+  // them (decode-sized batches, where every item jumps over several experts), found at
+  // set-up by the prefix-sum warp; n_tab = 0: the roles walk (see TileWalk)
+  uint16_t item_e[ITEM_TAB];
+  int n_tab;  // {g_act[e] * alpha_w[e] (the accumulator's scale), global scale of the requantised output}
 };
 
 template <bool DENSE>
@@ -182,13 +188,15 @@ struct Tile {
 // tile later (its latency is hidden behind the tile's work).
 struct TileWalk {
   int q, m, dq, dm, e;
+  int j, ntab;    // item index of this pair; items with j < ntab take their expert from item_e
   int4 cur, nxt;  // rec[e], rec[e + 1] (rec[e] again past the last expert)
   __device__ __forceinline__ TileWalk(const Smem& s, int pid, int npairs, int MT2, int E)
-      : q(pid / MT2), m(pid % MT2), dq(npairs / MT2), dm(npairs % MT2), e(0) {
+      : q(pid / MT2), m(pid % MT2), dq(npairs / MT2), dm(npairs % MT2), e(0), j(0), ntab(s.n_tab) {
     cur = s.rec[0];
     nxt = E > 1 ? s.rec[1] : cur;
   }
   __device__ __forceinline__ void advance(int MT2) {
+    ++j;
     m += dm;
     q += dq;
     if (m >= MT2) {
@@ -204,7 +212,13 @@ struct TileWalk {
 // experts (decode batches of a layer with many experts) costs log2(E) loads, not E.
 template <int NT = 1>
 __device__ __forceinline__ Tile decode_tile(const Smem& s, TileWalk& w, int E) {
-  if (w.cur.x <= w.q && w.e + 1 < E) {
+  if (NT == 1 && w.j < w.ntab) {  // the same for every item of the pair: table or walk
+    const int e = s.item_e[w.j];
+    if (e != w.e) {
+      w.e = e;
+      w.cur = s.rec[e];
+    }
+  } else if (w.cur.x <= w.q && w.e + 1 < E) {
     if (w.nxt.x > w.q) {
       ++w.e;
       w.cur = w.nxt;
@@ -307,7 +321,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   }
   __syncthreads();
   if (warp == 0) {  // end of expert e's token tiles = sum over e' <= e of ceil(T_e' / BN)
-    int run = 0;
+    int run = 0, nz = 0;  // tiles, experts that hold any
     for (int e0 = 0; e0 < E; e0 += 32) {
       const int e = e0 + lane;
       int v = 0;
@@ -320,7 +334,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       }
       if (e < E) S.rec[e].x = run + x;
       run += __shfl_sync(0xffffffffu, x, 31);
+      nz += __popc(__ballot_sync(0xffffffffu, v > 0));
     }
+    // decode-sized batches: the expert of each of this pair's items, one binary search
+    // per item by the lanes of this warp.  Used where a role's walk, which advances
+    // npairs / MT2 tiles an item, would jump over two or more experts an item on
+    // average and so search item after item; elsewhere the walk steps through the
+    // records it holds, which costs less than a table load.  Wide items run on large
+    // batches only.
+    __syncwarp();
+    const int tot = run * MT2, dq = npairs / MT2;
+    const int mine = pair_id < tot ? (tot - 1 - pair_id) / npairs + 1 : 0;
+    const int ntab = NT == 1 && mine >= 2 && mine <= ITEM_TAB && 2 * run < dq * nz ? mine : 0;
+    for (int j = lane; j < ntab; j += 32) {
+      const int qj = (pair_id + j * npairs) / MT2;
+      int lo = 0, hi = E - 1;  // the first expert whose tile end exceeds qj
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (S.rec[mid].x > qj) hi = mid;
+        else lo = mid + 1;
+      }
+      S.item_e[j] = (uint16_t)lo;
+    }
+    if (lane == 0) S.n_tab = ntab;
   }
   tc_fence_before();
   cluster_sync_all();

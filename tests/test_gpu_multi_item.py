@@ -13,7 +13,11 @@ walk.  The other GEMM tests have fewer items than the device has pairs, so here:
   kernel);
 * a layer whose item list is many times the device's own pair count (32 experts,
   top-4, H = 512, I = 256, 8192 tokens: 512 items per GEMM) runs at the uncapped
-  launch, and the whole layer is compared element by element;
+  launch, and the whole layer is compared element by element; on one pair its 512
+  items exceed the set-up table of per-item experts (128), so the roles walk them;
+* a decode-sized layer (64 experts holding one 128-token tile each) at 8, 16 and all
+  pairs, where each pair looks its items' experts up in a table built at set-up rather
+  than walking the expert records (the kernel's rule, restated in table_used);
 * wide items of the SwiGLU gate_up GEMM (two 128-token tiles of one expert, one MMA
   of N <= 256 per K step, a single 256-column accumulator): forced on layers whose
   experts hold 0, 7, 40, 128, 129, 250, 256, 300, 517 and 700 tokens, so items with a
@@ -40,6 +44,10 @@ pytestmark = pytest.mark.gpu
 LIMITS = (1, 2, 3)
 CAPPED = ("tiny", "ragged_multi_tile", "sparse_routing", "mid_ktail", "deep_k", "exact_per_half_alpha")
 MANY = W.LayerConfig("many_items", 46, 32, 4, 512, 256, (8192,), "uniform", True)
+# decode-sized: 64 experts of one tile each, so a pair's walk would jump over many experts
+# an item and the set-up table of per-item experts is used instead (at every launch size
+# below; see table_used)
+DECODE = W.LayerConfig("decode_items", 49, 64, 2, 512, 256, (256,), "uniform", True)
 # tokens per expert of the wide-item layers (top-1 routing, built directly)
 WIDE_COUNTS = (0, 7, 40, 128, 129, 250, 256, 300, 517, 700)
 WIDE = {
@@ -162,6 +170,14 @@ def test_many_items_down_bf16(many_layer):
     TG.test_down_bf16_within_tolerance(many_layer)
 
 
+def test_many_items_on_one_pair(many_layer):
+    """512 items on one pair: more than the set-up item table holds, so every role walks
+    the items and searches the expert records."""
+    with PairLimit(1):
+        TG.test_swiglu_requant_epilogue(many_layer)
+        TG.test_down_bf16_within_tolerance(many_layer)
+
+
 def test_many_items_forward(many_layer):
     TG.test_moe_forward_end_to_end(many_layer)
     TG.test_forward_is_deterministic(many_layer)
@@ -231,3 +247,31 @@ def test_tiles_per_item_arguments():
         assert M.moesq_gemm_tiles_per_item(0, sw, 4096 + 256, 128, 1) == 1
     with TilesPerItem(1):
         assert M.moesq_gemm_tiles_per_item(0, sw, 4096, 128, 1 << 20) == 1
+
+
+def table_used(counts, out_rows, pairs):
+    """The kernel's rule for the per-item expert table, for pair 0: 2 to 128 items, and a
+    walk that would advance over two or more experts an item on average."""
+    tiles = int(((counts + 127) // 128).sum())
+    nz = int((counts > 0).sum())
+    mt2 = (out_rows // 128 + 1) // 2
+    mine = -(-tiles * mt2 // pairs)
+    return 2 <= mine <= 128 and 2 * tiles < (pairs // mt2) * nz
+
+
+@pytest.fixture(scope="module")
+def decode_layer():
+    return TG.Layer(DECODE, 256)
+
+
+@pytest.mark.parametrize("limit", (0, 8, 16))
+def test_decode_items_from_table(decode_layer, limit):
+    L = decode_layer
+    counts = np.diff(L.perm["expert_offsets"])
+    with PairLimit(limit):
+        pairs = M.moesq_gemm_launch_pairs(0, M.EPI_BF16)
+        assert table_used(counts, 2 * DECODE.I, pairs) and table_used(counts, DECODE.H, pairs)
+        TG.test_gate_up_f32_within_tolerance(L)
+        TG.test_swiglu_requant_epilogue(L)
+        TG.test_down_bf16_within_tolerance(L)
+        TG.test_moe_forward_end_to_end(L)
