@@ -69,6 +69,7 @@ def parse_args():
     ap.add_argument("--shape-configs", default=",".join(SHAPE_CONFIGS))
     ap.add_argument("--no-storage", action="store_true", help="skip the Kimi-K2 storage benchmark key")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense comparison GEMMs")
+    ap.add_argument("--no-fused", action="store_true", help="skip the fused down + combine comparison")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-slots", type=int, default=256, help="slots in the CPU-baseline sample")
@@ -493,6 +494,56 @@ class Bench:
         del graphs
         return res
 
+    def fused_combine(self, steps, flush):
+        """The down GEMM with the weighted combine fused into its epilogue
+        (moesq_grouped_gemm_down_combine) against the down GEMM plus the separate
+        combine, each as one graph after an L2 flush; and whether the fused output is
+        bit-identical to the staged one."""
+        torch, M = self.torch, self.M
+        cfg, T = self.cfg, self.T
+        for s_ in self.STAGES:
+            getattr(self, s_)()
+        y = torch.empty_like(self.y)
+        out = torch.empty_like(self.out)
+        arrivals = torch.empty(T * (cfg.H // 128), dtype=torch.int32, device=self.dev)
+
+        def fused():
+            M.moesq_grouped_gemm_down_combine(self.lin["down"].struct, self.h_codes, self.h_sf, self.g_in_dn, self.eo,
+                                              self.po, self.S, self.P, self.slot_token, self.token_slot, self.w,
+                                              T, cfg.k, y.view(torch.uint16), out.view(torch.uint16), arrivals,
+                                              self.status)
+
+        def staged():
+            self.gemm_down()
+            self.combine()
+
+        fused()
+        torch.cuda.synchronize()
+        same = bool(torch.equal(out.view(torch.int16), self.out.view(torch.int16)))
+        graphs = {}
+        for name, fn in (("down_plus_combine", staged), ("fused", fused)):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fn()
+            graphs[name] = g
+        stream = torch.cuda.current_stream()
+        res = {}
+        for name, g in graphs.items():
+            for _ in range(3):
+                g.replay()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+            for a, b in ev:
+                if flush is not None:
+                    flush.zero_()
+                torch.cuda._sleep(1_000_000)
+                a.record(stream)
+                g.replay()
+                b.record(stream)
+            torch.cuda.synchronize()
+            res[name] = sum(a.elapsed_time(b) for a, b in ev) / steps
+        del graphs
+        return res, same
+
     def check_against_forward(self):
         """The staged step and the single moesq_moe_forward call give identical bytes."""
         torch = self.torch
@@ -833,6 +884,14 @@ def run_ours(args, rank, world, local_rank):
             "weight_bytes_per_dense_element": {"sparse": 0.34375, "dense": 0.53125},
             "weight_bytes_touched_GB": {k: {"sparse": by_w[k] * 0.34375 / 1e9, "dense": by_w[k] * 0.53125 / 1e9}
                                         for k in by_w},
+        }
+    if world == 1 and not args.no_fused:
+        d, same = b.fused_combine(10, flush)
+        out["fused_combine"] = {
+            "what": "down GEMM with the weighted combine fused into its epilogue (per-token arrival counts, the "
+                    "completing arrival sums the k rows in j order) vs the down GEMM and the separate combine",
+            "down_plus_combine_ms": d["down_plus_combine"], "fused_ms": d["fused"],
+            "fused_speedup": d["down_plus_combine"] / d["fused"], "bit_identical": same,
         }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         one = cpu_baseline(cfg, args.tokens, args.cpu_slots, threads=1)

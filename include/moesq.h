@@ -326,6 +326,31 @@ moesq_status moesq_grouped_gemm_workspace_size(const moesq_linear* W, int64_t S,
 moesq_status moesq_set_gemm_pair_limit(int32_t max_pairs);
 moesq_status moesq_gemm_launch_pairs(int32_t dense, int32_t epilogue, int32_t* pairs);
 
+/* Down GEMM with the weighted combine fused into its epilogue (the combine of the
+ * MoESQ README "Kernels" path, done where y is produced): out[t, :] = sum over j in
+ * 0..k-1, in that order, of topk_w[t, j] * y[token_slot[t, j], :], float32 products of
+ * the stored bf16 y without fused multiply-add, rounded once to bf16 -- bit-identical
+ * to moesq_grouped_gemm(MOESQ_EPI_BF16) followed by moesq_unpermute.  Deterministic:
+ * every (token, 128-output tile) counts its k slot arrivals (each after that slot's y
+ * row is written and fenced) and the arrival that completes the count sums the k rows.
+ *   W          MOESQ_LINEAR_DOWN weights; other GEMM arguments as moesq_grouped_gemm
+ *   S          == T * k, 1 <= k <= 32
+ *   slot_token, token_slot   moesq_permute's outputs for this batch (device i32)
+ *   topk_w     device f32 [T, k]
+ *   y          device bf16 [S, W.out] scratch: every slot's row, as MOESQ_EPI_BF16 writes it
+ *   out        device bf16 [T, W.out]
+ *   arrivals   device i32 [T * W.out / 128] scratch, zeroed by this call (stream-ordered)
+ * Returns as moesq_grouped_gemm; the fused epilogue writes y rows straight from
+ * registers (no staging), so on large batches it runs slower than the two kernels
+ * (the library's forward keeps them separate). */
+moesq_status moesq_grouped_gemm_down_combine(const moesq_linear* W, const uint8_t* act_codes,
+                                             const uint8_t* act_sf, const float* g_act,
+                                             const int32_t* expert_offsets, const int32_t* pad_offsets,
+                                             int64_t S, int64_t P_cap, const int32_t* slot_token,
+                                             const int32_t* token_slot, const float* topk_w, int64_t T,
+                                             int32_t k, uint16_t* y, uint16_t* out, int32_t* arrivals,
+                                             int32_t* d_status, moesq_stream_t stream);
+
 /* Work-item width of the sparse SwiGLU gate_up GEMM (the pages have no counterpart).
  * A work item is one weight-tile pair times one 128-token tile, or, on large batches,
  * two 128-token tiles of one expert computed by single MMAs of N <= 256 ("wide" items:

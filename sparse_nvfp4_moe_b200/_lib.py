@@ -59,6 +59,9 @@ _SIGS = {
                                               c_vp, c_vp, c_vp, c_vp]),
     "moesq_grouped_gemm": (ctypes.c_int, [ctypes.POINTER(Linear), c_vp, c_vp, c_vp, c_vp, c_vp, c_i64,
                                           c_i64, c_i32, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp, c_vp]),
+    "moesq_grouped_gemm_down_combine": (ctypes.c_int, [ctypes.POINTER(Linear), c_vp, c_vp, c_vp, c_vp, c_vp, c_i64,
+                                                       c_i64, c_vp, c_vp, c_vp, c_i64, c_i32, c_vp, c_vp, c_vp,
+                                                       c_vp, c_vp]),
     "moesq_grouped_gemm_dense": (ctypes.c_int, [ctypes.POINTER(Linear), c_vp, c_vp, c_vp, c_vp, c_vp, c_i64,
                                                 c_i64, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp]),
     "moesq_sf_expand_block16": (ctypes.c_int, [c_vp, c_vp, c_i64, c_vp]),
@@ -228,6 +231,15 @@ def moesq_grouped_gemm(W: Linear, act_codes, act_sf, g_act, expert_offsets, pad_
     _check("moesq_grouped_gemm", lib().moesq_grouped_gemm(
         ctypes.byref(W), _p(act_codes), _p(act_sf), _p(g_act), _p(expert_offsets), _p(pad_offsets), S,
         P_cap, epilogue, _p(g_next), _p(out), _p(out_sf), _p(ws), ws_bytes, _p(d_status),
+        _stream(stream)))
+
+
+def moesq_grouped_gemm_down_combine(W: Linear, act_codes, act_sf, g_act, expert_offsets, pad_offsets, S, P_cap,
+                                    slot_token, token_slot, topk_w, T, k, y, out, arrivals, d_status=None,
+                                    stream=None):
+    _check("moesq_grouped_gemm_down_combine", lib().moesq_grouped_gemm_down_combine(
+        ctypes.byref(W), _p(act_codes), _p(act_sf), _p(g_act), _p(expert_offsets), _p(pad_offsets), S, P_cap,
+        _p(slot_token), _p(token_slot), _p(topk_w), T, k, _p(y), _p(out), _p(arrivals), _p(d_status),
         _stream(stream)))
 
 

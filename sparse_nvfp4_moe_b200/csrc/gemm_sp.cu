@@ -110,6 +110,10 @@ constexpr uint32_t TM_E = 384, TM_SFA = 392, TM_SFB = 408;  // SFB: 8 columns pe
 static_assert(TM_SFB + 32 <= TMEM_COLS && STAGE_BYTES % 1024 == 0, "wide geometry");
 }  // namespace wide
 
+// The down GEMM with the weighted combine fused into its epilogue (see the bf16
+// epilogue): a template value of its own, not an `epilogue` argument of the C ABI.
+constexpr int EPI_BF16_COMBINE = 3;
+
 struct Params {
   const uint8_t* meta;
   const uint8_t* sfw;
@@ -125,6 +129,14 @@ struct Params {
   int E, M, K, epi, gate_up;
   int exact;  // gate_up with its own up global: alpha_w is [E, 2] (gate, up)
   int64_t S, P_cap;
+  // EPI_BF16_COMBINE only: routing, weights, per-(token, 128-output tile) arrival counts
+  // (zero at launch), the combined output [T, M] bf16; p.out is the per-slot y
+  const int32_t* slot_token;
+  const int32_t* token_slot;
+  const float* topk_w;
+  int32_t* arrivals;
+  uint16_t* comb_out;
+  int k;
 };
 
 struct Smem {
@@ -768,7 +780,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         } else {
           finish(hv, t.prow, t.n_rows, live);
         }
-      } else if constexpr (EPI == MOESQ_EPI_BF16) {
+      } else if constexpr (EPI == MOESQ_EPI_BF16 || EPI == EPI_BF16_COMBINE) {
         // Per 32-token column block kb, its four warps (one per lane quarter q) write
         // [32 tokens][128 outputs] bf16.  The interleaved weight rows put both outputs of
         // a bf16 pair in one thread of a 16x256b TMEM load (down: lanes j and 8 + j of a
@@ -794,7 +806,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // pair slots of the thread's two words per column
         const int w0 = gu ? 8 * q + j : 16 * (q & 1) + j;
         const int w1 = gu ? w0 : w0 + 8;
-        if (nblk == 32) {
+        if (EPI == MOESQ_EPI_BF16 && nblk == 32) {
           // a full block: the four warps stage [32 tokens][128 outputs] as two 64-output
           // halves [32 rows][128 B] in the TMA 128-byte swizzle (16-byte chunk c of row r
           // at c ^ (r & 7)) and one lane writes them with two TMA stores.  Words of one
@@ -848,6 +860,72 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
               *reinterpret_cast<__nv_bfloat162*>(yr + base0 + 2 * w0) = __floats2bfloat162_rn(w0v.x, w0v.y);
               *reinterpret_cast<__nv_bfloat162*>(yr + base1 + 2 * w1) = __floats2bfloat162_rn(w1v.x, w1v.y);
             }
+          }
+          if constexpr (EPI == EPI_BF16_COMBINE) {
+            // Fused weighted combine, deterministic: every (token, 128-output tile) counts
+            // its k arrivals, one per slot, each after that slot's y rows are written and
+            // fenced; the arrival that completes the count sums the token's k rows of the
+            // tile in j order, exactly as the separate combine does (float32, no fused
+            // multiply-add, products of the stored bf16 y), and writes the output.  Rows
+            // are read at L2 (other SMs wrote them).
+            __threadfence();
+            named_bar_sync(10 + kb, 128);  // the block's y rows are written and fenced
+            const int bt = (ew & 3) * 32 + lane;  // thread of the block
+            // per row of the block: the token completed by this arrival, else -1
+            volatile int32_t* done = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(epi) + kb * 8192);
+            if (bt < 32) {
+              int32_t tok_done = -1;
+              if (bt < nblk) {
+                const int32_t tok = p.slot_token[s0 + c_lo + bt];
+                __threadfence();  // release: the block's rows (fenced, then the barrier) before the count
+                if (atomicAdd(p.arrivals + (int64_t)tok * MT + mt, 1) == p.k - 1) tok_done = tok;
+              }
+              done[bt] = tok_done;
+              __threadfence();
+            }
+            named_bar_sync(10 + kb, 128);
+            for (int r = ew & 3; r < nblk; r += 4) {
+              const int64_t tok = done[r];
+              if (tok < 0) continue;
+              __threadfence();  // acquire: every arrival's rows before these loads
+              // lanes j < k hold slot j and its weight; the rows are loaded eight at a
+              // time before they are summed, in j order
+              int64_t sl = 0;
+              float wl = 0.0f;
+              if (lane < p.k) {
+                sl = p.token_slot[tok * p.k + lane];
+                wl = p.topk_w[tok * p.k + lane];
+              }
+              float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+              for (int j0 = 0; j0 < p.k; j0 += 8) {
+                uint2 uv[8];
+                float wv[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                  const int64_t sj = __shfl_sync(0xffffffffu, sl, (j0 + u) & 31);
+                  wv[u] = __shfl_sync(0xffffffffu, wl, (j0 + u) & 31);
+                  uv[u] = j0 + u < p.k ? __ldcg(reinterpret_cast<const uint2*>((const uint16_t*)p.out + sj * p.M +
+                                                                                 BM * mt + 4 * lane))
+                                       : make_uint2(0u, 0u);
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                  if (j0 + u < p.k) {
+                    const float wj = wv[u];
+                    acc[0] = __fadd_rn(acc[0], __fmul_rn(wj, __uint_as_float(uv[u].x << 16)));
+                    acc[1] = __fadd_rn(acc[1], __fmul_rn(wj, __uint_as_float(uv[u].x & 0xFFFF0000u)));
+                    acc[2] = __fadd_rn(acc[2], __fmul_rn(wj, __uint_as_float(uv[u].y << 16)));
+                    acc[3] = __fadd_rn(acc[3], __fmul_rn(wj, __uint_as_float(uv[u].y & 0xFFFF0000u)));
+                  }
+                }
+              }
+              const __nv_bfloat162 o0 = __floats2bfloat162_rn(acc[0], acc[1]), o1 = __floats2bfloat162_rn(acc[2], acc[3]);
+              uint2 o;
+              o.x = *reinterpret_cast<const uint32_t*>(&o0);
+              o.y = *reinterpret_cast<const uint32_t*>(&o1);
+              *reinterpret_cast<uint2*>(p.comb_out + tok * p.M + BM * mt + 4 * lane) = o;
+            }
+            named_bar_sync(10 + kb, 128);  // the flags are read before the next tile writes them
           }
         }
       } else {
@@ -1007,13 +1085,15 @@ static int tiles_per_item(bool dense, int32_t epilogue, int64_t K, int64_t E, in
 // CTA pairs of a launch: clusters of 2 CTAs, one CTA per SM, as many pairs as the
 // device can hold at once (cached per device and kernel), capped by g_pair_limit.
 template <bool DENSE>
-static moesq_status launch_pairs(int dev, int sms, int32_t epilogue, int* pairs_out, bool wide = false) {
+static moesq_status launch_pairs(int dev, int sms, int32_t epilogue, int* pairs_out, bool wide = false,
+                                 bool comb = false) {
   const size_t smem = wide ? sp::smem_bytes_wide() : sp::smem_bytes<DENSE>();
-  static int pairs_cache[64][4] = {{0}};
-  const int ei = wide ? 3 : epilogue - MOESQ_EPI_F32;
+  static int pairs_cache[64][5] = {{0}};
+  const int ei = comb ? 4 : wide ? 3 : epilogue - MOESQ_EPI_F32;
   int pairs = dev < 64 ? pairs_cache[dev][ei] : 0;
   if (pairs == 0) {
-    const void* fn = wide ? (const void*)sp::k_grouped_gemm_sp<MOESQ_EPI_SWIGLU_NVFP4, false, 2>
+    const void* fn = comb ? (const void*)sp::k_grouped_gemm_sp<sp::EPI_BF16_COMBINE, false, 1>
+                     : wide ? (const void*)sp::k_grouped_gemm_sp<MOESQ_EPI_SWIGLU_NVFP4, false, 2>
                      : epilogue == MOESQ_EPI_F32 ? (const void*)sp::k_grouped_gemm_sp<MOESQ_EPI_F32, DENSE>
                      : epilogue == MOESQ_EPI_BF16 ? (const void*)sp::k_grouped_gemm_sp<MOESQ_EPI_BF16, DENSE>
                                                   : (const void*)sp::k_grouped_gemm_sp<MOESQ_EPI_SWIGLU_NVFP4, DENSE>;
@@ -1041,12 +1121,23 @@ static moesq_status launch_pairs(int dev, int sms, int32_t epilogue, int* pairs_
 // the kept bytes, W->meta the sparse metadata); DENSE = true is the comparison
 // kernel on decoded weights (W->packed dense codes [E, out, K/2], no metadata, W->sf
 // and act_sf in the 16-element scale layout of moesq_sf_expand_block16).
+// The weighted combine fused into the down GEMM (moesq_grouped_gemm_down_combine).
+struct CombineArgs {
+  const int32_t* slot_token;
+  const int32_t* token_slot;
+  const float* topk_w;
+  int64_t T;
+  int k;
+  uint16_t* out;
+  int32_t* arrivals;
+};
+
 template <bool DENSE>
 static moesq_status grouped_gemm_impl(const moesq_linear* W, const uint8_t* act_codes, const uint8_t* act_sf,
                                       const float* g_act, const int32_t* expert_offsets,
                                       const int32_t* pad_offsets, int64_t S, int64_t P_cap, int32_t epilogue,
                                       const float* g_next, void* out, uint8_t* out_sf, int32_t* d_status,
-                                      moesq_stream_t stream) {
+                                      moesq_stream_t stream, const CombineArgs* comb = nullptr) {
   MOESQ_REQUIRE(W, MOESQ_ERR_INVALID_ARG);
   MOESQ_REQUIRE(W->packed && (DENSE || W->meta) && W->sf && W->alpha_w, MOESQ_ERR_INVALID_ARG);
   MOESQ_REQUIRE(act_codes && act_sf && g_act && expert_offsets && pad_offsets && out,
@@ -1067,11 +1158,21 @@ static moesq_status grouped_gemm_impl(const moesq_linear* W, const uint8_t* act_
     MOESQ_REQUIRE(W->out % 256 == 0, MOESQ_ERR_UNSUPPORTED_SHAPE);
   }
   if (gate_up) MOESQ_REQUIRE(W->out % 256 == 0, MOESQ_ERR_UNSUPPORTED_SHAPE);
+  if (comb) {
+    MOESQ_REQUIRE(!gate_up && epilogue == MOESQ_EPI_BF16, MOESQ_ERR_INVALID_ARG);  // sparse kernel only
+    MOESQ_REQUIRE(comb->slot_token && comb->token_slot && comb->topk_w && comb->out && comb->arrivals,
+                  MOESQ_ERR_INVALID_ARG);
+    MOESQ_REQUIRE(comb->k >= 1 && comb->k <= 32 && comb->T >= 0 && S == comb->T * comb->k, MOESQ_ERR_INVALID_ARG);
+    MOESQ_REQUIRE(moesq_aligned16(comb->out), MOESQ_ERR_INVALID_ARG);
+  }
   MOESQ_REQUIRE(moesq_aligned16(W->packed) && (DENSE || moesq_aligned16(W->meta)) && moesq_aligned16(W->sf) &&
                     moesq_aligned16(act_codes) && moesq_aligned16(act_sf) && moesq_aligned16(out) &&
                     moesq_aligned16(out_sf),
                 MOESQ_ERR_INVALID_ARG);
   if (S == 0) return MOESQ_OK;
+  if (comb && cudaMemsetAsync(comb->arrivals, 0, (size_t)comb->T * (size_t)(W->out / 128) * sizeof(int32_t),
+                              (cudaStream_t)stream) != cudaSuccess)
+    return MOESQ_ERR_CUDA;
   int dev = 0;
   const int sms = device_sms(&dev);
   if (sms < 0) return MOESQ_ERR_CUDA;
@@ -1157,7 +1258,7 @@ static moesq_status grouped_gemm_impl(const moesq_linear* W, const uint8_t* act_
 
   const size_t smem = wide ? sp::smem_bytes_wide() : sp::smem_bytes<DENSE>();
   int pairs = 0;
-  const moesq_status pst = launch_pairs<DENSE>(dev, sms, epilogue, &pairs, wide);
+  const moesq_status pst = launch_pairs<DENSE>(dev, sms, epilogue, &pairs, wide, comb != nullptr);
   if (pst != MOESQ_OK) return pst;
   sp::Params prm;
   prm.meta = W->meta;
@@ -1179,6 +1280,12 @@ static moesq_status grouped_gemm_impl(const moesq_linear* W, const uint8_t* act_
   prm.exact = W->kind == MOESQ_LINEAR_GATE_UP_EXACT ? 1 : 0;
   prm.S = S;
   prm.P_cap = P_cap;
+  prm.slot_token = comb ? comb->slot_token : nullptr;
+  prm.token_slot = comb ? comb->token_slot : nullptr;
+  prm.topk_w = comb ? comb->topk_w : nullptr;
+  prm.arrivals = comb ? comb->arrivals : nullptr;
+  prm.comb_out = comb ? comb->out : nullptr;
+  prm.k = comb ? comb->k : 0;
   cudaStream_t st = (cudaStream_t)stream;
   const dim3 grid((unsigned)(2 * pairs));
   cudaError_t err;
@@ -1188,8 +1295,12 @@ static moesq_status grouped_gemm_impl(const moesq_linear* W, const uint8_t* act_
                          tb16, te, tsfa, tsfb, ty, tb3, prm);
       break;
     case MOESQ_EPI_BF16:
-      err = moesq_launch(sp::k_grouped_gemm_sp<MOESQ_EPI_BF16, DENSE>, grid, dim3(sp::THREADS), smem, st, ta, tb,
-                         tb16, te, tsfa, tsfb, ty, tb3, prm);
+      if (comb)
+        err = moesq_launch(sp::k_grouped_gemm_sp<sp::EPI_BF16_COMBINE, false, 1>, grid, dim3(sp::THREADS), smem, st,
+                           ta, tb, tb16, te, tsfa, tsfb, ty, tb3, prm);
+      else
+        err = moesq_launch(sp::k_grouped_gemm_sp<MOESQ_EPI_BF16, DENSE>, grid, dim3(sp::THREADS), smem, st, ta, tb,
+                           tb16, te, tsfa, tsfb, ty, tb3, prm);
       break;
     default:
       if (wide)
@@ -1217,6 +1328,16 @@ extern "C" moesq_status moesq_grouped_gemm(const moesq_linear* W, const uint8_t*
   (void)ws_bytes;
   return grouped_gemm_impl<false>(W, act_codes, act_sf, g_act, expert_offsets, pad_offsets, S, P_cap, epilogue,
                                   g_next, out, out_sf, d_status, stream);
+}
+
+extern "C" moesq_status moesq_grouped_gemm_down_combine(
+    const moesq_linear* W, const uint8_t* act_codes, const uint8_t* act_sf, const float* g_act,
+    const int32_t* expert_offsets, const int32_t* pad_offsets, int64_t S, int64_t P_cap, const int32_t* slot_token,
+    const int32_t* token_slot, const float* topk_w, int64_t T, int32_t k, uint16_t* y, uint16_t* out,
+    int32_t* arrivals, int32_t* d_status, moesq_stream_t stream) {
+  const CombineArgs c{slot_token, token_slot, topk_w, T, k, out, arrivals};
+  return grouped_gemm_impl<false>(W, act_codes, act_sf, g_act, expert_offsets, pad_offsets, S, P_cap, MOESQ_EPI_BF16,
+                                  nullptr, y, nullptr, d_status, stream, &c);
 }
 
 extern "C" moesq_status moesq_grouped_gemm_dense(const moesq_linear* W, const uint8_t* act_codes,
