@@ -51,7 +51,14 @@ METRIC = "dense-equiv TFLOP/s & % roofline, sparse NVFP4 MoE grouped GEMM (1 B20
 UNIT = "TFLOP/s"
 B_W, B_A = 0.34375, 0.53125     # bytes per dense element: sparse weight storage, NVFP4-32 activation
 FP4_SPARSE_OVER_BF16 = 8.0      # nominal dense-equivalent sparse FP4 (18 PF) / dense bf16 (2.25 PF)
-KERNELS_PER_STEP = 7            # permute x3, routed quant, gate_up GEMM, down GEMM, combine
+def kernels_per_step(cfg, T):
+    """Library kernels one step launches: the permute (1 kernel up to 1024 slots, else 3),
+    the routed quant (a second, in-place kernel rearranges its row-major scales into the
+    tensor-core blocks when K % 1024 == 0, k <= 32 and the codes written reach 64 MiB),
+    the two GEMMs and the combine."""
+    perm = 1 if T * cfg.k <= 1024 else 3
+    quant = 2 if cfg.H % 1024 == 0 and cfg.k <= 32 and T * cfg.k * (cfg.H // 2) >= (64 << 20) else 1
+    return perm + quant + 3
 L2_BYTES = 126 * 1024 * 1024    # B200 L2
 DEFAULT_CONFIG, DEFAULT_TOKENS = "qwen3_235b_a22b", 65536
 SHAPE_CONFIGS = ("qwen3_30b_a3b", "qwen3_5_397b_a17b", "qwen3_235b_a22b", "kimi_k2")
@@ -863,7 +870,7 @@ def run_ours(args, rank, world, local_rank):
                    "l2": "flushed between timed steps (256 MiB write)", "parallelism": f"replicas x{world}"},
         "roofline": roof,
         "kernels": kernels,
-        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "gpu_launches": kernels_per_step(cfg, args.tokens) * args.steps,
         "staged_equals_forward": ok,
         "clocks": clocks,
     }

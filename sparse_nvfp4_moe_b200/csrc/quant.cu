@@ -173,13 +173,23 @@ __global__ void k_quant_act_routed(const uint16_t* __restrict__ x, int64_t T, in
 // lane quantises its group and stores 16 code bytes per slot (512 contiguous bytes per
 // warp and slot); lanes 4m..4m+3 hold the four scales that share a 512-byte block
 // position and lane 4m stores them as one 32-bit word.
+//
+// On large batches (`rows`) the scales go out as rows first: lane 4m's word lands at
+// bytes 32c + 4m of its slot's padded row of K/32 scale bytes (one 32-byte sector per
+// warp and slot), and k_sf_rows_to_blocks then rearranges each 128-row slab, in place,
+// into the 512-byte tensor-core blocks.  Written straight into the blocks, a slot's 32
+// words land in 32 different 32-byte sectors, each completed by 8 slots of other tokens
+// written at other times; once the codes streaming through L2 evict the partly written
+// sectors before they are complete, the scale stores, 4% of the bytes, took 44% of the
+// kernel's time (Qwen3-235B-A22B T = 65536: 483 us with them, 270 us without).  Small
+// batches, whose scales stay in L2, write the blocks directly and save the second kernel.
 __global__ void k_quant_act_routed_warp(const uint16_t* __restrict__ x, int64_t T, int64_t K,
                                         const int32_t* __restrict__ topk_ids,
                                         const int32_t* __restrict__ token_slot, int k,
                                         const int32_t* __restrict__ expert_offsets,
                                         const int32_t* __restrict__ pad_offsets, int E,
                                         const float* __restrict__ g_in, uint8_t* __restrict__ codes,
-                                        uint8_t* __restrict__ sf) {
+                                        uint8_t* __restrict__ sf, bool rows) {
   pdl_wait();  // the previous kernel's outputs are complete past here
   pdl_trigger();
   const int lane = threadIdx.x & 31;
@@ -234,10 +244,55 @@ __global__ void k_quant_act_routed_warp(const uint16_t* __restrict__ x, int64_t 
       }
       *reinterpret_cast<uint4*>(codes + row * (K / 2) + 16 * grp) = make_uint4(o[0], o[1], o[2], o[3]);
       if ((lane & 3) == 0) {
-        const int64_t blk = (row / 128) * (K / 128) + grp / 4;
-        *reinterpret_cast<uint32_t*>(sf + blk * 512 + sf_block_offset((uint32_t)(row % 128), 0u)) = word;
+        if (rows) {
+          *reinterpret_cast<uint32_t*>(sf + row * (K / 32) + grp) = word;
+        } else {
+          const int64_t blk = (row / 128) * (K / 128) + grp / 4;
+          *reinterpret_cast<uint32_t*>(sf + blk * 512 + sf_block_offset((uint32_t)(row % 128), 0u)) = word;
+        }
       }
     }
+  }
+}
+
+// In place, per 128-row slab of the scale buffer: rows of K/32 scale bytes (row r of the
+// slab at r * K/32) into the slab's K/128 blocks of 512 bytes (row r, scale j of block kk
+// at kk * 512 + (r % 32) * 16 + (r / 32) * 4 + j).  Both layouts of a slab fill the same
+// 128 * K/32 bytes at the same offset.  One block of threads per slab: coalesced 16-byte
+// loads into shared memory (rows padded by 4 bytes so that the gather is conflict-free),
+// then each thread writes one 16-byte piece (rows r, r + 32, r + 64, r + 96 of one block).
+// The slab count comes from pad_offsets[E] on the device.
+__global__ void k_sf_rows_to_blocks(uint8_t* __restrict__ sf, const int32_t* __restrict__ pad_offsets, int E,
+                                    int64_t K) {
+  extern __shared__ __align__(16) uint8_t rows[];
+  pdl_wait();
+  pdl_trigger();
+  const int rb = (int)(K / 32);   // bytes per row
+  const int rs = rb + 4;          // padded row stride in shared memory
+  const int64_t slab_bytes = (int64_t)128 * rb;
+  const int64_t nslab = pad_offsets[E] / 128;
+  for (int64_t b = blockIdx.x; b < nslab; b += gridDim.x) {
+    uint8_t* g = sf + b * slab_bytes;
+    for (int i = threadIdx.x; i < 128 * rb / 16; i += blockDim.x) {
+      const int r = (16 * i) / rb, c = (16 * i) % rb;
+      const uint4 v = *reinterpret_cast<const uint4*>(g + 16 * (int64_t)i);
+      uint32_t* d = reinterpret_cast<uint32_t*>(rows + r * rs + c);  // rs is 4-byte aligned only
+      d[0] = v.x;
+      d[1] = v.y;
+      d[2] = v.z;
+      d[3] = v.w;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < 128 * rb / 16; i += blockDim.x) {
+      const int kk = i / 32, r = i % 32;  // block kk, rows r + 32m: 16 bytes at kk * 512 + 16 r
+      uint4 v;
+      v.x = *reinterpret_cast<const uint32_t*>(rows + r * rs + 4 * kk);
+      v.y = *reinterpret_cast<const uint32_t*>(rows + (r + 32) * rs + 4 * kk);
+      v.z = *reinterpret_cast<const uint32_t*>(rows + (r + 64) * rs + 4 * kk);
+      v.w = *reinterpret_cast<const uint32_t*>(rows + (r + 96) * rs + 4 * kk);
+      *reinterpret_cast<uint4*>(g + (int64_t)kk * 512 + 16 * r) = v;
+    }
+    __syncthreads();
   }
 }
 
@@ -340,8 +395,21 @@ extern "C" moesq_status moesq_quant_act_routed(const uint16_t* x, int64_t T, int
   // thread per group: for small batches (decode) every slot's index loads in flight at
   // once, for large ones more warps
   if (K % 1024 == 0 && k <= 32) {
+    // scales as rows first once the codes written (S K/2 bytes) are half of L2 or more
+    const bool rows = T * k * (K / 2) >= ((int64_t)64 << 20);
     if (moesq_launch(k_quant_act_routed_warp, dim3((unsigned)g), dim3(128), 0, (cudaStream_t)stream, x, T, K, topk_ids,
-                     token_slot, k, expert_offsets, pad_offsets, E, g_in, codes, sf) != cudaSuccess)
+                     token_slot, k, expert_offsets, pad_offsets, E, g_in, codes, sf, rows) != cudaSuccess)
+      return MOESQ_ERR_CUDA;
+    if (!rows) return MOESQ_OK;
+    // the slabs: at most ceil((T k + 127 E) / 128) of them; a block per slab, up to 8 a SM
+    const size_t smem = (size_t)128 * (K / 32 + 4);
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(k_sf_rows_to_blocks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return MOESQ_ERR_CUDA;
+    int64_t slabs = (T * k + 127 * (int64_t)E) / 128 + 1;
+    if (slabs > 148 * 8) slabs = 148 * 8;
+    if (moesq_launch(k_sf_rows_to_blocks, dim3((unsigned)slabs), dim3(256), smem, (cudaStream_t)stream, sf, pad_offsets,
+                     E, K) != cudaSuccess)
       return MOESQ_ERR_CUDA;
     return MOESQ_OK;
   }

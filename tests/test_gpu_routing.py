@@ -156,13 +156,20 @@ def test_combine_golden_on_gpu(golden):
     assert out.float().cpu().numpy()[:, :2].tolist() == g["out"]
 
 
-@pytest.mark.parametrize("cfg_name,T", [("tiny", 64), ("qwen3_30b_a3b", 512), ("qwen3_5_397b_a17b", 16),
-                                        ("kimi_k2", 32)])
+ROUTED_CASES = [("tiny", 64, False), ("qwen3_30b_a3b", 512, False), ("qwen3_5_397b_a17b", 16, False),
+                ("kimi_k2", 32, False)]
+# batches whose codes reach 64 MiB: the scales are written as rows and rearranged into the
+# tensor-core blocks by a second kernel (Zipf routing: empty experts, ragged padding)
+ROUTED_ROWS_CASES = [("qwen3_30b_a3b", 8192, True), ("qwen3_5_397b_a17b", 4096, True)]
+
+
+@pytest.mark.parametrize("cfg_name,T,rows", ROUTED_CASES + ROUTED_ROWS_CASES)
 @pytest.mark.parametrize("shared_global", [False, True])
-def test_quant_act_routed_bit_exact(cfg_name, T, shared_global):
+def test_quant_act_routed_bit_exact(cfg_name, T, rows, shared_global):
     """Token-major quantisation (x read once per token) equals the per-slot oracle rule,
     with a global per expert and with one global shared by all experts (the kernel then
     reuses a group's codes across the token's slots)."""
+    assert (T * W.CONFIGS[cfg_name].k * W.CONFIGS[cfg_name].H // 2 >= 64 << 20) == rows
     cfg = W.CONFIGS[cfg_name]
     x = W.layer_input_bf16(cfg, T)
     ids, _ = W.routing(cfg, T)
