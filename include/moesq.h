@@ -254,7 +254,10 @@ moesq_status moesq_quant_act(const uint16_t* x, int64_t K, const int32_t* gather
  *   x          device bf16 [T, K];  topk_ids, token_slot  device i32 [T, k]
  *   expert_offsets, pad_offsets  device i32 [E+1] (moesq_permute);  g_in device f32 [E]
  *   codes, sf  padded operand outputs as for MOESQ_SF_KERNEL.
- * Same arithmetic as moesq_quant_act; ids outside [0, E) are treated as expert 0. */
+ * Same arithmetic as moesq_quant_act; ids outside [0, E) are treated as expert 0.
+ * One kernel launch, or two when K % 1024 == 0, k <= 32 and the codes written reach 64
+ * MiB (the scales are then written as rows and rearranged into the tensor-core blocks
+ * in place by a second kernel on the same stream); sf's padding rows hold no values. */
 moesq_status moesq_quant_act_routed(const uint16_t* x, int64_t T, int64_t K,
                                     const int32_t* topk_ids, const int32_t* token_slot, int32_t k,
                                     const int32_t* expert_offsets, const int32_t* pad_offsets,

@@ -32,7 +32,12 @@
 //   * on large batches runs the SwiGLU GEMM on wide items: two token tiles of an
 //     expert per item, one MMA of N <= 256 per K step, so the weight tile is read
 //     from shared memory once per 256 tokens (accumulators of consecutive items
-//     overlap in TMEM, see namespace wide).
+//     overlap in TMEM, see namespace wide);
+//   * on decode-sized batches takes each item's expert from a per-pair table built at
+//     set-up instead of searching the expert records item after item;
+//   * optionally fuses the weighted combine into the down GEMM's epilogue (a
+//     deterministic arrival count per token and output tile; slower than the
+//     separate combine, see moesq_grouped_gemm_down_combine).
 //
 // The same kernel, with a dense stage geometry (256-deep stages of four dense
 // kind::mxf4nvf4 MMAs, no metadata), is the dense comparison GEMM on decoded
@@ -82,7 +87,7 @@ constexpr int MAX_E = 1024;
 constexpr int ITEM_TAB = 128;  // work items per pair whose expert is looked up, not searched
 // Sixteen epilogue warps, four per sub-partition: the epilogue is bound by issue
 // and latency (TMEM loads, MUFU-heavy SiLU, lane exchanges), so it wants warps;
-// 18 warps leave 112 registers a thread.
+// the 18 warps are allocated as 20, which leaves 96 registers a thread.
 constexpr int EPI_WARPS = 16;
 constexpr int EPI_THREADS = 32 * EPI_WARPS;
 constexpr int THREADS = 64 + EPI_THREADS;  // producer warp, MMA warp, epilogue warps
@@ -154,12 +159,12 @@ struct Smem {
   // {end of its token tiles (prefix sum), first routed slot, first padded row,
   // routed-slot count}
   int4 rec[MAX_E];
-  float2 ag[MAX_E];
+  float2 ag[MAX_E];  // {g_act[e] * alpha_w[e] (the accumulator's scale), global scale of the requantised output}
   // the expert of each of this pair's work items when the pair has at most ITEM_TAB of
   // them (decode-sized batches, where every item jumps over several experts), found at
   // set-up by the prefix-sum warp; n_tab = 0: the roles walk (see TileWalk)
   uint16_t item_e[ITEM_TAB];
-  int n_tab;  // {g_act[e] * alpha_w[e] (the accumulator's scale), global scale of the requantised output}
+  int n_tab;
 };
 
 template <bool DENSE>
@@ -218,10 +223,11 @@ struct TileWalk {
   }
 };
 
-// The current item of `w`.  Empty experts end their tiles where they start; when
-// the next expert does not hold tile q either, a binary search over the tile-end
-// prefix sums finds the first expert that does, so a walk over thousands of empty
-// experts (decode batches of a layer with many experts) costs log2(E) loads, not E.
+// The current item of `w`: its expert from the set-up table when the pair has one
+// (decode-sized batches), else by the walk.  Empty experts end their tiles where they
+// start; when the next expert does not hold tile q either, a binary search over the
+// tile-end prefix sums finds the first expert that does, so a walk over thousands of
+// empty experts costs log2(E) loads, not E.
 template <int NT = 1>
 __device__ __forceinline__ Tile decode_tile(const Smem& s, TileWalk& w, int E) {
   if (NT == 1 && w.j < w.ntab) {  // the same for every item of the pair: table or walk
