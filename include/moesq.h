@@ -354,6 +354,17 @@ moesq_status moesq_grouped_gemm_down_combine(const moesq_linear* W, const uint8_
                                              int32_t k, uint16_t* y, uint16_t* out, int32_t* arrivals,
                                              int32_t* d_status, moesq_stream_t stream);
 
+/* Measured rate of the sparse block-scaled FP4 tensor-core MMA (the roofline
+ * denominator of the grouped GEMMs, with 8 x the measured bf16 GEMM rate as a floor):
+ * every CTA pair of the device issues `iters` x 4 tcgen05.mma.sp (cta_group::2,
+ * kind::mxf4nvf4, M = 256, dense K = 128, N = n) back to back on operands already in
+ * shared memory and TMEM, after one untimed launch.  Writes dense-equivalent TFLOP/s
+ * (2 M N K per MMA) to *tflops.  Synchronises the stream (a measurement call, not part
+ * of the hot path); a bounded wait that gives up raises MOESQ_DFLAG_TIMEOUT in d_status
+ * (may be NULL).  iters >= 1, 16 <= n <= 256, n % 16 == 0. */
+moesq_status moesq_measure_sparse_mma_peak(int32_t iters, int32_t n, double* tflops, int32_t* d_status,
+                                           moesq_stream_t stream);
+
 /* Work-item width of the sparse SwiGLU gate_up GEMM (the pages have no counterpart).
  * A work item is one weight-tile pair times one 128-token tile, or, on large batches,
  * two 128-token tiles of one expert computed by single MMAs of N <= 256 ("wide" items:

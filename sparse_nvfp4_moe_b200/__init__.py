@@ -8,7 +8,8 @@ shared library is missing.
 """
 from ._lib import (Linear, MoeLayer, MoesqError, declared_symbols, lib, moesq_decode,  # noqa: F401
                    moesq_encode, moesq_gather_act, moesq_gemm_launch_pairs, moesq_set_gemm_pair_limit,
-                   moesq_gemm_tiles_per_item, moesq_set_gemm_tiles_per_item, moesq_grouped_gemm, moesq_grouped_gemm_dense,
+                   moesq_gemm_tiles_per_item, moesq_set_gemm_tiles_per_item, moesq_measure_sparse_mma_peak,
+                   moesq_grouped_gemm, moesq_grouped_gemm_dense,
                    moesq_grouped_gemm_down_combine, moesq_moe_forward,
                    moesq_moe_forward_host, moesq_selftest_wait_timeout, moesq_sf_expand_block16,
                    moesq_permute, moesq_permute_noalloc, moesq_quant_act, moesq_quant_act_routed, moesq_quant_weight, moesq_repack_meta,

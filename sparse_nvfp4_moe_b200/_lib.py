@@ -68,6 +68,7 @@ _SIGS = {
     "moesq_set_gemm_pair_limit": (ctypes.c_int, [c_i32]),
     "moesq_gemm_launch_pairs": (ctypes.c_int, [c_i32, c_i32, ctypes.POINTER(c_i32)]),
     "moesq_set_gemm_tiles_per_item": (ctypes.c_int, [c_i32]),
+    "moesq_measure_sparse_mma_peak": (ctypes.c_int, [c_i32, c_i32, ctypes.POINTER(ctypes.c_double), c_vp, c_vp]),
     "moesq_gemm_tiles_per_item": (ctypes.c_int, [c_i32, c_i32, c_i64, c_i64, c_i64, ctypes.POINTER(c_i32)]),
     "moesq_selftest_wait_timeout": (ctypes.c_int, [c_vp, c_i64, c_vp, c_vp]),
     "moesq_gather_act": (ctypes.c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp]),
@@ -289,6 +290,14 @@ def moesq_gemm_launch_pairs(dense, epilogue):
     n = c_i32(0)
     _check("moesq_gemm_launch_pairs", lib().moesq_gemm_launch_pairs(dense, epilogue, ctypes.byref(n)))
     return n.value
+
+
+def moesq_measure_sparse_mma_peak(iters=2000, n=256, d_status=None, stream=None):
+    """Dense-equivalent TFLOP/s of back-to-back sparse FP4 MMAs on every CTA pair (synchronises)."""
+    v = ctypes.c_double(0.0)
+    _check("moesq_measure_sparse_mma_peak",
+           lib().moesq_measure_sparse_mma_peak(iters, n, ctypes.byref(v), _p(d_status), _stream(stream)))
+    return v.value
 
 
 def moesq_set_gemm_tiles_per_item(tiles):
