@@ -84,3 +84,39 @@ def test_ep_launch_count():
     assert bench.ep_launches(1, 8, 0) == 1 + 1 + 1
     assert bench.ep_launches(1, 8, 3) == 1 + 1 + (1 + 1 + 2 + 1) + 1
     assert bench.ep_launches(65536, 8, 524288) == 3 + 1 + (3 + 1 + 2 + 1) + 1
+
+
+def test_step_launch_count():
+    """Kernels one single-GPU step launches: permute (1 kernel up to 1024 slots, else 3),
+    the routed quant (plus the in-place scale rearrangement once its codes reach 64 MiB,
+    when H % 1024 == 0 and k <= 32), the two GEMMs and the combine."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as W
+    C = W.CONFIGS
+    assert bench.kernels_per_step(C["qwen3_235b_a22b"], 65536) == 3 + 2 + 3   # 1 GiB of codes
+    assert bench.kernels_per_step(C["qwen3_30b_a3b"], 16384) == 3 + 2 + 3    # 128 MiB
+    assert bench.kernels_per_step(C["qwen3_30b_a3b"], 4096) == 3 + 1 + 3     # 32 MiB
+    assert bench.kernels_per_step(C["qwen3_30b_a3b"], 64) == 1 + 1 + 3      # 512 slots
+    assert bench.kernels_per_step(C["kimi_k2"], 1) == 1 + 1 + 3
+    assert bench.kernels_per_step(C["tiny"], 64) == 1 + 1 + 3                # H = 256
+
+
+def test_fp4_peak_is_the_larger_of_microbenchmark_and_eight_bf16():
+    """The GEMM roofline's sparse FP4 peak: max(measured sparse-MMA rate, 8 x bf16 burst);
+    the sustained peak scales the microbenchmark by the bf16 sustained / burst ratio."""
+    sys.path.insert(0, ROOT)
+    import bench
+    peaks = dict(hbm_gbs=6542.4, bf16_tflops=1671.8, bf16_tflops_sustained=1410.6, source="measured")
+    assert bench.fp4_peaks(peaks) == pytest.approx((8 * 1671.8, 8 * 1410.6))
+    peaks["fp4sp_micro"] = 17764.0
+    burst, sust = bench.fp4_peaks(peaks)
+    assert burst == pytest.approx(17764.0)
+    assert sust == pytest.approx(17764.0 * 1410.6 / 1671.8)
+    peaks["fp4sp_micro"] = 9000.0       # a slower measurement never lowers the peak
+    assert bench.fp4_peaks(peaks)[0] == pytest.approx(8 * 1671.8)
+    # a row is tensor-bound when its FLOPs at the peak take longer than its bytes at HBM
+    bound, t, cls, target = bench.classify(1e15, 1e9, 5e8, peaks)
+    assert bound == "tensor" and cls == "prefill-sized" and target == 0.60
+    bound, t, cls, target = bench.classify(1e12, 1e9, 9e8, peaks)
+    assert bound == "hbm" and cls == "decode-sized" and target == 0.70
